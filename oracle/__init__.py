@@ -1,0 +1,110 @@
+"""GDPA oracle (plain fp64 C, OpenMP) and its ctypes loader.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+benchmark's CPU-baseline leg import this package.  The product library in
+``recsys_context_personalised_b200`` never imports it, and the oracle shares
+no code with the CUDA path.  The arithmetic lives in ``gdpa_oracle.c``; this
+file only compiles it, marshals arrays and converts results.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdpa_oracle.c")
+_LIB = os.path.join(_HERE, "libgdpa_oracle.so")
+_lib = None
+
+PHI = {"identity": 0, "silu": 1, "softmax": 2}
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
+    """Compile the oracle with gcc (IEEE double, no fast-math)."""
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+        return out
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-fno-fast-math",
+           "-ffp-contract=off", "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def load(path: str = None):
+    global _lib
+    if path is None and _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build() if path is None else path)
+    i32, i64p, fp, dp, f64 = (ctypes.c_int, ctypes.POINTER(ctypes.c_int64),
+                              ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_double),
+                              ctypes.c_double)
+    lib.gdpa_oracle_fwd.argtypes = [i32, i32, i32, i32, i64p, fp, fp, fp, i32, f64, dp, dp, i32]
+    lib.gdpa_oracle_fwd.restype = i32
+    lib.gdpa_oracle_bwd.argtypes = [i32, i32, i32, i32, i64p, fp, fp, fp, fp, i32, f64,
+                                    dp, dp, dp, i32]
+    lib.gdpa_oracle_bwd.restype = i32
+    lib.gdpa_oracle_max_threads.restype = i32
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _f32(x) -> np.ndarray:
+    """Exact float32 copy of a bf16/fp32 torch tensor or numpy array."""
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().float().numpy()
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def _ptr(a, ct):
+    return a.ctypes.data_as(ctypes.POINTER(ct))
+
+
+def _phi(phi) -> int:
+    return PHI[phi] if isinstance(phi, str) else int(phi)
+
+
+def max_threads(lib=None) -> int:
+    return (lib or load()).gdpa_oracle_max_threads()
+
+
+def fwd(q, k, v, offsets, phi, scale, nthreads: int = 0, lib=None):
+    """O [T,h,dh] float64 and LSE [h,T] float64 (NaN-free only for softmax)."""
+    lib = lib or load()
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    off = np.ascontiguousarray(offsets, dtype=np.int64)
+    B, h, m, dh = k.shape
+    T = int(off[-1])
+    assert q.shape == (T, h, dh) and v.shape == k.shape and off.shape == (B + 1,)
+    o = np.zeros((T, h, dh), dtype=np.float64)
+    lse = np.zeros((h, T), dtype=np.float64)
+    rc = lib.gdpa_oracle_fwd(B, h, dh, m, _ptr(off, ctypes.c_int64), _ptr(q, ctypes.c_float),
+                             _ptr(k, ctypes.c_float), _ptr(v, ctypes.c_float), _phi(phi),
+                             float(scale), _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double),
+                             int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"gdpa_oracle_fwd failed with code {rc}")
+    return o, lse
+
+
+def bwd(q, k, v, dout, offsets, phi, scale, nthreads: int = 0, lib=None):
+    """(dQ [T,h,dh], dK [B,h,m,dh], dV [B,h,m,dh]) in float64."""
+    lib = lib or load()
+    q, k, v, g = _f32(q), _f32(k), _f32(v), _f32(dout)
+    off = np.ascontiguousarray(offsets, dtype=np.int64)
+    B, h, m, dh = k.shape
+    T = int(off[-1])
+    assert q.shape == (T, h, dh) and g.shape == q.shape and v.shape == k.shape
+    dq = np.zeros((T, h, dh), dtype=np.float64)
+    dk = np.zeros((B, h, m, dh), dtype=np.float64)
+    dv = np.zeros((B, h, m, dh), dtype=np.float64)
+    rc = lib.gdpa_oracle_bwd(B, h, dh, m, _ptr(off, ctypes.c_int64), _ptr(q, ctypes.c_float),
+                             _ptr(k, ctypes.c_float), _ptr(v, ctypes.c_float),
+                             _ptr(g, ctypes.c_float), _phi(phi), float(scale),
+                             _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double),
+                             _ptr(dv, ctypes.c_double), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"gdpa_oracle_bwd failed with code {rc}")
+    return dq, dk, dv

@@ -1,0 +1,235 @@
+/*
+ * GDPA oracle: plain, slow, fp64 CPU implementation of Generalized Dot-Product
+ * Attention.  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the
+ * benchmark's CPU-baseline leg call it; the product library never does, and
+ * this file shares no code, header or constant with it.
+ *
+ * What it computes.  The Kunlun summary (gist.science, "Resumen Tecnico:
+ * Kunlun", section 2.2, GDPA bullet) recasts the Personalized FFN as a
+ * multi-head attention operator whose queries are the sequence tokens and
+ * whose keys and values are weights derived from the non-sequential context;
+ * the RecSysChannel review ("Kunlun ... [2/2]", items 1 and 2) adds that K and
+ * V come from the context features and the event sequence is turned into Q.
+ * Neither page prints a formula.  The plainest reading, which this oracle
+ * writes out, is, for every sample b and head j, with
+ *   Q^ = Q[off[b]:off[b+1], j, :]   (n_b x dh),
+ *   K^ = K[b, j], V^ = V[b, j]       (m x dh):
+ *
+ *   S  = s * Q^ K^T                  (n_b x m)
+ *   P  = phi(S)                      phi in {identity, SiLU, row softmax}
+ *   O  = P V^                        (n_b x dh)
+ *   LSE_i = M_i + ln sum_k exp(S_ik - M_i),  M_i = max_k S_ik  (softmax)
+ *
+ * and its gradient for an upstream dO:
+ *
+ *   dV = P^T dO^,  dP = dO^ V^T,
+ *   dS = dP                                   (identity)
+ *      = dP * sig(S) (1 + S (1 - sig(S)))     (SiLU, sig = logistic)
+ *      = P * (dP - D),  D_i = sum_k P_ik dP_ik (softmax)
+ *   dQ^ = s dS K^,  dK^ = s dS^T Q^.
+ *
+ * Every dot product is a plain loop accumulated in double.  Inputs are float
+ * arrays holding the exact values of the (bf16 or fp32) inputs.  Units
+ * (b, j) are independent and run under OpenMP; inside a unit nothing is
+ * blocked, fused or reordered.
+ *
+ * Layouts: q, o, dout, dq: [T, h, dh];  k, v, dk, dv: [B, h, m, dh];
+ * offsets: int64 [B+1];  lse: [h, T].  phi: 0 identity, 1 SiLU, 2 softmax.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define PHI_IDENTITY 0
+#define PHI_SILU 1
+#define PHI_SOFTMAX 2
+
+static double logistic(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/* S = s Q^ K^T for one unit; S is n x m, row-major. */
+static void logits(int n, int m, int dh, int h, const float* qb, const float* kb,
+                   double scale, double* S) {
+  for (int i = 0; i < n; ++i) {
+    const float* qi = qb + (size_t)i * h * dh;
+    for (int k = 0; k < m; ++k) {
+      const float* kk = kb + (size_t)k * dh;
+      double acc = 0.0;
+      for (int d = 0; d < dh; ++d) acc += (double)qi[d] * (double)kk[d];
+      S[(size_t)i * m + k] = scale * acc;
+    }
+  }
+}
+
+/* P = phi(S) in place of a separate array; for softmax also the row LSE. */
+static void activation(int n, int m, int phi, const double* S, double* P, double* lse_rows) {
+  for (int i = 0; i < n; ++i) {
+    const double* si = S + (size_t)i * m;
+    double* pi = P + (size_t)i * m;
+    if (phi == PHI_IDENTITY) {
+      for (int k = 0; k < m; ++k) pi[k] = si[k];
+    } else if (phi == PHI_SILU) {
+      for (int k = 0; k < m; ++k) pi[k] = si[k] / (1.0 + exp(-si[k]));
+    } else {
+      double mx = -INFINITY;
+      for (int k = 0; k < m; ++k) mx = si[k] > mx ? si[k] : mx;
+      double sum = 0.0;
+      for (int k = 0; k < m; ++k) sum += exp(si[k] - mx);
+      for (int k = 0; k < m; ++k) pi[k] = exp(si[k] - mx) / sum;
+      if (lse_rows) lse_rows[i] = mx + log(sum);
+    }
+  }
+}
+
+static int valid_args(int B, int h, int dh, int m, const int64_t* offsets) {
+  if (B < 0 || h <= 0 || dh <= 0 || m <= 0 || !offsets) return 0;
+  if (offsets[0] != 0) return 0;
+  for (int b = 0; b < B; ++b)
+    if (offsets[b + 1] < offsets[b]) return 0;
+  return 1;
+}
+
+/* Forward.  o: [T,h,dh] (required), lse: [h,T] (softmax only; may be NULL).
+ * Returns 0 on success, -1 on bad arguments, -2 if memory ran out. */
+int gdpa_oracle_fwd(int B, int h, int dh, int m, const int64_t* offsets,
+                    const float* q, const float* k, const float* v, int phi,
+                    double scale, double* o, double* lse, int nthreads) {
+  if (!valid_args(B, h, dh, m, offsets) || phi < 0 || phi > 2 || !q || !k || !v || !o)
+    return -1;
+  const int64_t T = offsets[B];
+  int failed = 0;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : failed)
+  for (long u = 0; u < (long)B * h; ++u) {
+    const int b = (int)(u / h), j = (int)(u % h);
+    const int64_t t0 = offsets[b];
+    const int n = (int)(offsets[b + 1] - t0);
+    if (n == 0) continue;
+    double* S = (double*)malloc(sizeof(double) * (size_t)n * m);
+    double* P = (double*)malloc(sizeof(double) * (size_t)n * m);
+    double* L = (double*)malloc(sizeof(double) * (size_t)n);
+    if (!S || !P || !L) {
+      free(S); free(P); free(L);
+      failed |= 1;
+      continue;
+    }
+    const float* qb = q + ((size_t)t0 * h + j) * dh;
+    const float* kb = k + ((size_t)b * h + j) * (size_t)m * dh;
+    const float* vb = v + ((size_t)b * h + j) * (size_t)m * dh;
+    logits(n, m, dh, h, qb, kb, scale, S);
+    activation(n, m, phi, S, P, L);
+    for (int i = 0; i < n; ++i) {
+      double* oi = o + ((size_t)(t0 + i) * h + j) * dh;
+      for (int d = 0; d < dh; ++d) {
+        double acc = 0.0;
+        for (int kk = 0; kk < m; ++kk) acc += P[(size_t)i * m + kk] * (double)vb[(size_t)kk * dh + d];
+        oi[d] = acc;
+      }
+      if (lse && phi == PHI_SOFTMAX) lse[(size_t)j * T + t0 + i] = L[i];
+    }
+    free(S); free(P); free(L);
+  }
+  return failed ? -2 : 0;
+}
+
+/* Backward.  dout: [T,h,dh]; dq: [T,h,dh]; dk, dv: [B,h,m,dh] (all required).
+ * P is recomputed from its definition; no forward state is taken. */
+int gdpa_oracle_bwd(int B, int h, int dh, int m, const int64_t* offsets,
+                    const float* q, const float* k, const float* v, const float* dout,
+                    int phi, double scale, double* dq, double* dk, double* dv,
+                    int nthreads) {
+  if (!valid_args(B, h, dh, m, offsets) || phi < 0 || phi > 2 || !q || !k || !v ||
+      !dout || !dq || !dk || !dv)
+    return -1;
+  int failed = 0;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : failed)
+  for (long u = 0; u < (long)B * h; ++u) {
+    const int b = (int)(u / h), j = (int)(u % h);
+    const int64_t t0 = offsets[b];
+    const int n = (int)(offsets[b + 1] - t0);
+    const float* qb = q + ((size_t)t0 * h + j) * dh;
+    const float* kb = k + ((size_t)b * h + j) * (size_t)m * dh;
+    const float* vb = v + ((size_t)b * h + j) * (size_t)m * dh;
+    const float* gb = dout + ((size_t)t0 * h + j) * dh;
+    double* dkb = dk + ((size_t)b * h + j) * (size_t)m * dh;
+    double* dvb = dv + ((size_t)b * h + j) * (size_t)m * dh;
+    memset(dkb, 0, sizeof(double) * (size_t)m * dh);
+    memset(dvb, 0, sizeof(double) * (size_t)m * dh);
+    if (n == 0) continue;
+    double* S = (double*)malloc(sizeof(double) * (size_t)n * m);
+    double* P = (double*)malloc(sizeof(double) * (size_t)n * m);
+    double* dP = (double*)malloc(sizeof(double) * (size_t)n * m);
+    if (!S || !P || !dP) {
+      free(S); free(P); free(dP);
+      failed |= 1;
+      continue;
+    }
+    logits(n, m, dh, h, qb, kb, scale, S);
+    activation(n, m, phi, S, P, NULL);
+    /* dP = dO^ V^T */
+    for (int i = 0; i < n; ++i)
+      for (int kk = 0; kk < m; ++kk) {
+        double acc = 0.0;
+        for (int d = 0; d < dh; ++d)
+          acc += (double)gb[(size_t)i * h * dh + d] * (double)vb[(size_t)kk * dh + d];
+        dP[(size_t)i * m + kk] = acc;
+      }
+    /* dV = P^T dO^ */
+    for (int kk = 0; kk < m; ++kk)
+      for (int d = 0; d < dh; ++d) {
+        double acc = 0.0;
+        for (int i = 0; i < n; ++i) acc += P[(size_t)i * m + kk] * (double)gb[(size_t)i * h * dh + d];
+        dvb[(size_t)kk * dh + d] = acc;
+      }
+    /* dS, overwriting dP */
+    for (int i = 0; i < n; ++i) {
+      double* dpi = dP + (size_t)i * m;
+      const double* si = S + (size_t)i * m;
+      const double* pi = P + (size_t)i * m;
+      if (phi == PHI_SILU) {
+        for (int kk = 0; kk < m; ++kk) {
+          const double sg = logistic(si[kk]);
+          dpi[kk] = dpi[kk] * sg * (1.0 + si[kk] * (1.0 - sg));
+        }
+      } else if (phi == PHI_SOFTMAX) {
+        double D = 0.0;
+        for (int kk = 0; kk < m; ++kk) D += pi[kk] * dpi[kk];
+        for (int kk = 0; kk < m; ++kk) dpi[kk] = pi[kk] * (dpi[kk] - D);
+      }
+    }
+    /* dQ^ = s dS K^ */
+    for (int i = 0; i < n; ++i) {
+      double* dqi = dq + ((size_t)(t0 + i) * h + j) * dh;
+      for (int d = 0; d < dh; ++d) {
+        double acc = 0.0;
+        for (int kk = 0; kk < m; ++kk) acc += dP[(size_t)i * m + kk] * (double)kb[(size_t)kk * dh + d];
+        dqi[d] = scale * acc;
+      }
+    }
+    /* dK^ = s dS^T Q^ */
+    for (int kk = 0; kk < m; ++kk)
+      for (int d = 0; d < dh; ++d) {
+        double acc = 0.0;
+        for (int i = 0; i < n; ++i) acc += dP[(size_t)i * m + kk] * (double)qb[(size_t)i * h * dh + d];
+        dkb[(size_t)kk * dh + d] = scale * acc;
+      }
+    free(S); free(P); free(dP);
+  }
+  return failed ? -2 : 0;
+}
+
+int gdpa_oracle_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
