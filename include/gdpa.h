@@ -1,0 +1,166 @@
+/*
+ * gdpa.h - C ABI of the B200 (sm_100a) GDPA library, libgdpa.so.
+ *
+ * GDPA (Generalized Dot-Product Attention) is Kunlun's Personalized FFN
+ * recast as a multi-head attention operator.  The Kunlun technical summary
+ * (gist.science/es/paper/2602.10016, section 2.2 "Optimizaciones de Modulos
+ * de Bajo Nivel", GDPA bullet) states that the sequence tokens act as the
+ * queries, that weights derived from the non-sequential context act as the
+ * keys and values, and that the transformation is fused into one
+ * FlashAttention-like kernel instead of separate memory-bound matmuls.  The
+ * RecSysChannel review ("Kunlun: Establishing Scaling Laws for Massive-Scale
+ * Recommendation Systems [2/2]", items 1 and 2) adds that K and V are
+ * obtained from the context features and the event sequence is turned into
+ * Q.  Neither page prints the formula; this library computes, for every
+ * sample b and head j (token rows t in [offsets[b], offsets[b+1])):
+ *
+ *     S = scale * Q_bj K_bj^T,    P = phi(S),    O_bj = P V_bj
+ *
+ * with phi = identity, SiLU (x * logistic(x)) or a row softmax, and its
+ * gradient.  Heads and samples are independent; there is no normalisation
+ * for the elementwise phi, no bias and no head mixing.
+ *
+ * Layouts (row-major, contiguous, every base pointer 16-byte aligned):
+ *   q, o, dout, dq : [T, h, dh]      jagged tokens, T = offsets[B]
+ *   k, v, dk, dv   : [B, h, m, dh]   one context key/value set per sample, head
+ *   offsets        : int32 [B + 1]   device memory, offsets[0] = 0,
+ *                                     non-decreasing, offsets[B] = T
+ *   lse            : fp32 [h, T]     natural-log row log-sum-exp (softmax)
+ * Element type of q, k, v, o, dout, dq, dk, dv: fp32 or bf16 (problem dtype).
+ *
+ * Ownership: the caller allocates every buffer, including the workspace whose
+ * size the *_workspace_size calls report.  The library allocates no device
+ * memory and keeps only small per-device host caches (launch attributes).
+ *
+ * Asynchrony: gdpa_fwd and gdpa_bwd only enqueue work on `stream` (a
+ * cudaStream_t passed as void*) and never synchronise.  All pointers passed to
+ * them are device pointers unless stated otherwise.
+ *
+ * Errors: argument errors are detected on the host and returned before any
+ * launch (GDPA_ERR_INVALID_ARG / GDPA_ERR_UNSUPPORTED).  A failed launch
+ * returns GDPA_ERR_CUDA.  Inconsistent device offsets (decreasing, a length
+ * above max_n, offsets[B] != T) and bounded-wait time-outs inside a kernel are
+ * detected on the device: the kernels then skip the bad work, and the code is
+ * left in the workspace's status word, which gdpa_workspace_status() reads.
+ */
+#ifndef GDPA_H_
+#define GDPA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDPA_API __attribute__((visibility("default")))
+#else
+#define GDPA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDPA_PHI_IDENTITY = 0,
+  GDPA_PHI_SILU = 1,
+  GDPA_PHI_SOFTMAX = 2
+} gdpa_phi_t;
+
+typedef enum {
+  GDPA_DTYPE_F32 = 0,   /* fp32 in / fp32 accumulate / fp32 out (SIMT kernels) */
+  GDPA_DTYPE_BF16 = 1   /* bf16 in / fp32 accumulate / bf16 out (tcgen05 kernels) */
+} gdpa_dtype_t;
+
+typedef enum {
+  GDPA_OK = 0,
+  GDPA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad offsets */
+  GDPA_ERR_UNSUPPORTED = 2,   /* valid but unsupported (e.g. dh not in {32,64,128}) */
+  GDPA_ERR_CUDA = 3,          /* a CUDA runtime/driver call or a launch failed */
+  GDPA_ERR_TIMEOUT = 4,       /* a bounded wait inside a kernel gave up */
+  GDPA_ERR_WORKSPACE = 5      /* workspace null, misaligned or too small */
+} gdpa_status_t;
+
+/* Problem description (host memory, read during the call only). */
+typedef struct {
+  int32_t B;             /* samples, >= 1 */
+  int32_t h;             /* heads, >= 1 */
+  int32_t dh;            /* head dim: 32, 64 or 128 */
+  int32_t m;             /* context keys/values per sample and head, >= 1 */
+  int32_t max_n;         /* upper bound on every n_b = offsets[b+1]-offsets[b], >= 0 */
+  int32_t dtype;         /* gdpa_dtype_t */
+  int64_t total_tokens;  /* T = offsets[B], 0 <= T < 2^31 */
+  int32_t phi;           /* gdpa_phi_t */
+  float scale;           /* s in S = s Q K^T */
+} gdpa_problem_t;
+
+/* Workspace bytes gdpa_fwd needs for `p` (written to *bytes). Host only. */
+GDPA_API gdpa_status_t gdpa_fwd_workspace_size(const gdpa_problem_t* p, size_t* bytes);
+
+/* Workspace bytes gdpa_bwd needs for `p` (written to *bytes). Host only. */
+GDPA_API gdpa_status_t gdpa_bwd_workspace_size(const gdpa_problem_t* p, size_t* bytes);
+
+/*
+ * Forward: o = phi(scale * q k^T) v per (sample, head).
+ *   q [T,h,dh], k/v [B,h,m,dh], offsets int32 [B+1]: inputs (device).
+ *   o [T,h,dh]: output (device), every valid row written.
+ *   lse fp32 [h,T]: output for phi = softmax (needed by gdpa_bwd); may be NULL
+ *     for softmax when no backward follows; ignored for the other phi.
+ *   workspace: device, >= gdpa_fwd_workspace_size bytes, 256-byte aligned.
+ *   stream: cudaStream_t (void*), may be NULL for the legacy default stream.
+ */
+GDPA_API gdpa_status_t gdpa_fwd(const gdpa_problem_t* p, const void* q, const int32_t* offsets,
+                       const void* k, const void* v, void* o, float* lse,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward for an upstream gradient dout of o.
+ *   q, k, v, offsets: as in gdpa_fwd.  o and lse: gdpa_fwd's outputs (read for
+ *   phi = softmax only; may be NULL otherwise).  dout [T,h,dh]: input.
+ *   dq [T,h,dh], dk/dv [B,h,m,dh]: outputs, every element written (dk, dv of a
+ *   sample with no tokens are zero).
+ *   workspace: device, >= gdpa_bwd_workspace_size bytes, 256-byte aligned.
+ */
+GDPA_API gdpa_status_t gdpa_bwd(const gdpa_problem_t* p, const void* q, const int32_t* offsets,
+                       const void* k, const void* v, const void* o, const float* lse,
+                       const void* dout, void* dq, void* dk, void* dv,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Device-detected status of the last gdpa_fwd/gdpa_bwd that used `workspace`
+ * (GDPA_OK, GDPA_ERR_INVALID_ARG for inconsistent offsets, GDPA_ERR_TIMEOUT).
+ * Synchronises `stream`; writes the code to *status (host).
+ */
+GDPA_API gdpa_status_t gdpa_workspace_status(const void* workspace, void* stream, int32_t* status);
+
+/* Static, human-readable name of a status code. */
+GDPA_API const char* gdpa_status_string(gdpa_status_t s);
+
+/* Number of kernels the last gdpa_fwd / gdpa_bwd call on this thread launched. */
+GDPA_API int32_t gdpa_last_launch_count(void);
+
+/*
+ * Per-kernel timing (host-thread local; for benchmarks, not for production).
+ * While enabled, each kernel launch of gdpa_fwd / gdpa_bwd on this host thread
+ * is bracketed by two CUDA events recorded on the call's stream.  Enabling
+ * (or disabling) discards any unread records.  Returns GDPA_ERR_CUDA if an
+ * event could not be created.
+ */
+GDPA_API gdpa_status_t gdpa_timing_enable(int32_t enable);
+
+typedef struct {
+  char name[48];       /* kernel name, NUL-terminated */
+  int32_t launches;    /* launches recorded since gdpa_timing_enable(1) */
+  float total_ms;      /* sum of their event-measured durations */
+} gdpa_kernel_time_t;
+
+/*
+ * Waits for the recorded events, then writes up to `cap` per-kernel sums to
+ * `out` (host) and returns how many distinct kernels were recorded (which may
+ * exceed cap), or -1 on a CUDA error.  The records are cleared.
+ */
+GDPA_API int32_t gdpa_timing_read(gdpa_kernel_time_t* out, int32_t cap);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDPA_H_ */

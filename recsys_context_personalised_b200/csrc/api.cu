@@ -1,0 +1,274 @@
+// C ABI entry points of libgdpa.so: argument validation, workspace layout and
+// kernel dispatch.  Every step of the operator runs in this library's kernels.
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+#include <vector>
+
+#include "gdpa_internal.cuh"
+
+namespace gdpa {
+
+static thread_local int g_launches = 0;
+
+struct TimingRec {
+  const char* name;
+  cudaEvent_t start, stop;
+};
+static thread_local bool g_timing = false;
+static thread_local std::vector<TimingRec> g_recs;
+
+KernelScope::KernelScope(const char* name, cudaStream_t s) : rec(-1), st(s) {
+  ++g_launches;
+  if (!g_timing) return;
+  TimingRec r{name, nullptr, nullptr};
+  if (cudaEventCreate(&r.start) != cudaSuccess || cudaEventCreate(&r.stop) != cudaSuccess) return;
+  cudaEventRecord(r.start, st);
+  g_recs.push_back(r);
+  rec = (int)g_recs.size() - 1;
+}
+
+KernelScope::~KernelScope() {
+  if (rec >= 0) cudaEventRecord(g_recs[rec].stop, st);
+}
+
+static void clear_records() {
+  for (auto& r : g_recs) {
+    if (r.start) cudaEventDestroy(r.start);
+    if (r.stop) cudaEventDestroy(r.stop);
+  }
+  g_recs.clear();
+}
+
+// bf16 problems run on the tcgen05 kernels when they are compiled in.
+cudaError_t launch_sm100_fwd(const gdpa_problem_t& p, const void* q, const void* k,
+                             const void* v, void* o, float* lse, WsHeader* ws,
+                             const Tile* tiles, cudaStream_t st);
+cudaError_t launch_sm100_bwd(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
+                             const void* k, const void* v, const float* lse, const float* dsum,
+                             const void* dout, void* dq, void* dk, void* dv, float* dq_acc,
+                             WsHeader* ws, const Tile* tiles, cudaStream_t st);
+bool sm100_fwd_available();
+bool sm100_bwd_available();
+
+namespace {
+
+struct FwdLayout {
+  size_t tiles_off, total;
+  int bm;
+};
+struct BwdLayout {
+  size_t tiles_off, dsum_off, dqacc_off, total;
+  int bm;
+};
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+gdpa_status_t check_problem(const gdpa_problem_t* p) {
+  if (!p) return GDPA_ERR_INVALID_ARG;
+  if (p->B < 1 || p->h < 1 || p->m < 1 || p->max_n < 0 || p->total_tokens < 0 ||
+      p->total_tokens >= (int64_t)1 << 31)
+    return GDPA_ERR_INVALID_ARG;
+  if ((int64_t)p->max_n * p->B < p->total_tokens) return GDPA_ERR_INVALID_ARG;
+  if (p->phi < GDPA_PHI_IDENTITY || p->phi > GDPA_PHI_SOFTMAX) return GDPA_ERR_INVALID_ARG;
+  if (p->dtype != GDPA_DTYPE_F32 && p->dtype != GDPA_DTYPE_BF16) return GDPA_ERR_INVALID_ARG;
+  if (!(p->scale == p->scale) || p->scale > 3.0e38f || p->scale < -3.0e38f)
+    return GDPA_ERR_INVALID_ARG;
+  if (p->dh != 32 && p->dh != 64 && p->dh != 128) return GDPA_ERR_UNSUPPORTED;
+  // element counts must fit the kernels' 64-bit index math; K/V rows < 2^31
+  if ((int64_t)p->B * p->h * p->m >= (int64_t)1 << 31) return GDPA_ERR_UNSUPPORTED;
+  if ((int64_t)p->B * p->h >= (int64_t)1 << 24) return GDPA_ERR_UNSUPPORTED;
+  return GDPA_OK;
+}
+
+int fwd_bm(const gdpa_problem_t& p) {
+  return (p.dtype == GDPA_DTYPE_BF16 && sm100_fwd_available()) ? kMmaBM : kSimtBM;
+}
+int bwd_bm(const gdpa_problem_t& p) {
+  return (p.dtype == GDPA_DTYPE_BF16 && sm100_bwd_available()) ? kMmaBM : kSimtBM;
+}
+
+FwdLayout fwd_layout(const gdpa_problem_t& p) {
+  FwdLayout L;
+  L.bm = fwd_bm(p);
+  L.tiles_off = sizeof(WsHeader);
+  L.total = align_up(L.tiles_off + sizeof(Tile) * (size_t)tile_capacity(p, L.bm), 256);
+  return L;
+}
+
+BwdLayout bwd_layout(const gdpa_problem_t& p) {
+  BwdLayout L;
+  L.bm = bwd_bm(p);
+  L.tiles_off = sizeof(WsHeader);
+  L.dsum_off = align_up(L.tiles_off + sizeof(Tile) * (size_t)tile_capacity(p, L.bm), 256);
+  L.dqacc_off = align_up(L.dsum_off + sizeof(float) * (size_t)p.h * (size_t)p.total_tokens, 256);
+  size_t dq_bytes = 0;
+  if (L.bm == kMmaBM) dq_bytes = sizeof(float) * (size_t)p.total_tokens * p.h * p.dh;
+  L.total = align_up(L.dqacc_off + dq_bytes, 256);
+  return L;
+}
+
+gdpa_status_t check_ws(const void* ws, size_t have, size_t need) {
+  if (!ws || ((uintptr_t)ws & 255u) != 0 || have < need) return GDPA_ERR_WORKSPACE;
+  return GDPA_OK;
+}
+
+gdpa_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return GDPA_OK;
+  fprintf(stderr, "gdpa: CUDA error %d (%s)\n", (int)e, cudaGetErrorString(e));
+  return GDPA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace gdpa
+
+using namespace gdpa;
+
+extern "C" {
+
+gdpa_status_t gdpa_fwd_workspace_size(const gdpa_problem_t* p, size_t* bytes) {
+  gdpa_status_t s = check_problem(p);
+  if (s != GDPA_OK) return s;
+  if (!bytes) return GDPA_ERR_INVALID_ARG;
+  *bytes = fwd_layout(*p).total;
+  return GDPA_OK;
+}
+
+gdpa_status_t gdpa_bwd_workspace_size(const gdpa_problem_t* p, size_t* bytes) {
+  gdpa_status_t s = check_problem(p);
+  if (s != GDPA_OK) return s;
+  if (!bytes) return GDPA_ERR_INVALID_ARG;
+  *bytes = bwd_layout(*p).total;
+  return GDPA_OK;
+}
+
+gdpa_status_t gdpa_fwd(const gdpa_problem_t* p, const void* q, const int32_t* offsets,
+                       const void* k, const void* v, void* o, float* lse, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  g_launches = 0;
+  gdpa_status_t s = check_problem(p);
+  if (s != GDPA_OK) return s;
+  if (!q || !offsets || !k || !v || !o) return GDPA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      ((uintptr_t)offsets & 3u) || ((uintptr_t)lse & 3u))
+    return GDPA_ERR_INVALID_ARG;
+  const FwdLayout L = fwd_layout(*p);
+  s = check_ws(workspace, workspace_bytes, L.total);
+  if (s != GDPA_OK) return s;
+  if (p->phi != GDPA_PHI_SOFTMAX) lse = nullptr;
+  cudaStream_t st = (cudaStream_t)stream;
+  WsHeader* ws = (WsHeader*)workspace;
+  Tile* tiles = (Tile*)((char*)workspace + L.tiles_off);
+  cudaError_t e = launch_schedule(*p, offsets, L.bm, ws, tiles, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (L.bm == kMmaBM)
+    e = launch_sm100_fwd(*p, q, k, v, o, lse, ws, tiles, st);
+  else
+    e = launch_simt_fwd(*p, q, k, v, o, lse, ws, tiles, tile_capacity(*p, L.bm), st);
+  return cuda_status(e);
+}
+
+gdpa_status_t gdpa_bwd(const gdpa_problem_t* p, const void* q, const int32_t* offsets,
+                       const void* k, const void* v, const void* o, const float* lse,
+                       const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  g_launches = 0;
+  gdpa_status_t s = check_problem(p);
+  if (s != GDPA_OK) return s;
+  if (!q || !offsets || !k || !v || !dout || !dq || !dk || !dv) return GDPA_ERR_INVALID_ARG;
+  if (p->phi == GDPA_PHI_SOFTMAX && (!o || !lse)) return GDPA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || (o && !aligned16(o)) || ((uintptr_t)offsets & 3u) ||
+      ((uintptr_t)lse & 3u))
+    return GDPA_ERR_INVALID_ARG;
+  const BwdLayout L = bwd_layout(*p);
+  s = check_ws(workspace, workspace_bytes, L.total);
+  if (s != GDPA_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  WsHeader* ws = (WsHeader*)workspace;
+  Tile* tiles = (Tile*)((char*)workspace + L.tiles_off);
+  float* dsum = (float*)((char*)workspace + L.dsum_off);
+  cudaError_t e = launch_schedule(*p, offsets, L.bm, ws, tiles, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (p->phi == GDPA_PHI_SOFTMAX) {
+    e = launch_row_dot(*p, o, dout, dsum, st);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  if (L.bm == kMmaBM) {
+    float* dq_acc = (float*)((char*)workspace + L.dqacc_off);
+    e = launch_sm100_bwd(*p, q, offsets, k, v, lse, dsum, dout, dq, dk, dv, dq_acc, ws, tiles, st);
+    return cuda_status(e);
+  }
+  e = launch_simt_bwd_dq(*p, q, k, v, lse, dsum, dout, dq, ws, tiles, tile_capacity(*p, L.bm), st);
+  if (e != cudaSuccess) return cuda_status(e);
+  e = launch_simt_bwd_dkdv(*p, q, offsets, k, v, lse, dsum, dout, dk, dv, ws, st);
+  return cuda_status(e);
+}
+
+gdpa_status_t gdpa_workspace_status(const void* workspace, void* stream, int32_t* status) {
+  if (!workspace || !status) return GDPA_ERR_INVALID_ARG;
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost,
+                                  (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  *status = v;
+  return GDPA_OK;
+}
+
+const char* gdpa_status_string(gdpa_status_t s) {
+  switch (s) {
+    case GDPA_OK: return "GDPA_OK";
+    case GDPA_ERR_INVALID_ARG: return "GDPA_ERR_INVALID_ARG: invalid argument or offsets";
+    case GDPA_ERR_UNSUPPORTED: return "GDPA_ERR_UNSUPPORTED: unsupported problem shape";
+    case GDPA_ERR_CUDA: return "GDPA_ERR_CUDA: CUDA call or kernel launch failed";
+    case GDPA_ERR_TIMEOUT: return "GDPA_ERR_TIMEOUT: a bounded wait inside a kernel expired";
+    case GDPA_ERR_WORKSPACE: return "GDPA_ERR_WORKSPACE: workspace null, misaligned or too small";
+  }
+  return "GDPA: unknown status";
+}
+
+int32_t gdpa_last_launch_count(void) { return g_launches; }
+
+gdpa_status_t gdpa_timing_enable(int32_t enable) {
+  clear_records();
+  g_timing = enable != 0;
+  return GDPA_OK;
+}
+
+int32_t gdpa_timing_read(gdpa_kernel_time_t* out, int32_t cap) {
+  std::vector<std::string> names;
+  std::vector<int> counts;
+  std::vector<float> totals;
+  for (auto& r : g_recs) {
+    if (cudaEventSynchronize(r.stop) != cudaSuccess) {
+      clear_records();
+      return -1;
+    }
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) {
+      clear_records();
+      return -1;
+    }
+    size_t i = 0;
+    while (i < names.size() && names[i] != r.name) ++i;
+    if (i == names.size()) {
+      names.push_back(r.name);
+      counts.push_back(0);
+      totals.push_back(0.f);
+    }
+    counts[i] += 1;
+    totals[i] += ms;
+  }
+  clear_records();
+  for (size_t i = 0; i < names.size() && (int32_t)i < cap && out; ++i) {
+    memset(out[i].name, 0, sizeof(out[i].name));
+    strncpy(out[i].name, names[i].c_str(), sizeof(out[i].name) - 1);
+    out[i].launches = counts[i];
+    out[i].total_ms = totals[i];
+  }
+  return (int32_t)names.size();
+}
+
+}  // extern "C"

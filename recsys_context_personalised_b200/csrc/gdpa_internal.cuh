@@ -1,0 +1,84 @@
+// Internal declarations shared by the GDPA library's translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdpa.h"
+
+namespace gdpa {
+
+// One work item of a jagged tile list: `rows` query rows of sample `b`,
+// head `head`, starting at global token `row0` (rows <= the list's tile size).
+struct __align__(16) Tile {
+  int32_t b, head, row0, rows;
+};
+
+// Workspace header (first 256 bytes of every workspace).
+struct __align__(16) WsHeader {
+  int32_t status;      // gdpa_status_t detected on the device (sticky per call)
+  int32_t tile_count;  // tiles written by the scheduler
+  int32_t pad[62];
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+constexpr int kSimtBM = 64;    // query rows per SIMT tile
+constexpr int kMmaBM = 128;    // query rows per tcgen05 tile (TMEM lanes)
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Upper bound of sum_b ceil(n_b / bm) * h given T and B.
+inline int64_t tile_capacity(const gdpa_problem_t& p, int bm) {
+  return (int64_t)p.h * (p.total_tokens / bm + p.B);
+}
+
+// Device-side error reporting: first error wins.
+__device__ __forceinline__ void report(WsHeader* ws, int code) {
+  atomicCAS(&ws->status, 0, code);
+}
+
+// ---------------------------------------------------------------------------
+// element conversions
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float to_f(float x) { return x; }
+  static __device__ __forceinline__ float from_f(float x) { return x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+  static __device__ __forceinline__ __nv_bfloat16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+// ---------------------------------------------------------------------------
+// launchers (each returns cudaSuccess or the launch error)
+
+// Builds the jagged tile list (tiles of `bm` rows) and clears the status word.
+cudaError_t launch_schedule(const gdpa_problem_t& p, const int32_t* offsets, int bm,
+                            WsHeader* ws, Tile* tiles, cudaStream_t st);
+
+// SIMT kernels (fp32 or bf16 elements; fp32 math).
+cudaError_t launch_simt_fwd(const gdpa_problem_t& p, const void* q, const void* k,
+                            const void* v, void* o, float* lse, WsHeader* ws,
+                            const Tile* tiles, int64_t tile_cap, cudaStream_t st);
+cudaError_t launch_row_dot(const gdpa_problem_t& p, const void* o, const void* dout,
+                           float* dsum, cudaStream_t st);
+cudaError_t launch_simt_bwd_dq(const gdpa_problem_t& p, const void* q, const void* k,
+                               const void* v, const float* lse, const float* dsum,
+                               const void* dout, void* dq, WsHeader* ws, const Tile* tiles,
+                               int64_t tile_cap, cudaStream_t st);
+cudaError_t launch_simt_bwd_dkdv(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
+                                 const void* k, const void* v, const float* lse,
+                                 const float* dsum, const void* dout, void* dk, void* dv,
+                                 WsHeader* ws, cudaStream_t st);
+
+// Brackets one kernel launch: counts it for gdpa_last_launch_count() and, while
+// gdpa_timing_enable(1) is in force, records CUDA events around it on `st`.
+struct KernelScope {
+  KernelScope(const char* name, cudaStream_t st);
+  ~KernelScope();
+  int rec;
+  cudaStream_t st;
+};
+
+}  // namespace gdpa

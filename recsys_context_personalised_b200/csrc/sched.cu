@@ -1,0 +1,91 @@
+// Jagged tile scheduler: device offsets -> list of (sample, head, row range)
+// work items, with no host synchronisation.
+//
+// Samples have different history lengths n_b (the Kunlun summary, section 1,
+// names irregular tensor shapes as a cause of low utilisation).  Every sample
+// b is cut into ceil(n_b / bm) query tiles; item order is sample-major, then
+// head, then tile, so the tiles that share one (sample, head) key/value set
+// are adjacent in the list and run at the same time on neighbouring SMs,
+// which keeps that K/V set resident in L2.
+#include "gdpa_internal.cuh"
+
+namespace gdpa {
+namespace {
+
+constexpr int kSchedThreads = 1024;
+
+__global__ void __launch_bounds__(kSchedThreads)
+schedule_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T, int max_n,
+                int bm, WsHeader* ws, Tile* __restrict__ tiles, int64_t cap) {
+  __shared__ int s_bad;
+  __shared__ int s_scan[kSchedThreads];
+  __shared__ long long s_carry;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    s_bad = 0;
+    s_carry = 0;
+    ws->status = GDPA_OK;
+    if (offsets[0] != 0 || (int64_t)offsets[B] != T) s_bad = 1;
+  }
+  __syncthreads();
+  for (int b = tid; b < B; b += kSchedThreads) {
+    const int n = offsets[b + 1] - offsets[b];
+    if (n < 0 || n > max_n) s_bad = 1;
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (tid == 0) {
+      ws->status = GDPA_ERR_INVALID_ARG;
+      ws->tile_count = 0;
+    }
+    return;
+  }
+  for (int base = 0; base < B; base += kSchedThreads) {
+    const int b = base + tid;
+    const int n = b < B ? offsets[b + 1] - offsets[b] : 0;
+    const int nt = (n + bm - 1) / bm;
+    s_scan[tid] = nt;
+    __syncthreads();
+    for (int d = 1; d < kSchedThreads; d <<= 1) {
+      const int add = tid >= d ? s_scan[tid - d] : 0;
+      __syncthreads();
+      s_scan[tid] += add;
+      __syncthreads();
+    }
+    const long long excl = s_carry + s_scan[tid] - nt;
+    if (b < B) {
+      const int t0 = offsets[b];
+      for (int j = 0; j < h; ++j)
+        for (int t = 0; t < nt; ++t) {
+          const long long idx = (long long)h * excl + (long long)j * nt + t;
+          if (idx < cap) {
+            Tile w;
+            w.b = b;
+            w.head = j;
+            w.row0 = t0 + t * bm;
+            w.rows = min(bm, n - t * bm);
+            tiles[idx] = w;
+          }
+        }
+    }
+    __syncthreads();
+    if (tid == kSchedThreads - 1) s_carry += s_scan[kSchedThreads - 1];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    const long long total = (long long)h * s_carry;
+    ws->tile_count = (int)(total < cap ? total : cap);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_schedule(const gdpa_problem_t& p, const int32_t* offsets, int bm,
+                            WsHeader* ws, Tile* tiles, cudaStream_t st) {
+  KernelScope ks_("gdpa_schedule", st);
+  schedule_kernel<<<1, kSchedThreads, 0, st>>>(offsets, p.B, p.h, p.total_tokens, p.max_n,
+                                                bm, ws, tiles, tile_capacity(p, bm));
+  return cudaGetLastError();
+}
+
+}  // namespace gdpa

@@ -1,0 +1,195 @@
+"""ctypes binding of libgdpa.so (the C ABI declared in include/gdpa.h).
+
+Argument marshalling only: every step of GDPA runs in the library's CUDA
+kernels.  PyTorch provides device memory and the current CUDA stream.  There
+is no CPU fallback: if the shared library is missing or fails to load, every
+call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdpa.so")
+
+PHI_IDENTITY, PHI_SILU, PHI_SOFTMAX = 0, 1, 2
+PHI = {"identity": PHI_IDENTITY, "silu": PHI_SILU, "softmax": PHI_SOFTMAX}
+DTYPE_F32, DTYPE_BF16 = 0, 1
+STATUS = {0: "GDPA_OK", 1: "GDPA_ERR_INVALID_ARG", 2: "GDPA_ERR_UNSUPPORTED",
+          3: "GDPA_ERR_CUDA", 4: "GDPA_ERR_TIMEOUT", 5: "GDPA_ERR_WORKSPACE"}
+
+EXPORTED = ("gdpa_fwd_workspace_size", "gdpa_bwd_workspace_size", "gdpa_fwd", "gdpa_bwd",
+            "gdpa_workspace_status", "gdpa_status_string", "gdpa_last_launch_count",
+            "gdpa_timing_enable", "gdpa_timing_read")
+
+
+class Problem(ctypes.Structure):
+    """Mirror of gdpa_problem_t."""
+    _fields_ = [("B", ctypes.c_int32), ("h", ctypes.c_int32), ("dh", ctypes.c_int32),
+                ("m", ctypes.c_int32), ("max_n", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("total_tokens", ctypes.c_int64), ("phi", ctypes.c_int32),
+                ("scale", ctypes.c_float)]
+
+
+class KernelTime(ctypes.Structure):
+    """Mirror of gdpa_kernel_time_t."""
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int32),
+                ("total_ms", ctypes.c_float)]
+
+
+class GdpaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libgdpa.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libgdpa.so not built at {path}; run __graft_entry__.build()")
+    lib = ctypes.CDLL(path)
+    vp, sz, pp = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(Problem)
+    lib.gdpa_fwd_workspace_size.argtypes = [pp, ctypes.POINTER(sz)]
+    lib.gdpa_bwd_workspace_size.argtypes = [pp, ctypes.POINTER(sz)]
+    lib.gdpa_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.gdpa_bwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.gdpa_workspace_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
+    lib.gdpa_status_string.argtypes = [ctypes.c_int]
+    lib.gdpa_status_string.restype = ctypes.c_char_p
+    lib.gdpa_last_launch_count.restype = ctypes.c_int32
+    lib.gdpa_timing_enable.argtypes = [ctypes.c_int32]
+    lib.gdpa_timing_enable.restype = ctypes.c_int
+    lib.gdpa_timing_read.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int32]
+    lib.gdpa_timing_read.restype = ctypes.c_int32
+    for name in EXPORTED[:5]:
+        getattr(lib, name).restype = ctypes.c_int
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def problem(B: int, h: int, dh: int, m: int, total_tokens: int, max_n: int, phi, scale: float,
+            dtype: torch.dtype) -> Problem:
+    phi = PHI[phi] if isinstance(phi, str) else int(phi)
+    dt = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}.get(dtype, -1)
+    return Problem(B, h, dh, m, max_n, dt, total_tokens, phi, scale)
+
+
+def problem_for(q: torch.Tensor, k: torch.Tensor, offsets_host, phi, scale: float,
+                max_n: Optional[int] = None) -> Problem:
+    """Problem of a batch; ``offsets_host`` is a host sequence (for T and max_n)."""
+    B, h, m, dh = k.shape
+    off = [int(x) for x in offsets_host]
+    T = off[-1]
+    if max_n is None:
+        max_n = max((off[i + 1] - off[i] for i in range(B)), default=0)
+    return problem(B, h, dh, m, T, max_n, phi, scale, q.dtype)
+
+
+def fwd_workspace_bytes(p: Problem) -> int:
+    n = ctypes.c_size_t()
+    rc = load().gdpa_fwd_workspace_size(ctypes.byref(p), ctypes.byref(n))
+    if rc:
+        raise GdpaError(rc, "gdpa_fwd_workspace_size")
+    return n.value
+
+
+def bwd_workspace_bytes(p: Problem) -> int:
+    n = ctypes.c_size_t()
+    rc = load().gdpa_bwd_workspace_size(ctypes.byref(p), ctypes.byref(n))
+    if rc:
+        raise GdpaError(rc, "gdpa_bwd_workspace_size")
+    return n.value
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A 256-byte aligned device buffer (torch's caching allocator aligns to 512)."""
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def fwd(p: Problem, q, offsets, k, v, o=None, lse=None, ws=None, stream=None
+        ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Run gdpa_fwd; allocates the outputs/workspace with torch when not given."""
+    lib = load()
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and p.phi == PHI_SOFTMAX:
+        lse = torch.empty((p.h, p.total_tokens), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(fwd_workspace_bytes(p), q.device)
+    rc = lib.gdpa_fwd(ctypes.byref(p), _ptr(q), _ptr(offsets), _ptr(k), _ptr(v), _ptr(o),
+                      _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise GdpaError(rc, "gdpa_fwd")
+    return o, lse
+
+
+def bwd(p: Problem, q, offsets, k, v, o, lse, dout, dq=None, dk=None, dv=None, ws=None,
+        stream=None):
+    """Run gdpa_bwd; returns (dq, dk, dv)."""
+    lib = load()
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if ws is None:
+        ws = workspace(bwd_workspace_bytes(p), q.device)
+    rc = lib.gdpa_bwd(ctypes.byref(p), _ptr(q), _ptr(offsets), _ptr(k), _ptr(v), _ptr(o),
+                      _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
+                      _stream(stream))
+    if rc:
+        raise GdpaError(rc, "gdpa_bwd")
+    return dq, dk, dv
+
+
+def workspace_status(ws: torch.Tensor, stream=None) -> int:
+    """Device-detected status of the last call that used ``ws`` (synchronises)."""
+    out = ctypes.c_int32()
+    rc = load().gdpa_workspace_status(_ptr(ws), _stream(stream), ctypes.byref(out))
+    if rc:
+        raise GdpaError(rc, "gdpa_workspace_status")
+    return out.value
+
+
+def last_launch_count() -> int:
+    return load().gdpa_last_launch_count()
+
+
+def status_string(code: int) -> str:
+    return load().gdpa_status_string(code).decode()
+
+
+def timing_enable(on: bool = True) -> None:
+    """Bracket every later kernel launch on this thread with CUDA events."""
+    rc = load().gdpa_timing_enable(1 if on else 0)
+    if rc:
+        raise GdpaError(rc, "gdpa_timing_enable")
+
+
+def timing_read() -> dict:
+    """{kernel name: (launches, total ms)} since timing_enable(True); clears."""
+    cap = 32
+    buf = (KernelTime * cap)()
+    n = load().gdpa_timing_read(buf, cap)
+    if n < 0:
+        raise GdpaError(3, "gdpa_timing_read")
+    return {buf[i].name.decode(): (buf[i].launches, buf[i].total_ms) for i in range(min(n, cap))}
