@@ -1,0 +1,539 @@
+// Fused GDPA forward for sm_100a: TMA + tcgen05 (TMEM accumulators).
+//
+// Operator (Kunlun summary, section 2.2, GDPA bullet: PFFN recast as a
+// multi-head attention operator fused into one FlashAttention-like kernel;
+// RecSysChannel review "Kunlun ... [2/2]", items 1-2: K and V come from the
+// context features, the event sequence is turned into Q).  Per work tile
+// (sample b, head j, up to 128 query rows) and per 128-key block:
+//   S = Q K^T            tcgen05.mma, A and B from shared memory, S in TMEM
+//   P = phi(s S)         activation warps: TMEM -> registers -> TMEM (bf16)
+//   O += P V             tcgen05.mma, A = P from TMEM, B = V from shared memory
+// softmax keeps running row statistics (online softmax, rescaling only when the
+// running max grows by more than 2^8); the elementwise phi needs none.
+//
+// CTA = 12 warps, one persistent CTA per SM, static round-robin over the tile list:
+//   warp 0      TMA producer (one lane): Q tile, then K_0, K_1, V_0, K_2, V_1, ...
+//   warp 1      MMA issuer (one lane)
+//   warp 2      TMEM allocator
+//   warps 4-7   activation group 0: key blocks with even global step
+//   warps 8-11  activation group 1: odd steps
+// The two activation groups alternate so that one computes phi while the
+// tensor core runs the other's MMAs.  For softmax each group owns its own
+// statistics and O accumulator (O_0, O_1), combined in the epilogue.
+//
+// TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256) (P_b aliases the
+// first 64 columns of S_b as packed bf16), O_0 [256, 256+dh), O_1 [256+dh, 256+2dh).
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "gdpa_internal.cuh"
+#include "sm100.cuh"
+
+namespace gdpa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 384;
+constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s per wait; a healthy wait is microseconds
+
+struct FwdArgs {
+  const Tile* tiles;
+  WsHeader* ws;
+  __nv_bfloat16* o;
+  float* lse;
+  int64_t T;
+  int h, m, nkv;
+  float scale;       // s
+  float scale_log2;  // s * log2(e)
+};
+
+template <int DH>
+struct FwdCfg {
+  static constexpr int BN = 128;
+  static constexpr int CH = DH < 64 ? DH : 64;          // elements per swizzled row
+  static constexpr int NCH = DH / CH;                   // chunks along dh
+  static constexpr uint32_t ROWB = CH * 2;              // bytes per row (64 or 128)
+  static constexpr uint32_t CHUNKB = 128 * ROWB;        // one [128 x CH] chunk
+  static constexpr uint32_t TILEB = NCH * CHUNKB;       // 128 * DH * 2
+  static constexpr uint32_t SW = DH < 64 ? kSw64 : kSw128;
+  static constexpr uint32_t ATOM = 8 * ROWB;            // 8-row group stride
+  static constexpr int NS = DH == 32 ? 8 : (DH == 64 ? 6 : 4);
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + DH;
+  // barrier slots
+  static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_SFULL = 4, B_PFULL = 6, B_OFULL = 8,
+                       B_OEMPTY = 9, B_DRAIN = 10, B_STATS = 11, B_KVFULL = 12,
+                       B_KVEMPTY = 12 + NS, NBAR = 12 + 2 * NS;
+  static constexpr uint32_t CTL_BYTES = 4096;
+  static constexpr uint32_t SMEM_USED = 1024 + (2 + NS) * TILEB + CTL_BYTES;
+  // at least 120 KB so that two CTAs never share an SM (each allocates all 512 TMEM columns)
+  static constexpr uint32_t SMEM = SMEM_USED > 120u * 1024u ? SMEM_USED : 120u * 1024u;
+};
+
+__device__ __forceinline__ float silu_tanh(float s, float half_scale) {
+  const float hx = s * half_scale;                 // x/2 with x = s * scale
+  return fmaf(hx, tanh_approx(hx), hx);             // x/2 * (1 + tanh(x/2)) = x * logistic(x)
+}
+
+template <int DH, int PHI>
+__global__ void __launch_bounds__(kThreads, 1)
+gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+  using C = FwdCfg<DH>;
+  constexpr bool SOFTMAX = PHI == GDPA_PHI_SOFTMAX;
+  constexpr uint32_t IDESC_S = idesc_bf16(128, 128, 0, 0);
+  constexpr uint32_t IDESC_O = idesc_bf16(128, DH, 0, 1);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sQ = base;
+  const uint32_t sKV = base + 2 * C::TILEB;
+  uint8_t* ctl = gbase + (2 + C::NS) * C::TILEB;
+  const uint32_t bar0 = smem_u32(ctl);
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 8 * C::NBAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 8 * C::NBAR + 4);
+  float* st_m = reinterpret_cast<float*>(ctl + 1024);         // [2][128]
+  float* st_l = st_m + 256;                                   // [2][128]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::B_QFULL + i), 1);
+      mbar_init(bar(C::B_QEMPTY + i), 1);
+      mbar_init(bar(C::B_SFULL + i), 1);
+      mbar_init(bar(C::B_PFULL + i), 128);
+    }
+    mbar_init(bar(C::B_OFULL), 1);
+    mbar_init(bar(C::B_OEMPTY), 256);
+    mbar_init(bar(C::B_DRAIN), 1);
+    mbar_init(bar(C::B_STATS), 256);
+    for (int i = 0; i < C::NS; ++i) {
+      mbar_init(bar(C::B_KVFULL + i), 1);
+      mbar_init(bar(C::B_KVEMPTY + i), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int count = a.ws->tile_count;
+  const int nkv = a.nkv;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t tc = 0, slot = 0, sphase = 0;
+      auto load_kv = [&](const CUtensorMap* map, const Tile& tl, int j) -> bool {
+        if (!mbar_wait(bar(C::B_KVEMPTY + slot), sphase ^ 1u, abort_flag, kTimeoutNs)) return false;
+        mbar_expect_tx(bar(C::B_KVFULL + slot), C::TILEB);
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c)
+          tma_load_4d(sKV + slot * C::TILEB + c * C::CHUNKB, map, bar(C::B_KVFULL + slot),
+                      c * C::CH, j * C::BN, tl.head, tl.b);
+        if (++slot == (uint32_t)C::NS) {
+          slot = 0;
+          sphase ^= 1u;
+        }
+        return true;
+      };
+      for (int t = blockIdx.x; t < count; t += gridDim.x, ++tc) {
+        const Tile tl = a.tiles[t];
+        const uint32_t qb = tc & 1u;
+        if (!mbar_wait(bar(C::B_QEMPTY + qb), ((tc >> 1) & 1u) ^ 1u, abort_flag, kTimeoutNs)) break;
+        mbar_expect_tx(bar(C::B_QFULL + qb), C::TILEB);
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c)
+          tma_load_3d(sQ + qb * C::TILEB + c * C::CHUNKB, &tmQ, bar(C::B_QFULL + qb), c * C::CH,
+                      tl.head, tl.row0);
+        bool ok = load_kv(&tmK, tl, 0);
+        for (int j = 1; ok && j < nkv; ++j) ok = load_kv(&tmK, tl, j) && load_kv(&tmV, tl, j - 1);
+        ok = ok && load_kv(&tmV, tl, nkv - 1);
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t tc = 0, slot = 0, sphase = 0, g = 0;
+      bool ok = true;
+      auto next_slot = [&]() {
+        if (++slot == (uint32_t)C::NS) {
+          slot = 0;
+          sphase ^= 1u;
+        }
+      };
+      for (int t = blockIdx.x; ok && t < count; t += gridDim.x, ++tc) {
+        const uint32_t qb = tc & 1u;
+        if (!mbar_wait(bar(C::B_QFULL + qb), (tc >> 1) & 1u, abort_flag, kTimeoutNs)) break;
+        tc_fence_after();
+        const uint32_t qaddr = sQ + qb * C::TILEB;
+        // O += P_i V_i for key block i at global step gi
+        auto issue_pv = [&](int i, uint32_t gi) -> bool {
+          const uint32_t bi = gi & 1u;
+          if (!mbar_wait(bar(C::B_PFULL + bi), (gi >> 1) & 1u, abort_flag, kTimeoutNs)) return false;
+          if (i == 0 && !mbar_wait(bar(C::B_OEMPTY), (tc & 1u) ^ 1u, abort_flag, kTimeoutNs))
+            return false;
+          if (!mbar_wait(bar(C::B_KVFULL + slot), sphase, abort_flag, kTimeoutNs)) return false;
+          tc_fence_after();
+          const uint32_t vaddr = sKV + slot * C::TILEB;
+          const uint32_t ocol = (SOFTMAX && bi) ? C::COL_O1 : C::COL_O0;
+          const bool first = SOFTMAX ? (i < 2) : (i == 0);
+          const uint32_t pcol = bi ? C::COL_S1 : C::COL_S0;
+#pragma unroll
+          for (int k = 0; k < C::BN / 16; ++k) {
+            const uint64_t bdesc = smem_desc(vaddr + k * 2 * C::ATOM, C::CHUNKB, C::ATOM, C::SW);
+            mma_ts(tmem + ocol, tmem + pcol + k * 8, bdesc, IDESC_O, (!first || k > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(C::B_KVEMPTY + slot));
+          next_slot();
+          return true;
+        };
+        for (int j = 0; ok && j < nkv; ++j, ++g) {
+          if (!mbar_wait(bar(C::B_KVFULL + slot), sphase, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t kaddr = sKV + slot * C::TILEB;
+          const uint32_t buf = g & 1u;
+          const uint32_t scol = buf ? C::COL_S1 : C::COL_S0;
+#pragma unroll
+          for (int k = 0; k < DH / 16; ++k) {
+            const int c = k / (C::CH / 16), kk = k % (C::CH / 16);
+            const uint64_t adesc = smem_desc(qaddr + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW);
+            const uint64_t bdesc = smem_desc(kaddr + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW);
+            mma_ss(tmem + scol, adesc, bdesc, IDESC_S, k > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(C::B_KVEMPTY + slot));
+          mma_commit(bar(C::B_SFULL + buf));
+          if (j == nkv - 1) mma_commit(bar(C::B_QEMPTY + qb));
+          next_slot();
+          if (j >= 1) ok = issue_pv(j - 1, g - 1);
+        }
+        if (ok) ok = issue_pv(nkv - 1, g - 1);
+        if (ok) mma_commit(bar(C::B_OFULL));
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ activation groups
+    const int grp = (warp - 4) >> 2;            // 0 or 1
+    const int quad = warp & 3;                  // TMEM lane quadrant
+    const int row = quad * 32 + lane;           // tile row owned by this thread
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t my_s = tmem + lane_off + (grp ? C::COL_S1 : C::COL_S0);
+    const float c2 = a.scale_log2;
+    const float half_scale = 0.5f * a.scale;
+    uint32_t tc = 0, g = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < count; t += gridDim.x, ++tc) {
+      const Tile tl = a.tiles[t];
+      const uint32_t g0 = g;
+      float m_run = -INFINITY, l_run = 0.f;
+      int steps = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const uint32_t gj = g0 + j;
+        if ((int)(gj & 1u) != grp) continue;
+        bool w = mbar_wait(bar(C::B_SFULL + grp), (gj >> 1) & 1u, abort_flag, kTimeoutNs);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int valid = min(C::BN, a.m - j * C::BN);
+        if constexpr (SOFTMAX) {
+          uint32_t s[128];
+          tmem_ld_x32(my_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+          tmem_ld_x32(my_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+          tmem_ld_x32(my_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+          tmem_ld_x32(my_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+          tmem_wait_ld();
+          float mx = c2 >= 0.f ? -INFINITY : INFINITY;
+          if (valid == C::BN) {
+            if (c2 >= 0.f) {
+#pragma unroll
+              for (int i = 0; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 128; ++i) mx = fminf(mx, __uint_as_float(s[i]));
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if (i < valid) mx = c2 >= 0.f ? fmaxf(mx, __uint_as_float(s[i])) : fminf(mx, __uint_as_float(s[i]));
+          }
+          const float m_new = mx * c2;
+          float alpha = 1.f;
+          bool resc = false;
+          if (steps == 0) {
+            m_run = m_new;
+          } else if (m_new > m_run + 8.0f) {
+            alpha = ex2_approx(m_run - m_new);
+            m_run = m_new;
+            resc = true;
+          }
+          const float neg_m = -m_run;
+          float rs = 0.f;
+          uint32_t pk[64];
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * i]), c2, neg_m));
+            float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * i + 1]), c2, neg_m));
+            if (valid < C::BN) {
+              p0 = (2 * i < valid) ? p0 : 0.f;
+              p1 = (2 * i + 1 < valid) ? p1 : 0.f;
+            }
+            rs += p0 + p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_x32(my_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+          tmem_st_x32(my_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+          l_run = l_run * alpha + rs;
+          if (__any_sync(0xffffffffu, resc)) {
+            const uint32_t my_o = tmem + lane_off + (grp ? C::COL_O1 : C::COL_O0);
+#pragma unroll
+            for (int c = 0; c < DH; c += 16) {
+              uint32_t ov[16];
+              tmem_ld_x16(my_o + c, ov);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              tmem_st_x16(my_o + c, ov);
+            }
+          }
+          tmem_wait_st();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t s[32];
+            tmem_ld_x32(my_s + 32 * c, s);
+            tmem_wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float x0 = __uint_as_float(s[2 * i]), x1 = __uint_as_float(s[2 * i + 1]);
+              float p0, p1;
+              if constexpr (PHI == GDPA_PHI_SILU) {
+                p0 = silu_tanh(x0, half_scale);
+                p1 = silu_tanh(x1, half_scale);
+              } else {
+                p0 = x0 * a.scale;
+                p1 = x1 * a.scale;
+              }
+              pk[i] = pack_bf16x2(p0, p1);
+            }
+            tmem_st_x16(my_s + 16 * c, pk);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(bar(C::B_PFULL + grp));
+        ++steps;
+      }
+      if (!ok) break;
+      g = g0 + nkv;
+      // ---------------------------------------------------------- epilogue
+      bool w = mbar_wait(bar(C::B_OFULL), tc & 1u, abort_flag, kTimeoutNs);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool has0 = nkv >= 2 || (g0 & 1u) == 0;
+      const bool has1 = nkv >= 2 || (g0 & 1u) == 1;
+      float f0 = 1.f, f1 = 0.f, inv = 1.f, M = 0.f, L = 1.f;
+      if constexpr (SOFTMAX) {
+        st_m[grp * 128 + row] = steps ? m_run : -INFINITY;
+        st_l[grp * 128 + row] = l_run;
+        mbar_arrive(bar(C::B_STATS));
+        w = mbar_wait(bar(C::B_STATS), tc & 1u, abort_flag, kTimeoutNs);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        const float m0 = st_m[row], m1 = st_m[128 + row];
+        const float l0 = st_l[row], l1 = st_l[128 + row];
+        M = fmaxf(m0, m1);
+        f0 = has0 ? ex2_approx(m0 - M) : 0.f;
+        f1 = has1 ? ex2_approx(m1 - M) : 0.f;
+        L = l0 * f0 + l1 * f1;
+        inv = 1.f / L;
+        f0 *= inv;
+        f1 *= inv;
+      }
+      const int col0 = grp * (DH / 2);
+      const bool store = row < tl.rows;
+      __nv_bfloat16* orow = a.o + ((int64_t)(tl.row0 + row) * a.h + tl.head) * DH + col0;
+#pragma unroll
+      for (int c = 0; c < DH / 2; c += 16) {
+        uint32_t v0[16], v1[16];
+        tmem_ld_x16(tmem + lane_off + C::COL_O0 + col0 + c, v0);
+        if (SOFTMAX && has1) tmem_ld_x16(tmem + lane_off + C::COL_O1 + col0 + c, v1);
+        tmem_wait_ld();
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float a0 = __uint_as_float(v0[2 * i]), a1 = __uint_as_float(v0[2 * i + 1]);
+          if constexpr (SOFTMAX) {
+            a0 = has0 ? a0 * f0 : 0.f;
+            a1 = has0 ? a1 * f0 : 0.f;
+            if (has1) {
+              a0 = fmaf(__uint_as_float(v1[2 * i]), f1, a0);
+              a1 = fmaf(__uint_as_float(v1[2 * i + 1]), f1, a1);
+            }
+          }
+          pk[i] = pack_bf16x2(a0, a1);
+        }
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+      }
+      if (SOFTMAX && grp == 0 && store && a.lse != nullptr)
+        a.lse[(int64_t)tl.head * a.T + tl.row0 + row] = (M + __log2f(L)) * 0.69314718055994531f;
+      tc_fence_before();
+      mbar_arrive(bar(C::B_OEMPTY));
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  __syncwarp();
+  __syncthreads();
+  if (*abort_flag) {
+    report(a.ws, GDPA_ERR_TIMEOUT);
+    volatile int never = 0;
+    if (warp == 1 && lane == 0) {
+      mma_commit(bar(C::B_DRAIN));                       // all MMAs issued so far
+      mbar_wait(bar(C::B_DRAIN), 0, &never, kTimeoutNs);
+    }
+    if (warp == 0 && lane == 0) {                         // let in-flight TMA loads land
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 200000ull) {
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <int DH>
+bool make_maps(const gdpa_problem_t& p, const void* q, const void* k, const void* v,
+               CUtensorMap* mq, CUtensorMap* mk, CUtensorMap* mv) {
+  using C = FwdCfg<DH>;
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const CUtensorMapSwizzle sw = DH < 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)DH, (cuuint64_t)p.h, (cuuint64_t)p.total_tokens};
+    const cuuint64_t strides[2] = {(cuuint64_t)DH * 2, (cuuint64_t)p.h * DH * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)C::CH, 1, 128};
+    if (enc(mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  const cuuint64_t dims[4] = {(cuuint64_t)DH, (cuuint64_t)p.m, (cuuint64_t)p.h, (cuuint64_t)p.B};
+  const cuuint64_t strides[3] = {(cuuint64_t)DH * 2, (cuuint64_t)p.m * DH * 2,
+                                 (cuuint64_t)p.h * p.m * DH * 2};
+  const cuuint32_t box[4] = {(cuuint32_t)C::CH, 128, 1, 1};
+  for (int i = 0; i < 2; ++i) {
+    if (enc(i ? mv : mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(i ? v : k), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  return true;
+}
+
+template <int DH, int PHI>
+cudaError_t launch_fwd_t(const gdpa_problem_t& p, const void* q, const void* k, const void* v,
+                         void* o, float* lse, WsHeader* ws, const Tile* tiles, cudaStream_t st) {
+  using C = FwdCfg<DH>;
+  CUtensorMap mq, mk, mv;
+  if (!make_maps<DH>(p, q, k, v, &mq, &mk, &mv)) return cudaErrorInvalidValue;
+  auto kern = gdpa_fwd_sm100_kernel<DH, PHI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return e;
+  FwdArgs args;
+  args.tiles = tiles;
+  args.ws = ws;
+  args.o = reinterpret_cast<__nv_bfloat16*>(o);
+  args.lse = lse;
+  args.T = p.total_tokens;
+  args.h = p.h;
+  args.m = p.m;
+  args.nkv = (p.m + 127) / 128;
+  args.scale = p.scale;
+  args.scale_log2 = p.scale * 1.4426950408889634f;
+  KernelScope ks_("gdpa_fwd_sm100", st);
+  kern<<<num_sms(), kThreads, C::SMEM, st>>>(mq, mk, mv, args);
+  return cudaGetLastError();
+}
+
+template <int DH>
+cudaError_t launch_fwd_dh(const gdpa_problem_t& p, const void* q, const void* k, const void* v,
+                          void* o, float* lse, WsHeader* ws, const Tile* tiles, cudaStream_t st) {
+  switch (p.phi) {
+    case GDPA_PHI_SOFTMAX: return launch_fwd_t<DH, GDPA_PHI_SOFTMAX>(p, q, k, v, o, lse, ws, tiles, st);
+    case GDPA_PHI_SILU: return launch_fwd_t<DH, GDPA_PHI_SILU>(p, q, k, v, o, lse, ws, tiles, st);
+    default: return launch_fwd_t<DH, GDPA_PHI_IDENTITY>(p, q, k, v, o, lse, ws, tiles, st);
+  }
+}
+
+}  // namespace
+
+bool sm100_fwd_available() { return true; }
+
+cudaError_t launch_sm100_fwd(const gdpa_problem_t& p, const void* q, const void* k,
+                             const void* v, void* o, float* lse, WsHeader* ws, const Tile* tiles,
+                             cudaStream_t st) {
+  if (p.total_tokens == 0) return cudaSuccess;
+  switch (p.dh) {
+    case 32: return launch_fwd_dh<32>(p, q, k, v, o, lse, ws, tiles, st);
+    case 64: return launch_fwd_dh<64>(p, q, k, v, o, lse, ws, tiles, st);
+    case 128: return launch_fwd_dh<128>(p, q, k, v, o, lse, ws, tiles, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace gdpa

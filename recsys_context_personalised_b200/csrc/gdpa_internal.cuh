@@ -57,6 +57,10 @@ template <> struct Elem<__nv_bfloat16> {
 cudaError_t launch_schedule(const gdpa_problem_t& p, const int32_t* offsets, int bm,
                             WsHeader* ws, Tile* tiles, cudaStream_t st);
 
+// Backward list of (sample, head, 128-key block) items, longest samples first.
+cudaError_t launch_schedule_kv(const gdpa_problem_t& p, const int32_t* offsets, WsHeader* ws,
+                               Tile* tiles, cudaStream_t st);
+
 // SIMT kernels (fp32 or bf16 elements; fp32 math).
 cudaError_t launch_simt_fwd(const gdpa_problem_t& p, const void* q, const void* k,
                             const void* v, void* o, float* lse, WsHeader* ws,

@@ -78,7 +78,86 @@ schedule_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T, in
   }
 }
 
+// Backward work list: one item per (sample, head, 128-key block), samples in
+// decreasing length order (longest-processing-time first), so that a static
+// round-robin over CTAs gives every SM about the same number of query tiles.
+// Item fields: b, head, row0 = first key of the block, rows = n_b.
+constexpr int kSortMax = 4096;   // 32 KB of static shared memory
+
+__global__ void __launch_bounds__(kSchedThreads)
+schedule_kv_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T, int max_n,
+                   int nkv, WsHeader* ws, Tile* __restrict__ tiles) {
+  __shared__ int s_bad;
+  __shared__ int2 s_key[kSortMax];   // (n_b, b)
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    s_bad = 0;
+    ws->status = GDPA_OK;
+    if (offsets[0] != 0 || (int64_t)offsets[B] != T) s_bad = 1;
+  }
+  __syncthreads();
+  for (int b = tid; b < B; b += kSchedThreads) {
+    const int n = offsets[b + 1] - offsets[b];
+    if (n < 0 || n > max_n) s_bad = 1;
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (tid == 0) {
+      ws->status = GDPA_ERR_INVALID_ARG;
+      ws->tile_count = 0;
+    }
+    return;
+  }
+  const bool sorted = B <= kSortMax;
+  int P2 = 1;
+  while (P2 < B) P2 <<= 1;
+  if (sorted) {
+    for (int i = tid; i < P2; i += kSchedThreads)
+      s_key[i] = i < B ? make_int2(offsets[i + 1] - offsets[i], i) : make_int2(-1, 0x7fffffff);
+    __syncthreads();
+    // bitonic sort: descending n, ascending b
+    for (int k = 2; k <= P2; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int i = tid; i < P2; i += kSchedThreads) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const int2 x = s_key[i], y = s_key[ixj];
+            const bool x_first = x.x > y.x || (x.x == y.x && x.y < y.y);
+            const bool up = (i & k) == 0;
+            if (up ? !x_first : x_first) {
+              s_key[i] = y;
+              s_key[ixj] = x;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+  }
+  const long long per_sample = (long long)h * nkv;
+  for (long long idx = tid; idx < (long long)B * per_sample; idx += kSchedThreads) {
+    const int r = (int)(idx / per_sample);
+    const int rem = (int)(idx % per_sample);
+    const int b = sorted ? s_key[r].y : r;
+    Tile w;
+    w.b = b;
+    w.head = rem / nkv;
+    w.row0 = (rem % nkv) * 128;
+    w.rows = offsets[b + 1] - offsets[b];
+    tiles[idx] = w;
+  }
+  if (tid == 0) ws->tile_count = (int)((long long)B * per_sample);
+}
+
 }  // namespace
+
+cudaError_t launch_schedule_kv(const gdpa_problem_t& p, const int32_t* offsets, WsHeader* ws,
+                               Tile* tiles, cudaStream_t st) {
+  KernelScope ks_("gdpa_schedule_kv", st);
+  schedule_kv_kernel<<<1, kSchedThreads, 0, st>>>(offsets, p.B, p.h, p.total_tokens, p.max_n,
+                                                   (p.m + 127) / 128, ws, tiles);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_schedule(const gdpa_problem_t& p, const int32_t* offsets, int bm,
                             WsHeader* ws, Tile* tiles, cudaStream_t st) {
