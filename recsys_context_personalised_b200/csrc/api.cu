@@ -41,14 +41,15 @@ static void clear_records() {
   g_recs.clear();
 }
 
-// bf16 problems run on the tcgen05 kernels when they are compiled in.
+// bf16 problems run on the tcgen05 kernels.
 cudaError_t launch_sm100_fwd(const gdpa_problem_t& p, const void* q, const void* k,
                              const void* v, void* o, float* lse, WsHeader* ws,
                              const Tile* tiles, cudaStream_t st);
 cudaError_t launch_sm100_bwd(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
-                             const void* k, const void* v, const float* lse, const float* dsum,
+                             const void* k, const void* v, const void* o, const float* lse,
                              const void* dout, void* dq, void* dk, void* dv, float* dq_acc,
-                             WsHeader* ws, const Tile* tiles, cudaStream_t st);
+                             float* dsum, WsHeader* ws, Tile* tiles, cudaStream_t st);
+int64_t sm100_bwd_items(const gdpa_problem_t& p);
 bool sm100_fwd_available();
 bool sm100_bwd_available();
 
@@ -101,7 +102,9 @@ BwdLayout bwd_layout(const gdpa_problem_t& p) {
   BwdLayout L;
   L.bm = bwd_bm(p);
   L.tiles_off = sizeof(WsHeader);
-  L.dsum_off = align_up(L.tiles_off + sizeof(Tile) * (size_t)tile_capacity(p, L.bm), 256);
+  int64_t items = tile_capacity(p, L.bm);
+  if (L.bm == kMmaBM) items = sm100_bwd_items(p);   // (sample, head, key block) list
+  L.dsum_off = align_up(L.tiles_off + sizeof(Tile) * (size_t)items, 256);
   L.dqacc_off = align_up(L.dsum_off + sizeof(float) * (size_t)p.h * (size_t)p.total_tokens, 256);
   size_t dq_bytes = 0;
   if (L.bm == kMmaBM) dq_bytes = sizeof(float) * (size_t)p.total_tokens * p.h * p.dh;
@@ -149,7 +152,9 @@ gdpa_status_t gdpa_fwd(const gdpa_problem_t* p, const void* q, const int32_t* of
   g_launches = 0;
   gdpa_status_t s = check_problem(p);
   if (s != GDPA_OK) return s;
-  if (!q || !offsets || !k || !v || !o) return GDPA_ERR_INVALID_ARG;
+  // with no tokens there is nothing to read from q or write to o
+  const bool empty = p->total_tokens == 0;
+  if (!offsets || !k || !v || (!empty && (!q || !o))) return GDPA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       ((uintptr_t)offsets & 3u) || ((uintptr_t)lse & 3u))
     return GDPA_ERR_INVALID_ARG;
@@ -176,8 +181,11 @@ gdpa_status_t gdpa_bwd(const gdpa_problem_t* p, const void* q, const int32_t* of
   g_launches = 0;
   gdpa_status_t s = check_problem(p);
   if (s != GDPA_OK) return s;
-  if (!q || !offsets || !k || !v || !dout || !dq || !dk || !dv) return GDPA_ERR_INVALID_ARG;
-  if (p->phi == GDPA_PHI_SOFTMAX && (!o || !lse)) return GDPA_ERR_INVALID_ARG;
+  // with no tokens q, o, lse, dout and dq are never touched; dk and dv are zeroed
+  const bool empty = p->total_tokens == 0;
+  if (!offsets || !k || !v || !dk || !dv) return GDPA_ERR_INVALID_ARG;
+  if (!empty && (!q || !dout || !dq)) return GDPA_ERR_INVALID_ARG;
+  if (!empty && p->phi == GDPA_PHI_SOFTMAX && (!o || !lse)) return GDPA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv) || (o && !aligned16(o)) || ((uintptr_t)offsets & 3u) ||
       ((uintptr_t)lse & 3u))
@@ -189,16 +197,16 @@ gdpa_status_t gdpa_bwd(const gdpa_problem_t* p, const void* q, const int32_t* of
   WsHeader* ws = (WsHeader*)workspace;
   Tile* tiles = (Tile*)((char*)workspace + L.tiles_off);
   float* dsum = (float*)((char*)workspace + L.dsum_off);
+  if (L.bm == kMmaBM) {
+    float* dq_acc = (float*)((char*)workspace + L.dqacc_off);
+    return cuda_status(launch_sm100_bwd(*p, q, offsets, k, v, o, lse, dout, dq, dk, dv, dq_acc,
+                                        dsum, ws, tiles, st));
+  }
   cudaError_t e = launch_schedule(*p, offsets, L.bm, ws, tiles, st);
   if (e != cudaSuccess) return cuda_status(e);
   if (p->phi == GDPA_PHI_SOFTMAX) {
     e = launch_row_dot(*p, o, dout, dsum, st);
     if (e != cudaSuccess) return cuda_status(e);
-  }
-  if (L.bm == kMmaBM) {
-    float* dq_acc = (float*)((char*)workspace + L.dqacc_off);
-    e = launch_sm100_bwd(*p, q, offsets, k, v, lse, dsum, dout, dq, dk, dv, dq_acc, ws, tiles, st);
-    return cuda_status(e);
   }
   e = launch_simt_bwd_dq(*p, q, k, v, lse, dsum, dout, dq, ws, tiles, tile_capacity(*p, L.bm), st);
   if (e != cudaSuccess) return cuda_status(e);

@@ -124,3 +124,491 @@ struct BwdCfg {
   static constexpr uint32_t SMEM_USED = 1024 + OFF_CTL + CTL_BYTES;
   static constexpr uint32_t SMEM = SMEM_USED > 120u * 1024u ? SMEM_USED : 120u * 1024u;
 };
+
+template <int DH, int PHI>
+__global__ void __launch_bounds__(kThreads, 1)
+gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmG,
+                      const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const BwdArgs a) {
+  using C = BwdCfg<DH>;
+  constexpr bool SOFTMAX = PHI == GDPA_PHI_SOFTMAX;
+  constexpr uint32_t IDESC_T = idesc_bf16(128, 128, 0, 0);   // S^T, dP^T
+  constexpr uint32_t IDESC_KV = idesc_bf16(128, DH, 0, 1);   // dV, dK (B MN-major)
+  constexpr uint32_t IDESC_Q = idesc_bf16(128, DH, 1, 1);    // dQ (A and B MN-major)
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sStg = base + C::OFF_STG;
+  const uint32_t sDS = base + C::OFF_DS;
+  uint8_t* ctl = gbase + C::OFF_CTL;
+  const uint32_t bar0 = smem_u32(ctl);
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 8 * C::NBAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 8 * C::NBAR + 4);
+  float* stats = reinterpret_cast<float*>(ctl + 1024);   // [8 warps][2][128]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_KVFULL), 1);
+    mbar_init(bar(C::B_KVEMPTY), 1);
+    mbar_init(bar(C::B_SFULL), 1);
+    mbar_init(bar(C::B_PFULL), 256);
+    mbar_init(bar(C::B_DQFULL), 1);
+    mbar_init(bar(C::B_DQEMPTY), 256);
+    mbar_init(bar(C::B_ACCFULL), 1);
+    mbar_init(bar(C::B_ACCEMPTY), 256);
+    mbar_init(bar(C::B_DRAIN), 1);
+    for (int i = 0; i < C::NSTG; ++i) {
+      mbar_init(bar(C::B_STFULL + i), 1);
+      mbar_init(bar(C::B_STEMPTY + i), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmG);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int count = a.ws->status == GDPA_ERR_INVALID_ARG ? 0 : a.ws->tile_count;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t ic = 0, stage = 0, sphase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
+        const Tile it = a.tiles[t];
+        if (it.rows == 0) continue;
+        const int nq = (it.rows + 127) >> 7;
+        const int t0 = a.offsets[it.b];
+        if (!mbar_wait(bar(C::B_KVEMPTY), (ic & 1u) ^ 1u, abort_flag, kTimeoutNs)) break;
+        mbar_expect_tx(bar(C::B_KVFULL), 2 * C::TILEB);
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          tma_load_4d(sK + c * C::CHUNKB, &tmK, bar(C::B_KVFULL), c * C::CH, it.row0, it.head, it.b);
+          tma_load_4d(sV + c * C::CHUNKB, &tmV, bar(C::B_KVFULL), c * C::CH, it.row0, it.head, it.b);
+        }
+        for (int i = 0; i < nq; ++i) {
+          if (!mbar_wait(bar(C::B_STEMPTY + stage), sphase ^ 1u, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = sStg + stage * 2 * C::TILEB;
+          mbar_expect_tx(bar(C::B_STFULL + stage), 2 * C::TILEB);
+#pragma unroll
+          for (int c = 0; c < C::NCH; ++c) {
+            tma_load_3d(dst + c * C::CHUNKB, &tmQ, bar(C::B_STFULL + stage), c * C::CH, it.head,
+                        t0 + 128 * i);
+            tma_load_3d(dst + C::TILEB + c * C::CHUNKB, &tmG, bar(C::B_STFULL + stage),
+                        c * C::CH, it.head, t0 + 128 * i);
+          }
+          if (++stage == (uint32_t)C::NSTG) {
+            stage = 0;
+            sphase ^= 1u;
+          }
+        }
+        ++ic;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t ic = 0, stage = 0, sphase = 0, qs = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
+        const Tile it = a.tiles[t];
+        if (it.rows == 0) continue;
+        const int nq = (it.rows + 127) >> 7;
+        if (!mbar_wait(bar(C::B_KVFULL), ic & 1u, abort_flag, kTimeoutNs)) break;
+        tc_fence_after();
+        for (int i = 0; i < nq; ++i, ++qs) {
+          if (!mbar_wait(bar(C::B_STFULL + stage), sphase, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t qaddr = sStg + stage * 2 * C::TILEB, gaddr = qaddr + C::TILEB;
+          // S^T = K Q_i^T
+#pragma unroll
+          for (int k = 0; k < DH / 16; ++k) {
+            const int c = k / (C::CH / 16), kk = k % (C::CH / 16);
+            mma_ss(tmem + C::COL_S, smem_desc(sK + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW),
+                   smem_desc(qaddr + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW), IDESC_T,
+                   k > 0 ? 1u : 0u);
+          }
+          // dP^T = V dO_i^T; its columns (and dQ's) must have been drained
+          if (qs >= 1 && !mbar_wait(bar(C::B_DQEMPTY), (qs - 1) & 1u, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < DH / 16; ++k) {
+            const int c = k / (C::CH / 16), kk = k % (C::CH / 16);
+            mma_ss(tmem + C::COL_DP, smem_desc(sV + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW),
+                   smem_desc(gaddr + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW), IDESC_T,
+                   k > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(C::B_SFULL));
+          if (!mbar_wait(bar(C::B_PFULL), qs & 1u, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          if (i == 0 && !mbar_wait(bar(C::B_ACCEMPTY), (ic & 1u) ^ 1u, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t first = i == 0;
+          // dV += P^T dO_i   (P^T rows 0-63 in columns 0-31, rows 64-127 in 64-95)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t acol = C::COL_S + (k < 4 ? 8 * k : 64 + 8 * (k - 4));
+            mma_ts(tmem + C::COL_DV, tmem + acol,
+                   smem_desc(gaddr + k * 2 * C::ATOM, C::CHUNKB, C::ATOM, C::SW), IDESC_KV,
+                   (!first || k > 0) ? 1u : 0u);
+          }
+          // dK += dS^T Q_i
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            mma_ss(tmem + C::COL_DK, smem_desc(sDS + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSw128),
+                   smem_desc(qaddr + k * 2 * C::ATOM, C::CHUNKB, C::ATOM, C::SW), IDESC_KV,
+                   (!first || k > 0) ? 1u : 0u);
+          }
+          // dQ_i = dS K
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            mma_ss(tmem + C::COL_DQ, smem_desc(sDS + k * 2048, 16384, 1024, kSw128),
+                   smem_desc(sK + k * 2 * C::ATOM, C::CHUNKB, C::ATOM, C::SW), IDESC_Q,
+                   k > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(C::B_STEMPTY + stage));
+          mma_commit(bar(C::B_DQFULL));
+          if (++stage == (uint32_t)C::NSTG) {
+            stage = 0;
+            sphase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(bar(C::B_KVEMPTY));
+        mma_commit(bar(C::B_ACCFULL));
+        ++ic;
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ activation groups
+    const int grp = (warp - 4) >> 2;
+    const int quad = warp & 3;
+    const int lrow = quad * 32 + lane;                 // TMEM lane: key (S^T, dV, dK) or row (dQ)
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    float* wst = stats + (warp - 4) * 256;             // this warp's row statistics
+    const float c2 = a.scale_log2, sc = a.scale, half_sc = 0.5f * a.scale;
+    uint32_t ic = 0, qs = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
+      const Tile it = a.tiles[t];
+      const int n = it.rows;
+      const int key = it.row0 + lrow;
+      __nv_bfloat16* kvout = (grp == 0 ? a.dv : a.dk) +
+                             (((int64_t)it.b * a.h + it.head) * a.m + key) * DH;
+      if (n == 0) {                                    // no tokens: dK = dV = 0
+        if (key < a.m) {
+          uint4* d4 = reinterpret_cast<uint4*>(kvout);
+#pragma unroll
+          for (int c = 0; c < DH / 8; ++c) d4[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        continue;
+      }
+      const int nq = (n + 127) >> 7;
+      const int t0 = a.offsets[it.b];
+      for (int i = 0; i < nq; ++i, ++qs) {
+        const int rbase = 128 * i + 64 * grp;          // first sample row of this group's half
+        if constexpr (SOFTMAX) {
+          __syncwarp();
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int r = 32 * u + lane, rg = rbase + r;
+            float l2 = 0.f, dd = 0.f;
+            if (rg < n) {
+              const int64_t at = (int64_t)it.head * a.T + t0 + rg;
+              l2 = a.lse[at] * 1.4426950408889634f;
+              dd = a.dsum[at];
+            }
+            wst[r] = l2;
+            wst[64 + r] = dd;
+          }
+          __syncwarp();
+        }
+        bool w = mbar_wait(bar(C::B_SFULL), qs & 1u, abort_flag, kTimeoutNs);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          const uint32_t col = 64 * grp + 32 * ch;
+          uint32_t s[32], dp[32];
+          tmem_ld_x32(tmem + lane_off + C::COL_S + col, s);
+          tmem_ld_x32(tmem + lane_off + C::COL_DP + col, dp);
+          tmem_wait_ld();
+          uint32_t pp[16], dd[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            float pv[2], dv2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int r = 32 * ch + c + e;
+              const float x = __uint_as_float(s[c + e]);
+              const float g = __uint_as_float(dp[c + e]);
+              float p, ds;
+              if constexpr (SOFTMAX) {
+                p = ex2_approx(fmaf(x, c2, -wst[r]));
+                ds = p * (g - wst[64 + r]);
+              } else if constexpr (PHI == GDPA_PHI_SILU) {
+                const float hx = x * half_sc;
+                const float th = tanh_approx(hx);
+                const float sg = fmaf(0.5f, th, 0.5f);          // logistic(x s)
+                p = fmaf(hx, th, hx);                             // x s * logistic(x s)
+                ds = g * sg * fmaf(x * sc, 1.f - sg, 1.f);
+              } else {
+                p = x * sc;
+                ds = g;
+              }
+              const bool valid = rbase + r < n;
+              pv[e] = valid ? p : 0.f;
+              dv2[e] = valid ? ds : 0.f;
+            }
+            pp[c / 2] = pack_bf16x2(pv[0], pv[1]);
+            dd[c / 2] = pack_bf16x2(dv2[0], dv2[1]);
+          }
+          tmem_st_x16(tmem + lane_off + C::COL_S + 64 * grp + 16 * ch, pp);
+          // dS^T line `lrow` of chunk `grp`, 16-byte pieces 4ch..4ch+3, 128B swizzle
+          const uint32_t line = sDS + grp * 16384 + lrow * 128;
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t j = 4 * ch + jj;
+            const uint32_t addr = line + ((j ^ (uint32_t)(lrow & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dd[4 * jj]),
+                         "r"(dd[4 * jj + 1]), "r"(dd[4 * jj + 2]), "r"(dd[4 * jj + 3])
+                         : "memory");
+          }
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_PFULL));
+        // dQ_i: lane = query row of tile i; this group drains half of the columns
+        w = mbar_wait(bar(C::B_DQFULL), qs & 1u, abort_flag, kTimeoutNs);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        {
+          const int rg = 128 * i + lrow;
+          float* dst = a.dq_acc + ((int64_t)(t0 + rg) * a.h + it.head) * DH + grp * (DH / 2);
+#pragma unroll
+          for (int c = 0; c < DH / 2; c += 16) {
+            uint32_t v[16];
+            tmem_ld_x16(tmem + lane_off + C::COL_DQ + grp * (DH / 2) + c, v);
+            tmem_wait_ld();
+            if (rg < n) {
+#pragma unroll
+              for (int u = 0; u < 16; u += 4)
+                red_add_v4(dst + c + u, __uint_as_float(v[u]), __uint_as_float(v[u + 1]),
+                           __uint_as_float(v[u + 2]), __uint_as_float(v[u + 3]));
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(C::B_DQEMPTY));
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- dV / dK of this key block
+      bool w = mbar_wait(bar(C::B_ACCFULL), ic & 1u, abort_flag, kTimeoutNs);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      {
+        const uint32_t src = tmem + lane_off + (grp == 0 ? C::COL_DV : C::COL_DK);
+        const float mul = grp == 0 ? 1.f : sc;
+#pragma unroll
+        for (int c = 0; c < DH; c += 16) {
+          uint32_t v[16];
+          tmem_ld_x16(src + c, v);
+          tmem_wait_ld();
+          uint32_t pk[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            pk[u] = pack_bf16x2(__uint_as_float(v[2 * u]) * mul, __uint_as_float(v[2 * u + 1]) * mul);
+          if (key < a.m) {
+            uint4* d4 = reinterpret_cast<uint4*>(kvout + c);
+            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::B_ACCEMPTY));
+      ++ic;
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  __syncwarp();
+  __syncthreads();
+  if (*abort_flag) {
+    report(a.ws, GDPA_ERR_TIMEOUT);
+    volatile int never = 0;
+    if (warp == 1 && lane == 0) {
+      mma_commit(bar(C::B_DRAIN));
+      mbar_wait(bar(C::B_DRAIN), 0, &never, kTimeoutNs);
+    }
+    if (warp == 0 && lane == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 200000ull) {
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ host side
+
+template <int DH>
+bool make_bwd_maps(const gdpa_problem_t& p, const void* q, const void* g, const void* k,
+                   const void* v, CUtensorMap* mq, CUtensorMap* mg, CUtensorMap* mk,
+                   CUtensorMap* mv) {
+  using C = BwdCfg<DH>;
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const CUtensorMapSwizzle sw = DH < 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const cuuint64_t qd[3] = {(cuuint64_t)DH, (cuuint64_t)p.h,
+                            (cuuint64_t)(p.total_tokens > 0 ? p.total_tokens : 1)};
+  const cuuint64_t qs[2] = {(cuuint64_t)DH * 2, (cuuint64_t)p.h * DH * 2};
+  const cuuint32_t qb[3] = {(cuuint32_t)C::CH, 1, 128};
+  for (int i = 0; i < 2; ++i)
+    if (enc(i ? mg : mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(i ? g : q), qd, qs,
+            qb, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  const cuuint64_t kd[4] = {(cuuint64_t)DH, (cuuint64_t)p.m, (cuuint64_t)p.h, (cuuint64_t)p.B};
+  const cuuint64_t ks[3] = {(cuuint64_t)DH * 2, (cuuint64_t)p.m * DH * 2,
+                            (cuuint64_t)p.h * p.m * DH * 2};
+  const cuuint32_t kb[4] = {(cuuint32_t)C::CH, 128, 1, 1};
+  for (int i = 0; i < 2; ++i)
+    if (enc(i ? mv : mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(i ? v : k), kd, ks,
+            kb, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  return true;
+}
+
+template <int DH, int PHI>
+cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
+                         const void* k, const void* v, const float* lse, const float* dsum,
+                         const void* g, void* dk, void* dv, float* dq_acc, WsHeader* ws,
+                         const Tile* tiles, cudaStream_t st) {
+  using C = BwdCfg<DH>;
+  CUtensorMap mq, mg, mk, mv;
+  if (p.total_tokens == 0) q = g = k;   // no query rows: the maps are never read
+  if (!make_bwd_maps<DH>(p, q, g, k, v, &mq, &mg, &mk, &mv)) return cudaErrorInvalidValue;
+  auto kern = gdpa_bwd_sm100_kernel<DH, PHI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return e;
+  BwdArgs args;
+  args.tiles = tiles;
+  args.ws = ws;
+  args.offsets = offsets;
+  args.lse = lse;
+  args.dsum = dsum;
+  args.dq_acc = dq_acc;
+  args.dk = reinterpret_cast<__nv_bfloat16*>(dk);
+  args.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+  args.T = p.total_tokens;
+  args.h = p.h;
+  args.m = p.m;
+  args.scale = p.scale;
+  args.scale_log2 = p.scale * 1.4426950408889634f;
+  KernelScope ks_("gdpa_bwd_sm100", st);
+  kern<<<device_sm_count(), kThreads, C::SMEM, st>>>(mq, mg, mk, mv, args);
+  return cudaGetLastError();
+}
+
+template <int DH>
+cudaError_t launch_bwd_dh(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
+                          const void* k, const void* v, const float* lse, const float* dsum,
+                          const void* g, void* dk, void* dv, float* dq_acc, WsHeader* ws,
+                          const Tile* tiles, cudaStream_t st) {
+  switch (p.phi) {
+    case GDPA_PHI_SOFTMAX:
+      return launch_bwd_t<DH, GDPA_PHI_SOFTMAX>(p, q, offsets, k, v, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st);
+    case GDPA_PHI_SILU:
+      return launch_bwd_t<DH, GDPA_PHI_SILU>(p, q, offsets, k, v, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st);
+    default:
+      return launch_bwd_t<DH, GDPA_PHI_IDENTITY>(p, q, offsets, k, v, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st);
+  }
+}
+
+}  // namespace
+
+bool sm100_bwd_available() { return true; }
+
+int64_t sm100_bwd_items(const gdpa_problem_t& p) {
+  return (int64_t)p.B * p.h * ((p.m + 127) / 128);
+}
+
+// schedule (LPT list) -> prep (zero dQ accumulator, softmax D) -> fused
+// backward -> dQ conversion.
+cudaError_t launch_sm100_bwd(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
+                             const void* k, const void* v, const void* o, const float* lse,
+                             const void* dout, void* dq, void* dk, void* dv, float* dq_acc,
+                             float* dsum, WsHeader* ws, Tile* tiles, cudaStream_t st) {
+  cudaError_t e = launch_schedule_kv(p, offsets, ws, tiles, st);
+  if (e != cudaSuccess) return e;
+  const int64_t rows = p.total_tokens * p.h;
+  const int sms = device_sm_count();
+  if (rows > 0) {
+    KernelScope ks_("gdpa_bwd_prep", st);
+    bwd_prep_kernel<<<sms * 8, 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dout),
+        dsum, reinterpret_cast<float4*>(dq_acc), rows, p.h, p.dh, p.total_tokens,
+        p.phi == GDPA_PHI_SOFTMAX ? 1 : 0);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  switch (p.dh) {
+    case 32: e = launch_bwd_dh<32>(p, q, offsets, k, v, lse, dsum, dout, dk, dv, dq_acc, ws, tiles, st); break;
+    case 64: e = launch_bwd_dh<64>(p, q, offsets, k, v, lse, dsum, dout, dk, dv, dq_acc, ws, tiles, st); break;
+    case 128: e = launch_bwd_dh<128>(p, q, offsets, k, v, lse, dsum, dout, dk, dv, dq_acc, ws, tiles, st); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess || rows == 0) return e;
+  KernelScope ks_("gdpa_dq_convert", st);
+  dq_convert_kernel<<<sms * 8, 256, 0, st>>>(reinterpret_cast<const float4*>(dq_acc),
+                                              reinterpret_cast<uint4*>(dq), rows * p.dh / 8,
+                                              p.scale);
+  return cudaGetLastError();
+}
+
+}  // namespace gdpa

@@ -30,6 +30,29 @@
 #include "sm100.cuh"
 
 namespace gdpa {
+
+// cuTensorMapEncodeTiled through the runtime's driver entry-point query (no
+// link-time dependency on libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
 namespace {
 
 using namespace sm100;
@@ -435,31 +458,11 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 
 // ------------------------------------------------------------------ host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-int num_sms() {
-  int dev = 0, n = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
-}
-
 template <int DH>
 bool make_maps(const gdpa_problem_t& p, const void* q, const void* k, const void* v,
                CUtensorMap* mq, CUtensorMap* mk, CUtensorMap* mv) {
   using C = FwdCfg<DH>;
-  auto enc = encode_fn();
+  auto enc = tensor_map_encoder();
   if (!enc) return false;
   const CUtensorMapSwizzle sw = DH < 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   const cuuint32_t estr[4] = {1, 1, 1, 1};
@@ -506,7 +509,7 @@ cudaError_t launch_fwd_t(const gdpa_problem_t& p, const void* q, const void* k, 
   args.scale = p.scale;
   args.scale_log2 = p.scale * 1.4426950408889634f;
   KernelScope ks_("gdpa_fwd_sm100", st);
-  kern<<<num_sms(), kThreads, C::SMEM, st>>>(mq, mk, mv, args);
+  kern<<<device_sm_count(), kThreads, C::SMEM, st>>>(mq, mk, mv, args);
   return cudaGetLastError();
 }
 

@@ -191,6 +191,19 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
+// Makes this thread's generic-proxy shared-memory writes visible to the async
+// proxy (tensor core / TMA reads that follow a barrier).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Four-wide fp32 reduction (add) to global memory, no return value.
+__device__ __forceinline__ void red_add_v4(float* gptr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(gptr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
 // ----------------------------------------------------------- misc math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
