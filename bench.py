@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--samples", type=int, default=0,
+                    help="run only the first N samples of the workload (small profiling case)")
     return ap.parse_args()
 
 
@@ -261,7 +263,8 @@ def main():
             dist.barrier()
 
     wl = syn.WORKLOADS[WORKLOAD]
-    d = syn.make_inputs(WORKLOAD, device=dev, seed=rank, backward=True)
+    subset = list(range(args.samples)) if 0 < args.samples < wl.B else None
+    d = syn.make_inputs(WORKLOAD, device=dev, seed=rank, backward=True, samples=subset)
     q, k, v, g = d["q"], d["k"], d["v"], d["dout"]
     T = int(d["offsets"][-1])
     off = torch.tensor(d["offsets"], dtype=torch.int32, device=dev)
@@ -383,8 +386,10 @@ def main():
               "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
               "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
               "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-              "config": {"workload": wl.name, "B": wl.B, "h": wl.h, "dh": wl.dh, "m": wl.m,
-                         "phi": wl.phi_name, "scale": wl.scale, "lengths": wl.lengths,
+              "config": {"workload": wl.name if subset is None else
+                         f"{wl.name} (first {len(subset)} samples only: profiling case)",
+                         "B": wl.B if subset is None else len(subset), "h": wl.h, "dh": wl.dh,
+                         "m": wl.m, "phi": wl.phi_name, "scale": wl.scale, "lengths": wl.lengths,
                          "tokens_per_rank": T, "parallelism": f"replicas x{world} (samples independent)",
                          "l2": "inputs (K, V 4.3 GB each) far larger than the 126 MB L2; no flush"},
               "pct_of_bf16_peak": 100.0 * value / (world * pk["bf16_sustained"]),
