@@ -159,6 +159,32 @@ typedef struct {
  */
 GDPA_API int32_t gdpa_timing_read(gdpa_kernel_time_t* out, int32_t cap);
 
+/*
+ * gdpa_fwd_no_alloc: gdpa_fwd for callers that cannot allocate device memory
+ * at call time (for example a host framework that has reserved all device
+ * memory for its own pool and gives plug-in operators no allocator, or a
+ * serving loop that cannot afford cudaMalloc's implicit synchronisation).
+ * The Kunlun pages have no counterpart of this call; it only moves gdpa_fwd's
+ * scratch out of the caller's hands.
+ *   Arguments as in gdpa_fwd, without the workspace: the caller passes inputs
+ *   and outputs only.  The scratch (status header + tile list) is a static
+ *   2 MiB device array inside the library, held by every device that loads
+ *   the library until the process exits.  Problems whose forward workspace
+ *   (gdpa_fwd_workspace_size) exceeds 2 MiB are rejected with
+ *   GDPA_ERR_WORKSPACE before any launch; that allows h * (T / r + B) <= 131,056
+ *   tiles, with r = 128 query rows per tile for bf16 and 64 for fp32.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture.  Allocates nothing: no cudaMalloc, cudaFree or allocating library
+ *   routine.  All calls share the one array, so calls that overlap on the GPU
+ *   (different streams, or different host threads, without ordering between
+ *   them) race on it and must be serialised by the caller.  The device status
+ *   of the last call is not readable through gdpa_workspace_status.
+ */
+GDPA_API gdpa_status_t gdpa_fwd_no_alloc(const gdpa_problem_t* p, const void* q,
+                                         const int32_t* offsets, const void* k, const void* v,
+                                         void* o, float* lse, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
