@@ -112,11 +112,14 @@ struct BwdCfg {
   static constexpr uint32_t DSB = 2 * 128 * 128;           // dS^T [128 keys][128 rows] bf16, SW128
   // TMEM columns
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + DH;
-  static constexpr uint32_t COL_DQ = DH <= 64 ? 256 + 2 * DH : COL_DP;
+  // dh <= 64: two dQ buffers of their own (the drain of step i-1 overlaps the
+  // MMAs of step i); dh = 128: one dQ buffer in the dP^T columns.
+  static constexpr bool DQ2 = DH <= 64;
+  static constexpr uint32_t COL_DQ = DQ2 ? 256 + 2 * DH : COL_DP;
   // barriers
   static constexpr int B_KVFULL = 0, B_KVEMPTY = 1, B_SFULL = 2, B_PFULL = 3, B_DQFULL = 4,
-                       B_DQEMPTY = 5, B_ACCFULL = 6, B_ACCEMPTY = 7, B_DRAIN = 8,
-                       B_STFULL = 9, B_STEMPTY = 9 + NSTG, NBAR = 9 + 2 * NSTG;
+                       B_DQEMPTY = 6, B_ACCFULL = 8, B_ACCEMPTY = 9, B_DRAIN = 10,
+                       B_STFULL = 11, B_STEMPTY = 11 + NSTG, NBAR = 11 + 2 * NSTG;
   static constexpr uint32_t OFF_K = 0, OFF_V = TILEB, OFF_STG = 2 * TILEB;
   static constexpr uint32_t OFF_DS = OFF_STG + NSTG * 2 * TILEB;
   static constexpr uint32_t OFF_CTL = OFF_DS + DSB;
@@ -156,8 +159,10 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     mbar_init(bar(C::B_KVEMPTY), 1);
     mbar_init(bar(C::B_SFULL), 1);
     mbar_init(bar(C::B_PFULL), 256);
-    mbar_init(bar(C::B_DQFULL), 1);
-    mbar_init(bar(C::B_DQEMPTY), 256);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::B_DQFULL + i), 1);
+      mbar_init(bar(C::B_DQEMPTY + i), 256);
+    }
     mbar_init(bar(C::B_ACCFULL), 1);
     mbar_init(bar(C::B_ACCEMPTY), 256);
     mbar_init(bar(C::B_DRAIN), 1);
@@ -249,8 +254,9 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                    smem_desc(qaddr + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW), IDESC_T,
                    k > 0 ? 1u : 0u);
           }
-          // dP^T = V dO_i^T; its columns (and dQ's) must have been drained
-          if (qs >= 1 && !mbar_wait(bar(C::B_DQEMPTY), (qs - 1) & 1u, abort_flag, kTimeoutNs)) {
+          // dP^T = V dO_i^T; with one dQ buffer in these columns, dQ_{i-1} must be drained
+          if (!C::DQ2 && qs >= 1 &&
+              !mbar_wait(bar(C::B_DQEMPTY), (qs - 1) & 1u, abort_flag, kTimeoutNs)) {
             ok = false;
             break;
           }
@@ -288,15 +294,22 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                    smem_desc(qaddr + k * 2 * C::ATOM, C::CHUNKB, C::ATOM, C::SW), IDESC_KV,
                    (!first || k > 0) ? 1u : 0u);
           }
-          // dQ_i = dS K
+          // dQ_i = dS K (into buffer qs % 2 when double-buffered, after its last drain)
+          const uint32_t dqb = C::DQ2 ? (qs & 1u) : 0u;
+          if (C::DQ2 && !mbar_wait(bar(C::B_DQEMPTY + dqb), ((qs >> 1) & 1u) ^ 1u, abort_flag,
+                                   kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            mma_ss(tmem + C::COL_DQ, smem_desc(sDS + k * 2048, 16384, 1024, kSw128),
+            mma_ss(tmem + C::COL_DQ + dqb * DH, smem_desc(sDS + k * 2048, 16384, 1024, kSw128),
                    smem_desc(sK + k * 2 * C::ATOM, C::CHUNKB, C::ATOM, C::SW), IDESC_Q,
                    k > 0 ? 1u : 0u);
           }
           mma_commit(bar(C::B_STEMPTY + stage));
-          mma_commit(bar(C::B_DQFULL));
+          mma_commit(bar(C::B_DQFULL + dqb));
           if (++stage == (uint32_t)C::NSTG) {
             stage = 0;
             sphase ^= 1u;
@@ -334,23 +347,58 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
       const int nq = (n + 127) >> 7;
       const int t0 = a.offsets[it.b];
+      // dQ_i drain: lane = query row of tile i; this group adds half of the columns
+      auto drain_dq = [&](int ii, uint32_t step) -> bool {
+        const uint32_t b = C::DQ2 ? (step & 1u) : 0u;
+        const uint32_t par = C::DQ2 ? ((step >> 1) & 1u) : (step & 1u);
+        const bool w = mbar_wait(bar(C::B_DQFULL + b), par, abort_flag, kTimeoutNs);
+        if (!__all_sync(0xffffffffu, w)) return false;
+        tc_fence_after();
+        const int rg = 128 * ii + lrow;
+        float* dst = a.dq_acc + ((int64_t)(t0 + rg) * a.h + it.head) * DH + grp * (DH / 2);
+#pragma unroll
+        for (int c = 0; c < DH / 2; c += 16) {
+          uint32_t v[16];
+          tmem_ld_x16(tmem + lane_off + C::COL_DQ + b * DH + grp * (DH / 2) + c, v);
+          tmem_wait_ld();
+          if (rg < n) {
+#pragma unroll
+            for (int u = 0; u < 16; u += 4)
+              red_add_v4(dst + c + u, __uint_as_float(v[u]), __uint_as_float(v[u + 1]),
+                         __uint_as_float(v[u + 2]), __uint_as_float(v[u + 3]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(C::B_DQEMPTY + b));
+        return true;
+      };
+      // softmax row statistics of a query tile, loaded one step ahead
+      float nl[2] = {0.f, 0.f}, nd[2] = {0.f, 0.f};
+      auto load_stats = [&](int ii) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int rg = 128 * ii + 64 * grp + 32 * u + lane;
+          nl[u] = 0.f;
+          nd[u] = 0.f;
+          if (rg < n) {
+            const int64_t at = (int64_t)it.head * a.T + t0 + rg;
+            nl[u] = a.lse[at] * 1.4426950408889634f;
+            nd[u] = a.dsum[at];
+          }
+        }
+      };
+      if constexpr (SOFTMAX) load_stats(0);
       for (int i = 0; i < nq; ++i, ++qs) {
         const int rbase = 128 * i + 64 * grp;          // first sample row of this group's half
         if constexpr (SOFTMAX) {
           __syncwarp();
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int r = 32 * u + lane, rg = rbase + r;
-            float l2 = 0.f, dd = 0.f;
-            if (rg < n) {
-              const int64_t at = (int64_t)it.head * a.T + t0 + rg;
-              l2 = a.lse[at] * 1.4426950408889634f;
-              dd = a.dsum[at];
-            }
-            wst[r] = l2;
-            wst[64 + r] = dd;
+            wst[32 * u + lane] = nl[u];
+            wst[64 + 32 * u + lane] = nd[u];
           }
           __syncwarp();
+          if (i + 1 < nq) load_stats(i + 1);
         }
         bool w = mbar_wait(bar(C::B_SFULL), qs & 1u, abort_flag, kTimeoutNs);
         if (!__all_sync(0xffffffffu, w)) {
@@ -411,32 +459,17 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar(C::B_PFULL));
-        // dQ_i: lane = query row of tile i; this group drains half of the columns
-        w = mbar_wait(bar(C::B_DQFULL), qs & 1u, abort_flag, kTimeoutNs);
-        if (!__all_sync(0xffffffffu, w)) {
+        if (!C::DQ2) {
+          if (!drain_dq(i, qs)) {
+            ok = false;
+            break;
+          }
+        } else if (i > 0 && !drain_dq(i - 1, qs - 1)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        {
-          const int rg = 128 * i + lrow;
-          float* dst = a.dq_acc + ((int64_t)(t0 + rg) * a.h + it.head) * DH + grp * (DH / 2);
-#pragma unroll
-          for (int c = 0; c < DH / 2; c += 16) {
-            uint32_t v[16];
-            tmem_ld_x16(tmem + lane_off + C::COL_DQ + grp * (DH / 2) + c, v);
-            tmem_wait_ld();
-            if (rg < n) {
-#pragma unroll
-              for (int u = 0; u < 16; u += 4)
-                red_add_v4(dst + c + u, __uint_as_float(v[u]), __uint_as_float(v[u + 1]),
-                           __uint_as_float(v[u + 2]), __uint_as_float(v[u + 3]));
-            }
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(bar(C::B_DQEMPTY));
       }
+      if (ok && C::DQ2 && !drain_dq(nq - 1, qs - 1)) ok = false;
       if (!ok) break;
       // ---------------------------------------------------------- dV / dK of this key block
       bool w = mbar_wait(bar(C::B_ACCFULL), ic & 1u, abort_flag, kTimeoutNs);

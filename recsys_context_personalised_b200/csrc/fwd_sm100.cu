@@ -285,19 +285,34 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           tmem_ld_x32(my_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
           tmem_ld_x32(my_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
           tmem_wait_ld();
-          float mx = c2 >= 0.f ? -INFINITY : INFINITY;
-          if (valid == C::BN) {
-            if (c2 >= 0.f) {
+          // row max (min when the scale is negative) over the valid columns, 8 independent chains
+          float mx;
+          {
+            const float ident = c2 >= 0.f ? -INFINITY : INFINITY;
+            float m8[8];
 #pragma unroll
-              for (int i = 0; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+            for (int u = 0; u < 8; ++u) m8[u] = ident;
+            if (valid == C::BN) {
+              if (c2 >= 0.f) {
+#pragma unroll
+                for (int i = 0; i < 128; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(s[i]));
+              } else {
+#pragma unroll
+                for (int i = 0; i < 128; ++i) m8[i & 7] = fminf(m8[i & 7], __uint_as_float(s[i]));
+              }
             } else {
 #pragma unroll
-              for (int i = 0; i < 128; ++i) mx = fminf(mx, __uint_as_float(s[i]));
+              for (int i = 0; i < 128; ++i)
+                if (i < valid)
+                  m8[i & 7] = c2 >= 0.f ? fmaxf(m8[i & 7], __uint_as_float(s[i]))
+                                        : fminf(m8[i & 7], __uint_as_float(s[i]));
             }
-          } else {
 #pragma unroll
-            for (int i = 0; i < 128; ++i)
-              if (i < valid) mx = c2 >= 0.f ? fmaxf(mx, __uint_as_float(s[i])) : fminf(mx, __uint_as_float(s[i]));
+            for (int u = 4; u > 0; u >>= 1)
+#pragma unroll
+              for (int v = 0; v < u; ++v)
+                m8[v] = c2 >= 0.f ? fmaxf(m8[v], m8[v + u]) : fminf(m8[v], m8[v + u]);
+            mx = m8[0];
           }
           const float m_new = mx * c2;
           float alpha = 1.f;
@@ -310,7 +325,7 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             resc = true;
           }
           const float neg_m = -m_run;
-          float rs = 0.f;
+          float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           uint32_t pk[64];
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
@@ -320,9 +335,11 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
               p0 = (2 * i < valid) ? p0 : 0.f;
               p1 = (2 * i + 1 < valid) ? p1 : 0.f;
             }
-            rs += p0 + p1;
+            rs8[(2 * i) & 7] += p0;
+            rs8[(2 * i + 1) & 7] += p1;
             pk[i] = pack_bf16x2(p0, p1);
           }
+          const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
           tmem_st_x32(my_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
           tmem_st_x32(my_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
           l_run = l_run * alpha + rs;
