@@ -126,6 +126,7 @@ struct BwdCfg {
   static constexpr uint32_t CTL_BYTES = 1024 + 8 * 2 * 128 * 4;  // barriers + per-warp row stats
   static constexpr uint32_t SMEM_USED = 1024 + OFF_CTL + CTL_BYTES;
   static constexpr uint32_t SMEM = SMEM_USED > 120u * 1024u ? SMEM_USED : 120u * 1024u;
+  static_assert(SMEM <= 232448u, "exceeds the 227 KB of shared memory a CTA can have");
 };
 
 template <int DH, int PHI>

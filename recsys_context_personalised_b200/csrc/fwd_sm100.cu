@@ -3,26 +3,29 @@
 // Operator (Kunlun summary, section 2.2, GDPA bullet: PFFN recast as a
 // multi-head attention operator fused into one FlashAttention-like kernel;
 // RecSysChannel review "Kunlun ... [2/2]", items 1-2: K and V come from the
-// context features, the event sequence is turned into Q).  Per work tile
-// (sample b, head j, up to 128 query rows) and per 128-key block:
+// context features, the event sequence is turned into Q).  Per query tile
+// (sample b, head j, up to 128 rows) and per 128-key block:
 //   S = Q K^T            tcgen05.mma, A and B from shared memory, S in TMEM
 //   P = phi(s S)         activation warps: TMEM -> registers -> TMEM (bf16)
 //   O += P V             tcgen05.mma, A = P from TMEM, B = V from shared memory
-// softmax keeps running row statistics (online softmax, rescaling only when the
-// running max grows by more than 2^8); the elementwise phi needs none.
+// softmax keeps running row statistics (online softmax, rescaling O only when
+// the running max grows by more than 2^8); the elementwise phi needs none.
 //
-// CTA = 12 warps, one persistent CTA per SM, static round-robin over the tile list:
-//   warp 0      TMA producer (one lane): Q tile, then K_0, K_1, V_0, K_2, V_1, ...
+// Each work item is a pair of consecutive tiles of the jagged tile list, A and
+// B, processed side by side: the MMA issuer interleaves their two dependency
+// chains (S_A, S_B, PV_A, S_A', PV_B, S_B', ...) so the tensor core always has
+// the other tile's work queued while one tile's activation runs.  When A and B
+// belong to the same (sample, head) they share every K/V block load; otherwise
+// each streams its own.
+//
+// CTA = 12 warps, one persistent CTA per SM, static round-robin over the pairs:
+//   warp 0      TMA producer (one lane)
 //   warp 1      MMA issuer (one lane)
 //   warp 2      TMEM allocator
-//   warps 4-7   activation group 0: key blocks with even global step
-//   warps 8-11  activation group 1: odd steps
-// The two activation groups alternate so that one computes phi while the
-// tensor core runs the other's MMAs.  For softmax each group owns its own
-// statistics and O accumulator (O_0, O_1), combined in the epilogue.
+//   warps 4-7   activation group A (tile A), warps 8-11 group B (tile B)
 //
-// TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256) (P_b aliases the
-// first 64 columns of S_b as packed bf16), O_0 [256, 256+dh), O_1 [256+dh, 256+2dh).
+// TMEM columns (512 allocated): S_A [0,128), S_B [128,256) (P_X aliases the
+// first 64 columns of S_X as packed bf16), O_A [256, 256+dh), O_B [256+dh, 256+2dh).
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -81,21 +84,39 @@ struct FwdCfg {
   static constexpr uint32_t TILEB = NCH * CHUNKB;       // 128 * DH * 2
   static constexpr uint32_t SW = DH < 64 ? kSw64 : kSw128;
   static constexpr uint32_t ATOM = 8 * ROWB;            // 8-row group stride
-  static constexpr int NS = DH == 32 ? 8 : (DH == 64 ? 6 : 4);
-  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + DH;
+  static constexpr int QST = DH == 128 ? 1 : 2;         // Q stages (a stage = tiles A and B)
+  static constexpr int NS = DH == 32 ? 16 : (DH == 64 ? 8 : 4);   // K/V ring slots
+  static constexpr uint32_t COL_S = 0, COL_O = 256;     // + 128*X, + DH*X for tile X
   // barrier slots
   static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_SFULL = 4, B_PFULL = 6, B_OFULL = 8,
-                       B_OEMPTY = 9, B_DRAIN = 10, B_STATS = 11, B_KVFULL = 12,
-                       B_KVEMPTY = 12 + NS, NBAR = 12 + 2 * NS;
-  static constexpr uint32_t CTL_BYTES = 4096;
-  static constexpr uint32_t SMEM_USED = 1024 + (2 + NS) * TILEB + CTL_BYTES;
+                       B_OEMPTY = 10, B_DRAIN = 12, B_KVFULL = 13, B_KVEMPTY = 13 + NS,
+                       NBAR = 13 + 2 * NS;
+  static constexpr uint32_t OFF_Q = 0, OFF_KV = QST * 2 * TILEB;
+  static constexpr uint32_t CTL_BYTES = 1024;
+  static constexpr uint32_t SMEM_USED = 1024 + OFF_KV + NS * TILEB + CTL_BYTES;
   // at least 120 KB so that two CTAs never share an SM (each allocates all 512 TMEM columns)
   static constexpr uint32_t SMEM = SMEM_USED > 120u * 1024u ? SMEM_USED : 120u * 1024u;
+  static_assert(SMEM <= 232448u, "exceeds the 227 KB of shared memory a CTA can have");
+  static_assert(8 * NBAR + 8 <= CTL_BYTES, "control block too small");
 };
 
 __device__ __forceinline__ float silu_tanh(float s, float half_scale) {
   const float hx = s * half_scale;                 // x/2 with x = s * scale
   return fmaf(hx, tanh_approx(hx), hx);             // x/2 * (1 + tanh(x/2)) = x * logistic(x)
+}
+
+// Work item p = tiles 2p (A) and 2p+1 (B, absent past the end of the list).
+struct Pair {
+  Tile a, b;
+  bool has_b, share;   // share: same (sample, head), so the K/V blocks are common
+};
+__device__ __forceinline__ Pair load_pair(const Tile* tiles, int count, int p) {
+  Pair r;
+  r.a = tiles[2 * p];
+  r.has_b = 2 * p + 1 < count;
+  r.b = r.has_b ? tiles[2 * p + 1] : r.a;
+  r.share = !r.has_b || (r.a.b == r.b.b && r.a.head == r.b.head);
+  return r;
 }
 
 template <int DH, int PHI>
@@ -112,15 +133,13 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t sQ = base;
-  const uint32_t sKV = base + 2 * C::TILEB;
-  uint8_t* ctl = gbase + (2 + C::NS) * C::TILEB;
+  const uint32_t sQ = base + C::OFF_Q;
+  const uint32_t sKV = base + C::OFF_KV;
+  uint8_t* ctl = gbase + C::OFF_KV + C::NS * C::TILEB;
   const uint32_t bar0 = smem_u32(ctl);
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 8 * C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 8 * C::NBAR + 4);
-  float* st_m = reinterpret_cast<float*>(ctl + 1024);         // [2][128]
-  float* st_l = st_m + 256;                                   // [2][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -129,11 +148,10 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       mbar_init(bar(C::B_QEMPTY + i), 1);
       mbar_init(bar(C::B_SFULL + i), 1);
       mbar_init(bar(C::B_PFULL + i), 128);
+      mbar_init(bar(C::B_OFULL + i), 1);
+      mbar_init(bar(C::B_OEMPTY + i), 128);
     }
-    mbar_init(bar(C::B_OFULL), 1);
-    mbar_init(bar(C::B_OEMPTY), 256);
     mbar_init(bar(C::B_DRAIN), 1);
-    mbar_init(bar(C::B_STATS), 256);
     for (int i = 0; i < C::NS; ++i) {
       mbar_init(bar(C::B_KVFULL + i), 1);
       mbar_init(bar(C::B_KVEMPTY + i), 1);
@@ -155,12 +173,14 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int count = a.ws->tile_count;
+  const int npairs = (count + 1) >> 1;
   const int nkv = a.nkv;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t tc = 0, slot = 0, sphase = 0;
+      uint32_t ic = 0, slot = 0, sphase = 0;
+      bool ok = true;
       auto load_kv = [&](const CUtensorMap* map, const Tile& tl, int j) -> bool {
         if (!mbar_wait(bar(C::B_KVEMPTY + slot), sphase ^ 1u, abort_flag, kTimeoutNs)) return false;
         mbar_expect_tx(bar(C::B_KVFULL + slot), C::TILEB);
@@ -174,104 +194,163 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         return true;
       };
-      for (int t = blockIdx.x; t < count; t += gridDim.x, ++tc) {
-        const Tile tl = a.tiles[t];
-        const uint32_t qb = tc & 1u;
-        if (!mbar_wait(bar(C::B_QEMPTY + qb), ((tc >> 1) & 1u) ^ 1u, abort_flag, kTimeoutNs)) break;
-        mbar_expect_tx(bar(C::B_QFULL + qb), C::TILEB);
+      for (int p = blockIdx.x; ok && p < npairs; p += gridDim.x, ++ic) {
+        const Pair pr = load_pair(a.tiles, count, p);
+        const uint32_t qs = ic % C::QST, qph = (ic / C::QST) & 1u;
+        if (!mbar_wait(bar(C::B_QEMPTY + qs), qph ^ 1u, abort_flag, kTimeoutNs)) break;
+        const uint32_t qaddr = sQ + qs * 2 * C::TILEB;
+        mbar_expect_tx(bar(C::B_QFULL + qs), (pr.has_b ? 2u : 1u) * C::TILEB);
 #pragma unroll
-        for (int c = 0; c < C::NCH; ++c)
-          tma_load_3d(sQ + qb * C::TILEB + c * C::CHUNKB, &tmQ, bar(C::B_QFULL + qb), c * C::CH,
-                      tl.head, tl.row0);
-        bool ok = load_kv(&tmK, tl, 0);
-        for (int j = 1; ok && j < nkv; ++j) ok = load_kv(&tmK, tl, j) && load_kv(&tmV, tl, j - 1);
-        ok = ok && load_kv(&tmV, tl, nkv - 1);
-        if (!ok) break;
+        for (int c = 0; c < C::NCH; ++c) {
+          tma_load_3d(qaddr + c * C::CHUNKB, &tmQ, bar(C::B_QFULL + qs), c * C::CH, pr.a.head,
+                      pr.a.row0);
+          if (pr.has_b)
+            tma_load_3d(qaddr + C::TILEB + c * C::CHUNKB, &tmQ, bar(C::B_QFULL + qs), c * C::CH,
+                        pr.b.head, pr.b.row0);
+        }
+        // K/V blocks in the order of their first use by the MMA issuer
+        if (pr.share) {
+          for (int j = 0; ok && j < nkv; ++j)
+            ok = load_kv(&tmK, pr.a, j) && load_kv(&tmV, pr.a, j);
+        } else {
+          ok = load_kv(&tmK, pr.a, 0) && load_kv(&tmK, pr.b, 0);
+          for (int j = 0; ok && j < nkv; ++j) {
+            ok = load_kv(&tmV, pr.a, j);
+            if (ok && j + 1 < nkv) ok = load_kv(&tmK, pr.a, j + 1);
+            if (ok) ok = load_kv(&tmV, pr.b, j);
+            if (ok && j + 1 < nkv) ok = load_kv(&tmK, pr.b, j + 1);
+          }
+        }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t tc = 0, slot = 0, sphase = 0, g = 0;
+      uint32_t ic = 0, slot = 0, sphase = 0;
+      uint32_t pc[2] = {0u, 0u};   // PV groups issued per tile slot (P barrier phase)
+      uint32_t oc[2] = {0u, 0u};   // items finished per tile slot (O barrier phase)
       bool ok = true;
-      auto next_slot = [&]() {
+      // next K/V ring slot, in the producer's load order
+      auto take = [&]() -> int {
+        if (!mbar_wait(bar(C::B_KVFULL + slot), sphase, abort_flag, kTimeoutNs)) return -1;
+        tc_fence_after();
+        const int s = (int)slot;
         if (++slot == (uint32_t)C::NS) {
           slot = 0;
           sphase ^= 1u;
         }
+        return s;
       };
-      for (int t = blockIdx.x; ok && t < count; t += gridDim.x, ++tc) {
-        const uint32_t qb = tc & 1u;
-        if (!mbar_wait(bar(C::B_QFULL + qb), (tc >> 1) & 1u, abort_flag, kTimeoutNs)) break;
+      for (int p = blockIdx.x; ok && p < npairs; p += gridDim.x, ++ic) {
+        const Pair pr = load_pair(a.tiles, count, p);
+        const uint32_t qs = ic % C::QST, qph = (ic / C::QST) & 1u;
+        if (!mbar_wait(bar(C::B_QFULL + qs), qph, abort_flag, kTimeoutNs)) break;
         tc_fence_after();
-        const uint32_t qaddr = sQ + qb * C::TILEB;
-        // O += P_i V_i for key block i at global step gi
-        auto issue_pv = [&](int i, uint32_t gi) -> bool {
-          const uint32_t bi = gi & 1u;
-          if (!mbar_wait(bar(C::B_PFULL + bi), (gi >> 1) & 1u, abort_flag, kTimeoutNs)) return false;
-          if (i == 0 && !mbar_wait(bar(C::B_OEMPTY), (tc & 1u) ^ 1u, abort_flag, kTimeoutNs))
-            return false;
-          if (!mbar_wait(bar(C::B_KVFULL + slot), sphase, abort_flag, kTimeoutNs)) return false;
-          tc_fence_after();
-          const uint32_t vaddr = sKV + slot * C::TILEB;
-          const uint32_t ocol = (SOFTMAX && bi) ? C::COL_O1 : C::COL_O0;
-          const bool first = SOFTMAX ? (i < 2) : (i == 0);
-          const uint32_t pcol = bi ? C::COL_S1 : C::COL_S0;
-#pragma unroll
-          for (int k = 0; k < C::BN / 16; ++k) {
-            const uint64_t bdesc = smem_desc(vaddr + k * 2 * C::ATOM, C::CHUNKB, C::ATOM, C::SW);
-            mma_ts(tmem + ocol, tmem + pcol + k * 8, bdesc, IDESC_O, (!first || k > 0) ? 1u : 0u);
-          }
-          mma_commit(bar(C::B_KVEMPTY + slot));
-          next_slot();
-          return true;
-        };
-        for (int j = 0; ok && j < nkv; ++j, ++g) {
-          if (!mbar_wait(bar(C::B_KVFULL + slot), sphase, abort_flag, kTimeoutNs)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t kaddr = sKV + slot * C::TILEB;
-          const uint32_t buf = g & 1u;
-          const uint32_t scol = buf ? C::COL_S1 : C::COL_S0;
+        const uint32_t qbase = sQ + qs * 2 * C::TILEB;
+        const int last_x = pr.has_b ? 1 : 0;
+        const bool sep = !pr.share;              // A and B each have their own K/V slots
+        // S_X(j) = Q_X K^T into S_X; the last S of the pair frees the Q stage
+        auto issue_s = [&](int x, int ks, int j) {
+          const uint32_t qaddr = qbase + x * C::TILEB, kaddr = sKV + ks * C::TILEB;
 #pragma unroll
           for (int k = 0; k < DH / 16; ++k) {
             const int c = k / (C::CH / 16), kk = k % (C::CH / 16);
-            const uint64_t adesc = smem_desc(qaddr + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW);
-            const uint64_t bdesc = smem_desc(kaddr + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW);
-            mma_ss(tmem + scol, adesc, bdesc, IDESC_S, k > 0 ? 1u : 0u);
+            mma_ss(tmem + C::COL_S + 128 * x,
+                   smem_desc(qaddr + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW),
+                   smem_desc(kaddr + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW), IDESC_S,
+                   k > 0 ? 1u : 0u);
           }
-          mma_commit(bar(C::B_KVEMPTY + slot));
-          mma_commit(bar(C::B_SFULL + buf));
-          if (j == nkv - 1) mma_commit(bar(C::B_QEMPTY + qb));
-          next_slot();
-          if (j >= 1) ok = issue_pv(j - 1, g - 1);
+          mma_commit(bar(C::B_SFULL + x));
+          if (x == last_x && j == nkv - 1) mma_commit(bar(C::B_QEMPTY + qs));
+        };
+        // O_X += P_X(j) V_j once the activation group has written P_X(j)
+        auto issue_pv = [&](int x, int vs, int j) -> bool {
+          if (!mbar_wait(bar(C::B_PFULL + x), pc[x] & 1u, abort_flag, kTimeoutNs)) return false;
+          ++pc[x];
+          if (j == 0 && !mbar_wait(bar(C::B_OEMPTY + x), (oc[x] & 1u) ^ 1u, abort_flag, kTimeoutNs))
+            return false;
+          tc_fence_after();
+          const uint32_t vaddr = sKV + vs * C::TILEB;
+#pragma unroll
+          for (int k = 0; k < C::BN / 16; ++k)
+            mma_ts(tmem + C::COL_O + DH * x, tmem + C::COL_S + 128 * x + k * 8,
+                   smem_desc(vaddr + k * 2 * C::ATOM, C::CHUNKB, C::ATOM, C::SW), IDESC_O,
+                   (j > 0 || k > 0) ? 1u : 0u);
+          if (j == nkv - 1) {
+            mma_commit(bar(C::B_OFULL + x));
+            ++oc[x];
+          }
+          return true;
+        };
+        auto release = [&](int s) { mma_commit(bar(C::B_KVEMPTY + s)); };
+
+        int ka = take();
+        if (ka < 0) break;
+        issue_s(0, ka, 0);
+        if (!pr.has_b || sep) release(ka);
+        if (pr.has_b) {
+          const int kb = sep ? take() : ka;
+          if (kb < 0) break;
+          issue_s(1, kb, 0);
+          release(kb);
         }
-        if (ok) ok = issue_pv(nkv - 1, g - 1);
-        if (ok) mma_commit(bar(C::B_OFULL));
+        for (int j = 0; ok && j < nkv; ++j) {
+          const int va = take();
+          if (va < 0 || !issue_pv(0, va, j)) {
+            ok = false;
+            break;
+          }
+          if (!pr.has_b || sep) release(va);
+          int kn = -1;
+          if (j + 1 < nkv) {
+            kn = take();
+            if (kn < 0) {
+              ok = false;
+              break;
+            }
+            issue_s(0, kn, j + 1);
+            if (!pr.has_b || sep) release(kn);
+          }
+          if (pr.has_b) {
+            const int vb = sep ? take() : va;
+            if (vb < 0 || !issue_pv(1, vb, j)) {
+              ok = false;
+              break;
+            }
+            release(vb);
+            if (j + 1 < nkv) {
+              const int kb = sep ? take() : kn;
+              if (kb < 0) {
+                ok = false;
+                break;
+              }
+              issue_s(1, kb, j + 1);
+              release(kb);
+            }
+          }
+        }
       }
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ activation groups
-    const int grp = (warp - 4) >> 2;            // 0 or 1
+    const int grp = (warp - 4) >> 2;            // tile slot: 0 = A, 1 = B
     const int quad = warp & 3;                  // TMEM lane quadrant
     const int row = quad * 32 + lane;           // tile row owned by this thread
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t my_s = tmem + lane_off + (grp ? C::COL_S1 : C::COL_S0);
+    const uint32_t my_s = tmem + lane_off + C::COL_S + 128 * grp;
+    const uint32_t my_o = tmem + lane_off + C::COL_O + DH * grp;
     const float c2 = a.scale_log2;
     const float half_scale = 0.5f * a.scale;
-    uint32_t tc = 0, g = 0;
+    uint32_t sc = 0, oc = 0;
     bool ok = true;
-    for (int t = blockIdx.x; ok && t < count; t += gridDim.x, ++tc) {
-      const Tile tl = a.tiles[t];
-      const uint32_t g0 = g;
+    for (int p = blockIdx.x; ok && p < npairs; p += gridDim.x) {
+      const Pair pr = load_pair(a.tiles, count, p);
+      if (grp == 1 && !pr.has_b) continue;
+      const Tile tl = grp ? pr.b : pr.a;
       float m_run = -INFINITY, l_run = 0.f;
       int steps = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const uint32_t gj = g0 + j;
-        if ((int)(gj & 1u) != grp) continue;
-        bool w = mbar_wait(bar(C::B_SFULL + grp), (gj >> 1) & 1u, abort_flag, kTimeoutNs);
+      for (int j = 0; j < nkv; ++j, ++sc) {
+        bool w = mbar_wait(bar(C::B_SFULL + grp), sc & 1u, abort_flag, kTimeoutNs);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
@@ -344,8 +423,7 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           tmem_st_x32(my_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
           l_run = l_run * alpha + rs;
           if (__any_sync(0xffffffffu, resc)) {
-            const uint32_t my_o = tmem + lane_off + (grp ? C::COL_O1 : C::COL_O0);
-#pragma unroll
+            #pragma unroll
             for (int c = 0; c < DH; c += 16) {
               uint32_t ov[16];
               tmem_ld_x16(my_o + c, ov);
@@ -385,69 +463,36 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         ++steps;
       }
       if (!ok) break;
-      g = g0 + nkv;
       // ---------------------------------------------------------- epilogue
-      bool w = mbar_wait(bar(C::B_OFULL), tc & 1u, abort_flag, kTimeoutNs);
+      bool w = mbar_wait(bar(C::B_OFULL + grp), oc & 1u, abort_flag, kTimeoutNs);
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const bool has0 = nkv >= 2 || (g0 & 1u) == 0;
-      const bool has1 = nkv >= 2 || (g0 & 1u) == 1;
-      float f0 = 1.f, f1 = 0.f, inv = 1.f, M = 0.f, L = 1.f;
-      if constexpr (SOFTMAX) {
-        st_m[grp * 128 + row] = steps ? m_run : -INFINITY;
-        st_l[grp * 128 + row] = l_run;
-        mbar_arrive(bar(C::B_STATS));
-        w = mbar_wait(bar(C::B_STATS), tc & 1u, abort_flag, kTimeoutNs);
-        if (!__all_sync(0xffffffffu, w)) {
-          ok = false;
-          break;
-        }
-        const float m0 = st_m[row], m1 = st_m[128 + row];
-        const float l0 = st_l[row], l1 = st_l[128 + row];
-        M = fmaxf(m0, m1);
-        f0 = has0 ? ex2_approx(m0 - M) : 0.f;
-        f1 = has1 ? ex2_approx(m1 - M) : 0.f;
-        L = l0 * f0 + l1 * f1;
-        inv = 1.f / L;
-        f0 *= inv;
-        f1 *= inv;
-      }
-      const int col0 = grp * (DH / 2);
+      const float inv = SOFTMAX ? 1.f / l_run : 1.f;
       const bool store = row < tl.rows;
-      __nv_bfloat16* orow = a.o + ((int64_t)(tl.row0 + row) * a.h + tl.head) * DH + col0;
+      __nv_bfloat16* orow = a.o + ((int64_t)(tl.row0 + row) * a.h + tl.head) * DH;
 #pragma unroll
-      for (int c = 0; c < DH / 2; c += 16) {
-        uint32_t v0[16], v1[16];
-        tmem_ld_x16(tmem + lane_off + C::COL_O0 + col0 + c, v0);
-        if (SOFTMAX && has1) tmem_ld_x16(tmem + lane_off + C::COL_O1 + col0 + c, v1);
+      for (int c = 0; c < DH; c += 16) {
+        uint32_t v[16];
+        tmem_ld_x16(my_o + c, v);
         tmem_wait_ld();
         uint32_t pk[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float a0 = __uint_as_float(v0[2 * i]), a1 = __uint_as_float(v0[2 * i + 1]);
-          if constexpr (SOFTMAX) {
-            a0 = has0 ? a0 * f0 : 0.f;
-            a1 = has0 ? a1 * f0 : 0.f;
-            if (has1) {
-              a0 = fmaf(__uint_as_float(v1[2 * i]), f1, a0);
-              a1 = fmaf(__uint_as_float(v1[2 * i + 1]), f1, a1);
-            }
-          }
-          pk[i] = pack_bf16x2(a0, a1);
-        }
+        for (int i = 0; i < 8; ++i)
+          pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv, __uint_as_float(v[2 * i + 1]) * inv);
         if (store) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c);
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
-      if (SOFTMAX && grp == 0 && store && a.lse != nullptr)
-        a.lse[(int64_t)tl.head * a.T + tl.row0 + row] = (M + __log2f(L)) * 0.69314718055994531f;
+      if (SOFTMAX && store && a.lse != nullptr)
+        a.lse[(int64_t)tl.head * a.T + tl.row0 + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
       tc_fence_before();
-      mbar_arrive(bar(C::B_OEMPTY));
+      mbar_arrive(bar(C::B_OEMPTY + grp));
+      ++oc;
     }
   }
 

@@ -84,6 +84,17 @@ def test_small_jagged(case, phi, dh, dtype):
     check(out, d, phi, scale, True, dtype, f"n={n} m={m}")
 
 
+@pytest.mark.parametrize("phi", ["identity", "silu", "softmax"])
+@pytest.mark.parametrize("n", [[100], [300, 7], [129, 0, 640]])
+def test_odd_head_count(n, phi):
+    """h = 3: the work list can hold an odd number of tiles and mixes tiles of
+    different (sample, head) in one CTA work item."""
+    d = syn.random_problem(21, len(n), 3, 64, 300, n, dtype=torch.bfloat16, std=0.6)
+    scale = 0.125 if phi == "softmax" else 0.5
+    out = run_gpu(d, phi, scale, True)
+    check(out, d, phi, scale, True, torch.bfloat16, f"h=3 n={n}")
+
+
 def check_single_key_softmax(out, d, scale, tol):
     """Softmax over one key: P = 1, so dS = dP - D = 0 and dQ = dK = 0 exactly.
 
