@@ -247,12 +247,15 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           }
           tc_fence_after();
           const uint32_t qaddr = sStg + stage * 2 * C::TILEB, gaddr = qaddr + C::TILEB;
+          // descriptors built once per group: between two MMAs (whose issue waits
+          // for the tensor core) only a constant add remains
+          const uint64_t dk0 = smem_desc(sK, 16, C::ATOM, C::SW), dv0 = smem_desc(sV, 16, C::ATOM, C::SW);
+          const uint64_t dq0 = smem_desc(qaddr, 16, C::ATOM, C::SW), dg0 = smem_desc(gaddr, 16, C::ATOM, C::SW);
           // S^T = K Q_i^T
 #pragma unroll
           for (int k = 0; k < DH / 16; ++k) {
-            const int c = k / (C::CH / 16), kk = k % (C::CH / 16);
-            mma_ss(tmem + C::COL_S, smem_desc(sK + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW),
-                   smem_desc(qaddr + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW), IDESC_T,
+            const uint32_t off = (k / (C::CH / 16)) * C::CHUNKB + (k % (C::CH / 16)) * 32;
+            mma_ss(tmem + C::COL_S, desc_advance(dk0, off), desc_advance(dq0, off), IDESC_T,
                    k > 0 ? 1u : 0u);
           }
           // dP^T = V dO_i^T; with one dQ buffer in these columns, dQ_{i-1} must be drained
@@ -264,9 +267,8 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < DH / 16; ++k) {
-            const int c = k / (C::CH / 16), kk = k % (C::CH / 16);
-            mma_ss(tmem + C::COL_DP, smem_desc(sV + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW),
-                   smem_desc(gaddr + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW), IDESC_T,
+            const uint32_t off = (k / (C::CH / 16)) * C::CHUNKB + (k % (C::CH / 16)) * 32;
+            mma_ss(tmem + C::COL_DP, desc_advance(dv0, off), desc_advance(dg0, off), IDESC_T,
                    k > 0 ? 1u : 0u);
           }
           mma_commit(bar(C::B_SFULL));
@@ -279,22 +281,22 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             break;
           }
           tc_fence_after();
-          const uint32_t first = i == 0;
+          const uint32_t acc0 = i == 0 ? 0u : 1u;
+          const uint64_t gmn0 = smem_desc(gaddr, C::CHUNKB, C::ATOM, C::SW);   // dO_i, MN-major
+          const uint64_t qmn0 = smem_desc(qaddr, C::CHUNKB, C::ATOM, C::SW);   // Q_i, MN-major
+          const uint64_t dsk0 = smem_desc(sDS, 16, 1024, kSw128);              // dS^T, K-major
           // dV += P^T dO_i   (P^T rows 0-63 in columns 0-31, rows 64-127 in 64-95)
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const uint32_t acol = C::COL_S + (k < 4 ? 8 * k : 64 + 8 * (k - 4));
-            mma_ts(tmem + C::COL_DV, tmem + acol,
-                   smem_desc(gaddr + k * 2 * C::ATOM, C::CHUNKB, C::ATOM, C::SW), IDESC_KV,
-                   (!first || k > 0) ? 1u : 0u);
+            mma_ts(tmem + C::COL_DV, tmem + acol, desc_advance(gmn0, k * 2 * C::ATOM), IDESC_KV,
+                   k > 0 ? 1u : acc0);
           }
           // dK += dS^T Q_i
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            mma_ss(tmem + C::COL_DK, smem_desc(sDS + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSw128),
-                   smem_desc(qaddr + k * 2 * C::ATOM, C::CHUNKB, C::ATOM, C::SW), IDESC_KV,
-                   (!first || k > 0) ? 1u : 0u);
-          }
+          for (int k = 0; k < 8; ++k)
+            mma_ss(tmem + C::COL_DK, desc_advance(dsk0, (k >> 2) * 16384 + (k & 3) * 32),
+                   desc_advance(qmn0, k * 2 * C::ATOM), IDESC_KV, k > 0 ? 1u : acc0);
           // dQ_i = dS K (into buffer qs % 2 when double-buffered, after its last drain)
           const uint32_t dqb = C::DQ2 ? (qs & 1u) : 0u;
           if (C::DQ2 && !mbar_wait(bar(C::B_DQEMPTY + dqb), ((qs >> 1) & 1u) ^ 1u, abort_flag,
@@ -303,12 +305,12 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             break;
           }
           tc_fence_after();
+          const uint64_t dsm0 = smem_desc(sDS, 16384, 1024, kSw128);           // dS, MN-major
+          const uint64_t kmn0 = smem_desc(sK, C::CHUNKB, C::ATOM, C::SW);      // K, MN-major
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            mma_ss(tmem + C::COL_DQ + dqb * DH, smem_desc(sDS + k * 2048, 16384, 1024, kSw128),
-                   smem_desc(sK + k * 2 * C::ATOM, C::CHUNKB, C::ATOM, C::SW), IDESC_Q,
-                   k > 0 ? 1u : 0u);
-          }
+          for (int k = 0; k < 8; ++k)
+            mma_ss(tmem + C::COL_DQ + dqb * DH, desc_advance(dsm0, k * 2048),
+                   desc_advance(kmn0, k * 2 * C::ATOM), IDESC_Q, k > 0 ? 1u : 0u);
           mma_commit(bar(C::B_STEMPTY + stage));
           mma_commit(bar(C::B_DQFULL + dqb));
           if (++stage == (uint32_t)C::NSTG) {

@@ -87,6 +87,10 @@ struct FwdCfg {
   static constexpr int QST = DH == 128 ? 1 : 2;         // Q stages (a stage = tiles A and B)
   static constexpr int NS = DH == 32 ? 16 : (DH == 64 ? 8 : 4);   // K/V ring slots
   static constexpr uint32_t COL_S = 0, COL_O = 256;     // + 128*X, + DH*X for tile X
+  // dh <= 64: P_X has columns of its own, [384 + 64X, 448 + 64X); dh = 128: P_X
+  // aliases the first 64 columns of S_X
+  static constexpr bool P_SEP = DH <= 64;
+  static constexpr uint32_t COL_P = P_SEP ? 384 : COL_S;  // + 64*X (P_SEP) or + 128*X
   // barrier slots
   static constexpr int B_QFULL = 0, B_QEMPTY = 2, B_SFULL = 4, B_PFULL = 6, B_OFULL = 8,
                        B_OEMPTY = 10, B_DRAIN = 12, B_KVFULL = 13, B_KVEMPTY = 13 + NS,
@@ -251,14 +255,15 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         const bool sep = !pr.share;              // A and B each have their own K/V slots
         // S_X(j) = Q_X K^T into S_X; the last S of the pair frees the Q stage
         auto issue_s = [&](int x, int ks, int j) {
-          const uint32_t qaddr = qbase + x * C::TILEB, kaddr = sKV + ks * C::TILEB;
+          // descriptors built once per group: between two MMAs (whose issue waits
+          // for the tensor core) only a constant add remains
+          const uint64_t a0 = smem_desc(qbase + x * C::TILEB, 16, C::ATOM, C::SW);
+          const uint64_t b0 = smem_desc(sKV + ks * C::TILEB, 16, C::ATOM, C::SW);
+          const uint32_t dcol = tmem + C::COL_S + 128 * x;
 #pragma unroll
           for (int k = 0; k < DH / 16; ++k) {
-            const int c = k / (C::CH / 16), kk = k % (C::CH / 16);
-            mma_ss(tmem + C::COL_S + 128 * x,
-                   smem_desc(qaddr + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW),
-                   smem_desc(kaddr + c * C::CHUNKB + kk * 32, 16, C::ATOM, C::SW), IDESC_S,
-                   k > 0 ? 1u : 0u);
+            const uint32_t off = (k / (C::CH / 16)) * C::CHUNKB + (k % (C::CH / 16)) * 32;
+            mma_ss(dcol, desc_advance(a0, off), desc_advance(b0, off), IDESC_S, k > 0 ? 1u : 0u);
           }
           mma_commit(bar(C::B_SFULL + x));
           if (x == last_x && j == nkv - 1) mma_commit(bar(C::B_QEMPTY + qs));
@@ -270,12 +275,13 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           if (j == 0 && !mbar_wait(bar(C::B_OEMPTY + x), (oc[x] & 1u) ^ 1u, abort_flag, kTimeoutNs))
             return false;
           tc_fence_after();
-          const uint32_t vaddr = sKV + vs * C::TILEB;
+          const uint64_t v0 = smem_desc(sKV + vs * C::TILEB, C::CHUNKB, C::ATOM, C::SW);
+          const uint32_t ocol = tmem + C::COL_O + DH * x;
+          const uint32_t pcol = tmem + C::COL_P + (C::P_SEP ? 64 : 128) * x;
+          const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
           for (int k = 0; k < C::BN / 16; ++k)
-            mma_ts(tmem + C::COL_O + DH * x, tmem + C::COL_S + 128 * x + k * 8,
-                   smem_desc(vaddr + k * 2 * C::ATOM, C::CHUNKB, C::ATOM, C::SW), IDESC_O,
-                   (j > 0 || k > 0) ? 1u : 0u);
+            mma_ts(ocol, pcol + k * 8, desc_advance(v0, k * 2 * C::ATOM), IDESC_O, k > 0 ? 1u : acc0);
           if (j == nkv - 1) {
             mma_commit(bar(C::B_OFULL + x));
             ++oc[x];
@@ -339,6 +345,7 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t my_s = tmem + lane_off + C::COL_S + 128 * grp;
     const uint32_t my_o = tmem + lane_off + C::COL_O + DH * grp;
+    const uint32_t my_p = tmem + lane_off + C::COL_P + (C::P_SEP ? 64 : 128) * grp;
     const float c2 = a.scale_log2;
     const float half_scale = 0.5f * a.scale;
     uint32_t sc = 0, oc = 0;
@@ -358,69 +365,92 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         tc_fence_after();
         const int valid = min(C::BN, a.m - j * C::BN);
         if constexpr (SOFTMAX) {
-          uint32_t s[128];
-          tmem_ld_x32(my_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-          tmem_ld_x32(my_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-          tmem_ld_x32(my_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-          tmem_ld_x32(my_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-          tmem_wait_ld();
-          // row max (min when the scale is negative) over the valid columns, 8 independent chains
-          float mx;
-          {
-            const float ident = c2 >= 0.f ? -INFINITY : INFINITY;
+          // The row is handled in two 64-column halves read from TMEM, so at most
+          // 64 logits and the 64 packed P words are live at once.
+          // Row offset m_run (log2 units): the first key block of a tile takes the
+          // exact row max.  Later blocks reuse m_run as long as every
+          // p = 2^(x - m_run) stays <= 2^8, which a row sum <= 2^8 guarantees;
+          // otherwise (or on overflow, where the sum is not finite) the exact max
+          // of this block is taken and m_run moves when it grew by more than 2^8.
+          // Softmax does not depend on the offset, so this only skips the max.
+          uint32_t sh[64];
+          auto load_half = [&](int hf) {
+            tmem_ld_x32(my_s + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&sh[0]));
+            tmem_ld_x32(my_s + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sh[32]));
+            tmem_wait_ld();
+          };
+          auto row_max = [&]() -> float {
             float m8[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) m8[u] = ident;
-            if (valid == C::BN) {
-              if (c2 >= 0.f) {
+            for (int u = 0; u < 8; ++u) m8[u] = c2 >= 0.f ? -INFINITY : INFINITY;
 #pragma unroll
-                for (int i = 0; i < 128; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(s[i]));
-              } else {
+            for (int hf = 0; hf < 2; ++hf) {
+              load_half(hf);
 #pragma unroll
-                for (int i = 0; i < 128; ++i) m8[i & 7] = fminf(m8[i & 7], __uint_as_float(s[i]));
+              for (int i = 0; i < 64; ++i) {
+                const float x = __uint_as_float(sh[i]);
+                if (valid == C::BN || 64 * hf + i < valid)
+                  m8[i & 7] = c2 >= 0.f ? fmaxf(m8[i & 7], x) : fminf(m8[i & 7], x);
               }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 128; ++i)
-                if (i < valid)
-                  m8[i & 7] = c2 >= 0.f ? fmaxf(m8[i & 7], __uint_as_float(s[i]))
-                                        : fminf(m8[i & 7], __uint_as_float(s[i]));
             }
 #pragma unroll
             for (int u = 4; u > 0; u >>= 1)
 #pragma unroll
               for (int v = 0; v < u; ++v)
                 m8[v] = c2 >= 0.f ? fmaxf(m8[v], m8[v + u]) : fminf(m8[v], m8[v + u]);
-            mx = m8[0];
-          }
-          const float m_new = mx * c2;
-          float alpha = 1.f;
-          bool resc = false;
-          if (steps == 0) {
-            m_run = m_new;
-          } else if (m_new > m_run + 8.0f) {
-            alpha = ex2_approx(m_run - m_new);
-            m_run = m_new;
-            resc = true;
-          }
-          const float neg_m = -m_run;
-          float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          uint32_t pk[64];
+            return m8[0] * c2;
+          };
+          uint32_t pk[C::P_SEP ? 32 : 64];
+          auto exp_pack = [&]() -> float {
+            const float neg_m = -m_run;
+            float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            float p0 = ex2_approx(fmaf(__uint_as_float(s[2 * i]), c2, neg_m));
-            float p1 = ex2_approx(fmaf(__uint_as_float(s[2 * i + 1]), c2, neg_m));
-            if (valid < C::BN) {
-              p0 = (2 * i < valid) ? p0 : 0.f;
-              p1 = (2 * i + 1 < valid) ? p1 : 0.f;
+            for (int hf = 0; hf < 2; ++hf) {
+              load_half(hf);
+              uint32_t* pkh = C::P_SEP ? pk : pk + 32 * hf;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int col = 64 * hf + 2 * i;
+                float p0 = ex2_approx(fmaf(__uint_as_float(sh[2 * i]), c2, neg_m));
+                float p1 = ex2_approx(fmaf(__uint_as_float(sh[2 * i + 1]), c2, neg_m));
+                if (valid < C::BN) {
+                  p0 = col < valid ? p0 : 0.f;
+                  p1 = col + 1 < valid ? p1 : 0.f;
+                }
+                rs8[(2 * i) & 7] += p0;
+                rs8[(2 * i + 1) & 7] += p1;
+                pkh[i] = pack_bf16x2(p0, p1);
+              }
+              if (C::P_SEP) tmem_st_x32(my_p + 32 * hf, *reinterpret_cast<uint32_t(*)[32]>(pkh));
             }
-            rs8[(2 * i) & 7] += p0;
-            rs8[(2 * i + 1) & 7] += p1;
-            pk[i] = pack_bf16x2(p0, p1);
+            return ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+          };
+          float alpha = 1.f, rs = 0.f;
+          bool resc = false;
+          // pass 0: the first key block of the tile takes the exact max, later
+          // blocks reuse m_run; pass 1 (rare) redoes the block with the exact max
+#pragma unroll 1
+          for (int pass = 0; pass < 2; ++pass) {
+            const bool need_max = pass == 0 ? steps == 0 : !(rs <= 256.f);
+            if (__any_sync(0xffffffffu, need_max)) {
+              const float m_new = row_max();
+              if (need_max) {
+                if (pass == 0) {
+                  m_run = m_new;
+                } else if (m_new > m_run + 8.0f) {
+                  alpha = ex2_approx(m_run - m_new);
+                  m_run = m_new;
+                  resc = true;
+                }
+              }
+            }
+            rs = exp_pack();
+            if (pass == 1 || steps == 0 || !__any_sync(0xffffffffu, !(rs <= 256.f))) break;
           }
-          const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-          tmem_st_x32(my_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-          tmem_st_x32(my_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+          if (!C::P_SEP) {
+            tmem_st_x32(my_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+            tmem_st_x32(my_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+          }
           l_run = l_run * alpha + rs;
           if (__any_sync(0xffffffffu, resc)) {
             #pragma unroll
@@ -454,7 +484,7 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
               }
               pk[i] = pack_bf16x2(p0, p1);
             }
-            tmem_st_x16(my_s + 16 * c, pk);
+            tmem_st_x16(my_p + 16 * c, pk);
           }
           tmem_wait_st();
         }

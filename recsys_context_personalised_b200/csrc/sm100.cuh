@@ -204,6 +204,13 @@ __device__ __forceinline__ void red_add_v4(float* gptr, float a, float b, float 
                : "memory");
 }
 
+// Advances a shared-memory matrix descriptor by `bytes` (a multiple of 16 that
+// keeps the start address inside shared memory): only the start-address field
+// of the low word changes.  With `bytes` a compile-time constant this is one add.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
 // ----------------------------------------------------------- misc math
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

@@ -95,6 +95,23 @@ def test_odd_head_count(n, phi):
     check(out, d, phi, scale, True, torch.bfloat16, f"h=3 n={n}")
 
 
+@pytest.mark.parametrize("dh", [32, 64, 128])
+def test_softmax_row_max_growth(dh):
+    """Logits that grow from one key block to the next (and one that jumps by
+    far more than 2^8 in log2 units) exercise the exact-max fallback and the
+    O rescaling of the online softmax."""
+    n, m = [200, 77], 640
+    d = syn.random_problem(31, len(n), 2, dh, m, n, dtype=torch.bfloat16, std=0.5)
+    growth = torch.ones(m)
+    for j in range(5):
+        growth[128 * j:128 * (j + 1)] = 1.0 + 1.5 * j
+    growth[600:] = 12.0
+    d["k"] = (d["k"].float() * growth[None, None, :, None]).bfloat16()
+    scale = 1.0 / dh ** 0.5
+    out = run_gpu(d, "softmax", scale, True)
+    check(out, d, "softmax", scale, True, torch.bfloat16, f"growth dh={dh}")
+
+
 def check_single_key_softmax(out, d, scale, tol):
     """Softmax over one key: P = 1, so dS = dP - D = 0 and dQ = dK = 0 exactly.
 
