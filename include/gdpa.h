@@ -160,6 +160,18 @@ typedef struct {
 GDPA_API int32_t gdpa_timing_read(gdpa_kernel_time_t* out, int32_t cap);
 
 /*
+ * Self-test of the device-side failure path.  Launches one small kernel on
+ * `stream` whose thread waits, with the same bounded mbarrier wait the GDPA
+ * kernels use, on a barrier that nothing ever completes.  After timeout_us
+ * microseconds (1 .. 5,000,000) the wait gives up, GDPA_ERR_TIMEOUT is written
+ * to the status word of `workspace` (>= 256 bytes, 256-byte aligned, device)
+ * and the kernel returns; the context stays usable.  Read the result with
+ * gdpa_workspace_status().  The Kunlun pages have no counterpart of this call.
+ */
+GDPA_API gdpa_status_t gdpa_selftest_wait_timeout(void* workspace, size_t workspace_bytes,
+                                                  uint32_t timeout_us, void* stream);
+
+/*
  * gdpa_fwd_no_alloc: gdpa_fwd for callers that cannot allocate device memory
  * at call time (for example a host framework that has reserved all device
  * memory for its own pool and gives plug-in operators no allocator, or a

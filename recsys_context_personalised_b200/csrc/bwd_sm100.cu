@@ -528,6 +528,438 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   if (warp == 2) tmem_dealloc(tmem, 512);
 }
 
+// ---------------------------------------------------------------- half-tile pipeline (dh <= 64)
+//
+// Same products as above, but each 128-row query tile is processed as two
+// 64-row halves with their own S^T/dP^T buffers in TMEM, so that activation
+// group h works on half h while the tensor core computes the other half:
+//   ST(i,0) ST(i,1) | dVdK(i,0) ST(i+1,0) | dVdK(i,1) dQ(i) ST(i+1,1) | ...
+// where ST(i,h) = {S^T, dP^T} of rows 64h..64h+63 of tile i (M = 128 keys,
+// N = 64 rows), dVdK(i,h) adds that half's P^T dO and dS^T Q (K = 64 rows),
+// and dQ(i) = dS K over the whole tile once both halves of dS^T are written.
+// dS^T and dQ are double-buffered by tile parity.
+//
+// TMEM: S^T_h [128h, 128h+64), dP^T_h [128h+64, 128h+128) (P^T_h aliases the
+// first 32 columns of S^T_h), dV [256, 256+dh), dK [256+dh, 256+2dh),
+// dQ_c [256+2dh+c*dh, 256+3dh+c*dh).
+template <int DH>
+struct BwdHalfCfg {
+  static_assert(DH <= 64, "half-tile pipeline needs dh <= 64");
+  static constexpr int CH = DH;
+  static constexpr uint32_t ROWB = CH * 2;
+  static constexpr uint32_t TILEB = 128 * ROWB;            // [128 x DH] bf16
+  static constexpr uint32_t SW = DH < 64 ? kSw64 : kSw128;
+  static constexpr uint32_t ATOM = 8 * ROWB;
+  static constexpr int NSTG = 2;
+  static constexpr uint32_t DSB = 2 * 128 * 128;           // one dS^T buffer
+  static constexpr uint32_t COL_DV = 256, COL_DK = 256 + DH, COL_DQ = 256 + 2 * DH;
+  static constexpr int B_KVFULL = 0, B_KVEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_DQFULL = 6,
+                       B_DQEMPTY = 8, B_ACCFULL = 10, B_ACCEMPTY = 11, B_DRAIN = 12,
+                       B_STFULL = 13, B_STEMPTY = 13 + NSTG, NBAR = 13 + 2 * NSTG;
+  static constexpr uint32_t OFF_K = 0, OFF_V = TILEB, OFF_STG = 2 * TILEB;
+  static constexpr uint32_t OFF_DS = OFF_STG + NSTG * 2 * TILEB;
+  static constexpr uint32_t OFF_CTL = OFF_DS + 2 * DSB;
+  static constexpr uint32_t CTL_BYTES = 1024 + 8 * 2 * 128 * 4;
+  static constexpr uint32_t SMEM_USED = 1024 + OFF_CTL + CTL_BYTES;
+  static constexpr uint32_t SMEM = SMEM_USED > 120u * 1024u ? SMEM_USED : 120u * 1024u;
+  static_assert(SMEM <= 232448u, "exceeds the 227 KB of shared memory a CTA can have");
+  static_assert(COL_DQ + 2 * DH <= 512, "TMEM columns");
+};
+
+template <int DH, int PHI>
+__global__ void __launch_bounds__(kThreads, 1)
+gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmG,
+                     const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const BwdArgs a) {
+  using C = BwdHalfCfg<DH>;
+  constexpr bool SOFTMAX = PHI == GDPA_PHI_SOFTMAX;
+  constexpr uint32_t IDESC_T = idesc_bf16(128, 64, 0, 0);    // S^T, dP^T of a half: N = 64 rows
+  constexpr uint32_t IDESC_KV = idesc_bf16(128, DH, 0, 1);   // dV, dK (B MN-major)
+  constexpr uint32_t IDESC_Q = idesc_bf16(128, DH, 1, 1);    // dQ (A and B MN-major)
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sStg = base + C::OFF_STG;
+  const uint32_t sDS = base + C::OFF_DS;
+  uint8_t* ctl = gbase + C::OFF_CTL;
+  const uint32_t bar0 = smem_u32(ctl);
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 8 * C::NBAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 8 * C::NBAR + 4);
+  float* stats = reinterpret_cast<float*>(ctl + 1024);   // [8 warps][2][128]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_KVFULL), 1);
+    mbar_init(bar(C::B_KVEMPTY), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::B_SFULL + i), 1);
+      mbar_init(bar(C::B_PFULL + i), 128);
+      mbar_init(bar(C::B_DQFULL + i), 1);
+      mbar_init(bar(C::B_DQEMPTY + i), 256);
+    }
+    mbar_init(bar(C::B_ACCFULL), 1);
+    mbar_init(bar(C::B_ACCEMPTY), 256);
+    mbar_init(bar(C::B_DRAIN), 1);
+    for (int i = 0; i < C::NSTG; ++i) {
+      mbar_init(bar(C::B_STFULL + i), 1);
+      mbar_init(bar(C::B_STEMPTY + i), 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmG);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int count = a.ws->status == GDPA_ERR_INVALID_ARG ? 0 : a.ws->tile_count;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t ic = 0, stage = 0, sphase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
+        const Tile it = a.tiles[t];
+        if (it.rows == 0) continue;
+        const int nq = (it.rows + 127) >> 7;
+        const int t0 = a.offsets[it.b];
+        if (!mbar_wait(bar(C::B_KVEMPTY), (ic & 1u) ^ 1u, abort_flag, kTimeoutNs)) break;
+        mbar_expect_tx(bar(C::B_KVFULL), 2 * C::TILEB);
+        tma_load_4d(sK, &tmK, bar(C::B_KVFULL), 0, it.row0, it.head, it.b);
+        tma_load_4d(sV, &tmV, bar(C::B_KVFULL), 0, it.row0, it.head, it.b);
+        for (int i = 0; i < nq; ++i) {
+          if (!mbar_wait(bar(C::B_STEMPTY + stage), sphase ^ 1u, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = sStg + stage * 2 * C::TILEB;
+          mbar_expect_tx(bar(C::B_STFULL + stage), 2 * C::TILEB);
+          tma_load_3d(dst, &tmQ, bar(C::B_STFULL + stage), 0, it.head, t0 + 128 * i);
+          tma_load_3d(dst + C::TILEB, &tmG, bar(C::B_STFULL + stage), 0, it.head, t0 + 128 * i);
+          if (++stage == (uint32_t)C::NSTG) {
+            stage = 0;
+            sphase ^= 1u;
+          }
+        }
+        ++ic;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t ic = 0, stage = 0, sphase = 0, qs = 0;
+      bool ok = true;
+      const uint64_t dk0 = smem_desc(sK, 16, C::ATOM, C::SW), dv0 = smem_desc(sV, 16, C::ATOM, C::SW);
+      const uint64_t kmn0 = smem_desc(sK, C::TILEB, C::ATOM, C::SW);       // K, MN-major (dQ)
+      // ST(h): S^T_h = K Q[64h..64h+63]^T and dP^T_h = V dO[64h..64h+63]^T of the tile in `st`
+      auto issue_st = [&](uint32_t st, int h) {
+        const uint32_t qaddr = sStg + st * 2 * C::TILEB + 64 * h * C::ROWB;
+        const uint64_t q0 = smem_desc(qaddr, 16, C::ATOM, C::SW);
+        const uint64_t g0 = smem_desc(qaddr + C::TILEB, 16, C::ATOM, C::SW);
+#pragma unroll
+        for (int k = 0; k < DH / 16; ++k)
+          mma_ss(tmem + 128 * h, desc_advance(dk0, k * 32), desc_advance(q0, k * 32), IDESC_T,
+                 k > 0 ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < DH / 16; ++k)
+          mma_ss(tmem + 128 * h + 64, desc_advance(dv0, k * 32), desc_advance(g0, k * 32), IDESC_T,
+                 k > 0 ? 1u : 0u);
+        mma_commit(bar(C::B_SFULL + h));
+      };
+      // dVdK(h): dV += P^T_h dO[64h..], dK += dS^T[64h..] Q[64h..] of the tile in `st`
+      auto issue_dvdk = [&](uint32_t st, int h, uint32_t c, bool first) {
+        const uint32_t qaddr = sStg + st * 2 * C::TILEB + 64 * h * C::ROWB;
+        const uint64_t gmn = smem_desc(qaddr + C::TILEB, C::TILEB, C::ATOM, C::SW);   // dO, MN-major
+        const uint64_t qmn = smem_desc(qaddr, C::TILEB, C::ATOM, C::SW);              // Q, MN-major
+        const uint64_t dsk = smem_desc(sDS + c * C::DSB + h * 16384, 16, 1024, kSw128);  // dS^T, K-major
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_ts(tmem + C::COL_DV, tmem + 128 * h + 8 * k, desc_advance(gmn, k * 2 * C::ATOM),
+                 IDESC_KV, (first && k == 0) ? 0u : 1u);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_ss(tmem + C::COL_DK, desc_advance(dsk, k * 32), desc_advance(qmn, k * 2 * C::ATOM),
+                 IDESC_KV, (first && k == 0) ? 0u : 1u);
+      };
+      auto wait_stage = [&](uint32_t st, uint32_t ph) -> bool {
+        if (!mbar_wait(bar(C::B_STFULL + st), ph, abort_flag, kTimeoutNs)) return false;
+        tc_fence_after();
+        return true;
+      };
+      for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
+        const Tile it = a.tiles[t];
+        if (it.rows == 0) continue;
+        const int nq = (it.rows + 127) >> 7;
+        if (!mbar_wait(bar(C::B_KVFULL), ic & 1u, abort_flag, kTimeoutNs)) break;
+        tc_fence_after();
+        if (!wait_stage(stage, sphase)) break;
+        issue_st(stage, 0);
+        issue_st(stage, 1);
+        for (int i = 0; i < nq; ++i, ++qs) {
+          const uint32_t c = qs & 1u;
+          uint32_t nst = stage + 1, nph = sphase;
+          if (nst == (uint32_t)C::NSTG) {
+            nst = 0;
+            nph ^= 1u;
+          }
+          // half 0 of tile i, then the next tile's half-0 products
+          if (!mbar_wait(bar(C::B_PFULL + 0), qs & 1u, abort_flag, kTimeoutNs) ||
+              (i == 0 && !mbar_wait(bar(C::B_ACCEMPTY), (ic & 1u) ^ 1u, abort_flag, kTimeoutNs))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_dvdk(stage, 0, c, i == 0);
+          if (i + 1 < nq) {
+            if (!wait_stage(nst, nph)) {
+              ok = false;
+              break;
+            }
+            issue_st(nst, 0);
+          }
+          // half 1, the tile's dQ, then the next tile's half-1 products
+          if (!mbar_wait(bar(C::B_PFULL + 1), qs & 1u, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_dvdk(stage, 1, c, false);
+          mma_commit(bar(C::B_STEMPTY + stage));
+          if (!mbar_wait(bar(C::B_DQEMPTY + c), ((qs >> 1) & 1u) ^ 1u, abort_flag, kTimeoutNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          {
+            const uint64_t dsm = smem_desc(sDS + c * C::DSB, 16384, 1024, kSw128);   // dS, MN-major
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              mma_ss(tmem + C::COL_DQ + c * DH, desc_advance(dsm, k * 2048),
+                     desc_advance(kmn0, k * 2 * C::ATOM), IDESC_Q, k > 0 ? 1u : 0u);
+            mma_commit(bar(C::B_DQFULL + c));
+          }
+          if (i + 1 < nq) issue_st(nst, 1);
+          stage = nst;
+          sphase = nph;
+        }
+        if (!ok) break;
+        mma_commit(bar(C::B_KVEMPTY));
+        mma_commit(bar(C::B_ACCFULL));
+        ++ic;
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ activation groups
+    const int grp = (warp - 4) >> 2;                   // the 64-row half this group owns
+    const int quad = warp & 3;
+    const int lrow = quad * 32 + lane;                 // TMEM lane: key (S^T, dV, dK) or row (dQ)
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    float* wst = stats + (warp - 4) * 256;
+    const float c2 = a.scale_log2, sc = a.scale, half_sc = 0.5f * a.scale;
+    uint32_t ic = 0, qs = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
+      const Tile it = a.tiles[t];
+      const int n = it.rows;
+      const int key = it.row0 + lrow;
+      __nv_bfloat16* kvout = (grp == 0 ? a.dv : a.dk) +
+                             (((int64_t)it.b * a.h + it.head) * a.m + key) * DH;
+      if (n == 0) {                                    // no tokens: dK = dV = 0
+        if (key < a.m) {
+          uint4* d4 = reinterpret_cast<uint4*>(kvout);
+#pragma unroll
+          for (int c = 0; c < DH / 8; ++c) d4[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        continue;
+      }
+      const int nq = (n + 127) >> 7;
+      const int t0 = a.offsets[it.b];
+      // dQ of tile ii (buffer step & 1): lane = query row; this group adds half the columns
+      auto drain_dq = [&](int ii, uint32_t step) -> bool {
+        const uint32_t b = step & 1u;
+        const bool w = mbar_wait(bar(C::B_DQFULL + b), (step >> 1) & 1u, abort_flag, kTimeoutNs);
+        if (!__all_sync(0xffffffffu, w)) return false;
+        tc_fence_after();
+        const int rg = 128 * ii + lrow;
+        float* dst = a.dq_acc + ((int64_t)(t0 + rg) * a.h + it.head) * DH + grp * (DH / 2);
+#pragma unroll
+        for (int c = 0; c < DH / 2; c += 16) {
+          uint32_t v[16];
+          tmem_ld_x16(tmem + lane_off + C::COL_DQ + b * DH + grp * (DH / 2) + c, v);
+          tmem_wait_ld();
+          if (rg < n) {
+#pragma unroll
+            for (int u = 0; u < 16; u += 4)
+              red_add_v4(dst + c + u, __uint_as_float(v[u]), __uint_as_float(v[u + 1]),
+                         __uint_as_float(v[u + 2]), __uint_as_float(v[u + 3]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(C::B_DQEMPTY + b));
+        return true;
+      };
+      float nl[2] = {0.f, 0.f}, nd[2] = {0.f, 0.f};
+      auto load_stats = [&](int ii) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int rg = 128 * ii + 64 * grp + 32 * u + lane;
+          nl[u] = 0.f;
+          nd[u] = 0.f;
+          if (rg < n) {
+            const int64_t at = (int64_t)it.head * a.T + t0 + rg;
+            nl[u] = a.lse[at] * 1.4426950408889634f;
+            nd[u] = a.dsum[at];
+          }
+        }
+      };
+      if constexpr (SOFTMAX) load_stats(0);
+      for (int i = 0; i < nq; ++i, ++qs) {
+        const int rbase = 128 * i + 64 * grp;          // first sample row of this group's half
+        const uint32_t dsb = sDS + (qs & 1u) * C::DSB + grp * 16384;
+        if constexpr (SOFTMAX) {
+          __syncwarp();
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            wst[32 * u + lane] = nl[u];
+            wst[64 + 32 * u + lane] = nd[u];
+          }
+          __syncwarp();
+          if (i + 1 < nq) load_stats(i + 1);
+        }
+        bool w = mbar_wait(bar(C::B_SFULL + grp), qs & 1u, abort_flag, kTimeoutNs);
+        if (!__all_sync(0xffffffffu, w)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t s[32], dp[32];
+          tmem_ld_x32(tmem + lane_off + 128 * grp + 32 * ch, s);
+          tmem_ld_x32(tmem + lane_off + 128 * grp + 64 + 32 * ch, dp);
+          tmem_wait_ld();
+          uint32_t pp[16], dd[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            float pv[2], dv2[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int r = 32 * ch + c + e;
+              const float x = __uint_as_float(s[c + e]);
+              const float g = __uint_as_float(dp[c + e]);
+              float p, ds;
+              if constexpr (SOFTMAX) {
+                p = ex2_approx(fmaf(x, c2, -wst[r]));
+                ds = p * (g - wst[64 + r]);
+              } else if constexpr (PHI == GDPA_PHI_SILU) {
+                const float hx = x * half_sc;
+                const float th = tanh_approx(hx);
+                const float sg = fmaf(0.5f, th, 0.5f);          // logistic(x s)
+                p = fmaf(hx, th, hx);                             // x s * logistic(x s)
+                ds = g * sg * fmaf(x * sc, 1.f - sg, 1.f);
+              } else {
+                p = x * sc;
+                ds = g;
+              }
+              const bool valid = rbase + r < n;
+              pv[e] = valid ? p : 0.f;
+              dv2[e] = valid ? ds : 0.f;
+            }
+            pp[c / 2] = pack_bf16x2(pv[0], pv[1]);
+            dd[c / 2] = pack_bf16x2(dv2[0], dv2[1]);
+          }
+          tmem_st_x16(tmem + lane_off + 128 * grp + 16 * ch, pp);
+          // dS^T line `lrow` of this half's chunk, 16-byte pieces 4ch..4ch+3, 128B swizzle
+          const uint32_t line = dsb + lrow * 128;
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t j = 4 * ch + jj;
+            const uint32_t addr = line + ((j ^ (uint32_t)(lrow & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dd[4 * jj]),
+                         "r"(dd[4 * jj + 1]), "r"(dd[4 * jj + 2]), "r"(dd[4 * jj + 3])
+                         : "memory");
+          }
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_PFULL + grp));
+        if (i > 0 && !drain_dq(i - 1, qs - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok && !drain_dq(nq - 1, qs - 1)) ok = false;
+      if (!ok) break;
+      // ---------------------------------------------------------- dV / dK of this key block
+      bool w = mbar_wait(bar(C::B_ACCFULL), ic & 1u, abort_flag, kTimeoutNs);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      {
+        const uint32_t src = tmem + lane_off + (grp == 0 ? C::COL_DV : C::COL_DK);
+        const float mul = grp == 0 ? 1.f : sc;
+#pragma unroll
+        for (int c = 0; c < DH; c += 16) {
+          uint32_t v[16];
+          tmem_ld_x16(src + c, v);
+          tmem_wait_ld();
+          uint32_t pk[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            pk[u] = pack_bf16x2(__uint_as_float(v[2 * u]) * mul, __uint_as_float(v[2 * u + 1]) * mul);
+          if (key < a.m) {
+            uint4* d4 = reinterpret_cast<uint4*>(kvout + c);
+            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::B_ACCEMPTY));
+      ++ic;
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  __syncwarp();
+  __syncthreads();
+  if (*abort_flag) {
+    report(a.ws, GDPA_ERR_TIMEOUT);
+    volatile int never = 0;
+    if (warp == 1 && lane == 0) {
+      mma_commit(bar(C::B_DRAIN));
+      mbar_wait(bar(C::B_DRAIN), 0, &never, kTimeoutNs);
+    }
+    if (warp == 0 && lane == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 200000ull) {
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+
 // ------------------------------------------------------------------ host side
 
 template <int DH>
@@ -586,6 +1018,15 @@ cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* 
   args.m = p.m;
   args.scale = p.scale;
   args.scale_log2 = p.scale * 1.4426950408889634f;
+  if constexpr (DH <= 64) {
+    using H = BwdHalfCfg<DH>;
+    auto hk = gdpa_bwd_half_kernel<DH, PHI>;
+    e = cudaFuncSetAttribute(hk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H::SMEM);
+    if (e != cudaSuccess) return e;
+    KernelScope ks_("gdpa_bwd_sm100", st);
+    hk<<<device_sm_count(), kThreads, H::SMEM, st>>>(mq, mg, mk, mv, args);
+    return cudaGetLastError();
+  }
   KernelScope ks_("gdpa_bwd_sm100", st);
   kern<<<device_sm_count(), kThreads, C::SMEM, st>>>(mq, mg, mk, mv, args);
   return cudaGetLastError();

@@ -85,6 +85,15 @@ def test_null_and_misaligned_pointers_rejected_before_launch():
                         4096, 4096, ws, 1 << 30, None) == 1
 
 
+def test_selftest_rejects_bad_arguments():
+    lib = pkg.load()
+    lib.gdpa_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32,
+                                               ctypes.c_void_p]
+    assert lib.gdpa_selftest_wait_timeout(None, 256, 10, None) == 1
+    assert lib.gdpa_selftest_wait_timeout(1 << 20, 16, 10, None) == 1
+    assert lib.gdpa_selftest_wait_timeout(1 << 20, 256, 0, None) == 1
+
+
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(ImportError):
         G.load(str(tmp_path / "libgdpa.so"))

@@ -112,6 +112,33 @@ def test_softmax_row_max_growth(dh):
     check(out, d, "softmax", scale, True, torch.bfloat16, f"growth dh={dh}")
 
 
+@pytest.mark.parametrize("phi", ["identity", "silu", "softmax"])
+def test_negative_scale(phi):
+    """A negative scale flips the logits (the softmax kernels then track a row
+    minimum of the raw dot products)."""
+    n, m = [150, 33], 300
+    d = syn.random_problem(41, len(n), 2, 64, m, n, dtype=torch.bfloat16, std=0.6)
+    out = run_gpu(d, phi, -0.3, True)
+    check(out, d, phi, -0.3, True, torch.bfloat16, "negative scale")
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A device wait that can never complete gives up after its limit, reports
+    GDPA_ERR_TIMEOUT through the workspace status word, and later work runs."""
+    import ctypes
+    lib = pkg.load()
+    lib.gdpa_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32,
+                                               ctypes.c_void_p]
+    lib.gdpa_selftest_wait_timeout.restype = ctypes.c_int
+    ws = pkg.workspace(256, DEV)
+    stream = torch.cuda.current_stream().cuda_stream
+    assert lib.gdpa_selftest_wait_timeout(ws.data_ptr(), ws.numel(), 20000, stream) == 0
+    assert pkg.workspace_status(ws) == 4
+    d = syn.random_problem(5, 2, 2, 64, 64, [10, 20], dtype=torch.bfloat16)
+    out = run_gpu(d, "silu", 0.5, False)
+    check(out, d, "silu", 0.5, False, torch.bfloat16, "after time-out")
+
+
 def check_single_key_softmax(out, d, scale, tol):
     """Softmax over one key: P = 1, so dS = dP - D = 0 and dQ = dK = 0 exactly.
 
