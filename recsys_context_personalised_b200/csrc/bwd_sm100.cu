@@ -555,15 +555,23 @@ struct BwdHalfCfg {
   static constexpr uint32_t COL_DV = 256, COL_DK = 256 + DH, COL_DQ = 256 + 2 * DH;
   static constexpr int B_KVFULL = 0, B_KVEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_DQFULL = 6,
                        B_DQEMPTY = 8, B_ACCFULL = 10, B_ACCEMPTY = 11, B_DRAIN = 12,
-                       B_STFULL = 13, B_STEMPTY = 13 + NSTG, NBAR = 13 + 2 * NSTG;
+                       B_DQSYNC = 13, B_STFULL = 15, B_STEMPTY = 15 + NSTG,
+                       NBAR = 15 + 2 * NSTG;
   static constexpr uint32_t OFF_K = 0, OFF_V = TILEB, OFF_STG = 2 * TILEB;
   static constexpr uint32_t OFF_DS = OFF_STG + NSTG * 2 * TILEB;
-  static constexpr uint32_t OFF_CTL = OFF_DS + 2 * DSB;
+  // dQ staging for the bulk reduce, one per group: [128 rows][DH/2 fp32], laid
+  // out with the swizzle of the reduce's tensor map (128 B rows: 128B, 64 B rows: 64B)
+  static constexpr uint32_t DQROWB = DH / 2 * 4;
+  static constexpr uint32_t DQSTGB = 128 * DQROWB;
+  static constexpr uint32_t OFF_DQS = OFF_DS + 2 * DSB;
+  static constexpr uint32_t OFF_CTL = OFF_DQS + 2 * DQSTGB;
   static constexpr uint32_t CTL_BYTES = 1024 + 8 * 2 * 128 * 4;
   static constexpr uint32_t SMEM_USED = 1024 + OFF_CTL + CTL_BYTES;
   static constexpr uint32_t SMEM = SMEM_USED > 120u * 1024u ? SMEM_USED : 120u * 1024u;
   static_assert(SMEM <= 232448u, "exceeds the 227 KB of shared memory a CTA can have");
   static_assert(COL_DQ + 2 * DH <= 512, "TMEM columns");
+  static_assert(OFF_DQS % 1024 == 0 && DQSTGB % 1024 == 0, "swizzle atoms need 1024-B alignment");
+  static_assert(8 * NBAR <= 1016, "barriers, TMEM slot and abort flag share the first 1 KB");
 };
 
 template <int DH, int PHI>
@@ -571,7 +579,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmG,
                      const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const BwdArgs a) {
+                     const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ CUtensorMap tmDQ, const BwdArgs a) {
   using C = BwdHalfCfg<DH>;
   constexpr bool SOFTMAX = PHI == GDPA_PHI_SOFTMAX;
   constexpr uint32_t IDESC_T = idesc_bf16(128, 64, 0, 0);    // S^T, dP^T of a half: N = 64 rows
@@ -604,6 +613,8 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
     mbar_init(bar(C::B_ACCFULL), 1);
     mbar_init(bar(C::B_ACCEMPTY), 256);
     mbar_init(bar(C::B_DRAIN), 1);
+    mbar_init(bar(C::B_DQSYNC + 0), 128);
+    mbar_init(bar(C::B_DQSYNC + 1), 128);
     for (int i = 0; i < C::NSTG; ++i) {
       mbar_init(bar(C::B_STFULL + i), 1);
       mbar_init(bar(C::B_STEMPTY + i), 1);
@@ -616,6 +627,7 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
     prefetch_tmap(&tmG);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    prefetch_tmap(&tmDQ);
   }
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -770,7 +782,8 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     float* wst = stats + (warp - 4) * 256;
     const float c2 = a.scale_log2, sc = a.scale, half_sc = 0.5f * a.scale;
-    uint32_t ic = 0, qs = 0;
+    const uint32_t sDQS = base + C::OFF_DQS + grp * C::DQSTGB;
+    uint32_t ic = 0, qs = 0, dq_sync_phase = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
       const Tile it = a.tiles[t];
@@ -788,28 +801,47 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
       const int nq = (n + 127) >> 7;
       const int t0 = a.offsets[it.b];
-      // dQ of tile ii (buffer step & 1): lane = query row; this group adds half the columns
+      // dQ of tile ii (buffer step & 1): lane = query row.  The group stages its
+      // half of the columns in shared memory and one thread adds the whole
+      // [128 x DH/2] box into the fp32 accumulator with one bulk reduce.  Rows
+      // past the sample carry exact zeros (their dS entries are zero), so the
+      // box may overlap the next sample; rows past T are clipped by the map.
+      auto group_sync = [&]() -> bool {
+        mbar_arrive(bar(C::B_DQSYNC + grp));
+        const bool w = mbar_wait(bar(C::B_DQSYNC + grp), dq_sync_phase, abort_flag, kTimeoutNs);
+        dq_sync_phase ^= 1u;
+        return __all_sync(0xffffffffu, w);
+      };
       auto drain_dq = [&](int ii, uint32_t step) -> bool {
         const uint32_t b = step & 1u;
         const bool w = mbar_wait(bar(C::B_DQFULL + b), (step >> 1) & 1u, abort_flag, kTimeoutNs);
         if (!__all_sync(0xffffffffu, w)) return false;
         tc_fence_after();
-        const int rg = 128 * ii + lrow;
-        float* dst = a.dq_acc + ((int64_t)(t0 + rg) * a.h + it.head) * DH + grp * (DH / 2);
-#pragma unroll
-        for (int c = 0; c < DH / 2; c += 16) {
-          uint32_t v[16];
-          tmem_ld_x16(tmem + lane_off + C::COL_DQ + b * DH + grp * (DH / 2) + c, v);
-          tmem_wait_ld();
-          if (rg < n) {
-#pragma unroll
-            for (int u = 0; u < 16; u += 4)
-              red_add_v4(dst + c + u, __uint_as_float(v[u]), __uint_as_float(v[u + 1]),
-                         __uint_as_float(v[u + 2]), __uint_as_float(v[u + 3]));
-          }
-        }
+        uint32_t v[DH / 2];
+        const uint32_t src = tmem + lane_off + C::COL_DQ + b * DH + grp * (DH / 2);
+        if constexpr (DH == 64)
+          tmem_ld_x32(src, v);
+        else
+          tmem_ld_x16(src, v);
+        tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar(C::B_DQEMPTY + b));
+        // the previous reduce from the staging area must have finished reading it
+        if (lrow == 0) bulk_wait_group_read0();
+        if (!group_sync()) return false;
+        const uint32_t line = sDQS + lrow * C::DQROWB;
+        const uint32_t sw = C::DQROWB == 128 ? (uint32_t)(lrow & 7) : (uint32_t)((lrow >> 1) & 3);
+#pragma unroll
+        for (int j = 0; j < (int)(C::DQROWB / 16); ++j)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(line + ((j ^ sw) << 4)),
+                       "r"(v[4 * j]), "r"(v[4 * j + 1]), "r"(v[4 * j + 2]), "r"(v[4 * j + 3])
+                       : "memory");
+        fence_proxy_async_smem();
+        if (!group_sync()) return false;
+        if (lrow == 0) {
+          tma_reduce_add_3d(&tmDQ, sDQS, grp * (DH / 2), it.head, t0 + 128 * ii);
+          bulk_commit_group();
+        }
         return true;
       };
       float nl[2] = {0.f, 0.f}, nd[2] = {0.f, 0.f};
@@ -935,6 +967,7 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
       mbar_arrive(bar(C::B_ACCEMPTY));
       ++ic;
     }
+    if (lrow == 0) bulk_wait_group0();               // reduces done before the CTA exits
   }
 
   // ------------------------------------------------------------ teardown
@@ -992,6 +1025,23 @@ bool make_bwd_maps(const gdpa_problem_t& p, const void* q, const void* g, const 
   return true;
 }
 
+// The fp32 dQ accumulator [T, h, DH] as the target of the half kernel's bulk
+// reduces: boxes of DH/2 columns x 128 rows of one head.
+template <int DH>
+bool make_dq_map(const gdpa_problem_t& p, float* dq_acc, CUtensorMap* m) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const CUtensorMapSwizzle sw = DH / 2 * 4 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const cuuint64_t d[3] = {(cuuint64_t)DH, (cuuint64_t)p.h,
+                           (cuuint64_t)(p.total_tokens > 0 ? p.total_tokens : 1)};
+  const cuuint64_t str[2] = {(cuuint64_t)DH * 4, (cuuint64_t)p.h * DH * 4};
+  const cuuint32_t box[3] = {(cuuint32_t)(DH / 2), 1, 128};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dq_acc, d, str, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int DH, int PHI>
 cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
                          const void* k, const void* v, const float* lse, const float* dsum,
@@ -1021,10 +1071,12 @@ cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* 
   if constexpr (DH <= 64) {
     using H = BwdHalfCfg<DH>;
     auto hk = gdpa_bwd_half_kernel<DH, PHI>;
+    CUtensorMap mdq;
+    if (!make_dq_map<DH>(p, dq_acc, &mdq)) return cudaErrorInvalidValue;
     e = cudaFuncSetAttribute(hk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H::SMEM);
     if (e != cudaSuccess) return e;
     KernelScope ks_("gdpa_bwd_sm100", st);
-    hk<<<device_sm_count(), kThreads, H::SMEM, st>>>(mq, mg, mk, mv, args);
+    hk<<<device_sm_count(), kThreads, H::SMEM, st>>>(mq, mg, mk, mv, mdq, args);
     return cudaGetLastError();
   }
   KernelScope ks_("gdpa_bwd_sm100", st);
