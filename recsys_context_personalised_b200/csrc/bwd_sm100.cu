@@ -580,7 +580,9 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmG,
                      const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV,
-                     const __grid_constant__ CUtensorMap tmDQ, const BwdArgs a) {
+                     const __grid_constant__ CUtensorMap tmDQ,
+                     const __grid_constant__ CUtensorMap tmDV,
+                     const __grid_constant__ CUtensorMap tmDK, const BwdArgs a) {
   using C = BwdHalfCfg<DH>;
   constexpr bool SOFTMAX = PHI == GDPA_PHI_SOFTMAX;
   constexpr uint32_t IDESC_T = idesc_bf16(128, 64, 0, 0);    // S^T, dP^T of a half: N = 64 rows
@@ -628,6 +630,8 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
     prefetch_tmap(&tmDQ);
+    prefetch_tmap(&tmDV);
+    prefetch_tmap(&tmDK);
   }
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -784,6 +788,9 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
     const float c2 = a.scale_log2, sc = a.scale, half_sc = 0.5f * a.scale;
     const uint32_t sDQS = base + C::OFF_DQS + grp * C::DQSTGB;
     uint32_t ic = 0, qs = 0, dq_sync_phase = 0;
+    // a dV/dK bulk store may still be reading the dS^T half of buffer acc_par
+    bool acc_pending = false;
+    uint32_t acc_par = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
       const Tile it = a.tiles[t];
@@ -826,9 +833,11 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar(C::B_DQEMPTY + b));
-        // the previous reduce from the staging area must have finished reading it
+        // the previous reduce from the staging area (and any dV/dK store) must
+        // have finished reading shared memory
         if (lrow == 0) bulk_wait_group_read0();
         if (!group_sync()) return false;
+        acc_pending = false;
         const uint32_t line = sDQS + lrow * C::DQROWB;
         const uint32_t sw = C::DQROWB == 128 ? (uint32_t)(lrow & 7) : (uint32_t)((lrow >> 1) & 3);
 #pragma unroll
@@ -878,6 +887,14 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
           break;
         }
         tc_fence_after();
+        if (acc_pending && (qs & 1u) == acc_par) {       // dS^T half below was a store's source
+          if (lrow == 0) bulk_wait_group_read0();
+          if (!group_sync()) {
+            ok = false;
+            break;
+          }
+          acc_pending = false;
+        }
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           uint32_t s[32], dp[32];
@@ -945,26 +962,51 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
       tc_fence_after();
       {
+        // Group 0 writes dV, group 1 dK (times the scale): the rows go as bf16
+        // into this group's half of the last tile's dS^T buffer (its readers
+        // are all in the completed products), swizzled like the output's
+        // tensor map, and leave in one bulk tensor store; keys past m are
+        // clipped by the map.
         const uint32_t src = tmem + lane_off + (grp == 0 ? C::COL_DV : C::COL_DK);
         const float mul = grp == 0 ? 1.f : sc;
+        const uint32_t par = (qs - 1) & 1u;
+        const uint32_t stg = sDS + par * C::DSB + grp * 16384;
+        const uint32_t line = stg + lrow * (DH * 2);
+        const uint32_t sw = DH == 64 ? (uint32_t)(lrow & 7) : (uint32_t)((lrow >> 1) & 3);
 #pragma unroll
-        for (int c = 0; c < DH; c += 16) {
-          uint32_t v[16];
-          tmem_ld_x16(src + c, v);
+        for (int c = 0; c < DH; c += 32) {
+          uint32_t v[32];
+          tmem_ld_x32(src + c, v);
           tmem_wait_ld();
-          uint32_t pk[8];
+          if (c + 32 == DH) {
+            tc_fence_before();
+            mbar_arrive(bar(C::B_ACCEMPTY));            // the accumulators are free
+          }
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            pk[u] = pack_bf16x2(__uint_as_float(v[2 * u]) * mul, __uint_as_float(v[2 * u + 1]) * mul);
-          if (key < a.m) {
-            uint4* d4 = reinterpret_cast<uint4*>(kvout + c);
-            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          for (int j = 0; j < 4; ++j) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              pk[u] = pack_bf16x2(__uint_as_float(v[8 * j + 2 * u]) * mul,
+                                  __uint_as_float(v[8 * j + 2 * u + 1]) * mul);
+            const uint32_t chunk = (uint32_t)(c / 8 + j);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(line + ((chunk ^ sw) << 4)),
+                         "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                         : "memory");
           }
         }
+        fence_proxy_async_smem();
+        if (!group_sync()) {
+          ok = false;
+          break;
+        }
+        if (lrow == 0) {
+          tma_store_4d(grp == 0 ? &tmDV : &tmDK, stg, 0, it.row0, it.head, it.b);
+          bulk_commit_group();
+        }
+        acc_pending = true;
+        acc_par = par;
       }
-      tc_fence_before();
-      mbar_arrive(bar(C::B_ACCEMPTY));
       ++ic;
     }
     if (lrow == 0) bulk_wait_group0();               // reduces done before the CTA exits
@@ -1071,12 +1113,15 @@ cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* 
   if constexpr (DH <= 64) {
     using H = BwdHalfCfg<DH>;
     auto hk = gdpa_bwd_half_kernel<DH, PHI>;
-    CUtensorMap mdq;
+    CUtensorMap mdq, mdv, mdk, unused_q, unused_g;
     if (!make_dq_map<DH>(p, dq_acc, &mdq)) return cudaErrorInvalidValue;
+    // the outputs dV, dK have the layout (and so the maps) of the inputs K, V
+    if (!make_bwd_maps<DH>(p, q, g, dk, dv, &unused_q, &unused_g, &mdk, &mdv))
+      return cudaErrorInvalidValue;
     e = cudaFuncSetAttribute(hk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H::SMEM);
     if (e != cudaSuccess) return e;
     KernelScope ks_("gdpa_bwd_sm100", st);
-    hk<<<device_sm_count(), kThreads, H::SMEM, st>>>(mq, mg, mk, mv, mdq, args);
+    hk<<<device_sm_count(), kThreads, H::SMEM, st>>>(mq, mg, mk, mv, mdq, mdv, mdk, args);
     return cudaGetLastError();
   }
   KernelScope ks_("gdpa_bwd_sm100", st);
