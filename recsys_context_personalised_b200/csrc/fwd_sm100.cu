@@ -96,8 +96,16 @@ struct FwdCfg {
                        B_OEMPTY = 10, B_DRAIN = 12, B_KVFULL = 13, B_KVEMPTY = 13 + NS,
                        NBAR = 13 + 2 * NS;
   static constexpr uint32_t OFF_Q = 0, OFF_KV = QST * 2 * TILEB;
+  // O epilogue: per activation warp, 32 rows x 64 columns of bf16 (128 B rows)
+  // to turn its rows into whole-line global stores
+  static constexpr uint32_t OSTG_WARP = 32 * 128;
+  static constexpr uint32_t OFF_OSTG = OFF_KV + NS * TILEB;
+  static constexpr uint32_t OFF_CTL = OFF_OSTG + 8 * OSTG_WARP;   // barriers, TMEM slot, abort flag
   static constexpr uint32_t CTL_BYTES = 1024;
-  static constexpr uint32_t SMEM_USED = 1024 + OFF_KV + NS * TILEB + CTL_BYTES;
+  static constexpr uint32_t SMEM_USED = 1024 + OFF_CTL + CTL_BYTES;
+  static_assert(OFF_KV >= QST * 2 * TILEB && OFF_OSTG >= OFF_KV + NS * TILEB &&
+                    OFF_CTL >= OFF_OSTG + 8 * OSTG_WARP,
+                "shared-memory regions overlap");
   // at least 120 KB so that two CTAs never share an SM (each allocates all 512 TMEM columns)
   static constexpr uint32_t SMEM = SMEM_USED > 120u * 1024u ? SMEM_USED : 120u * 1024u;
   static_assert(SMEM <= 232448u, "exceeds the 227 KB of shared memory a CTA can have");
@@ -139,7 +147,7 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t sQ = base + C::OFF_Q;
   const uint32_t sKV = base + C::OFF_KV;
-  uint8_t* ctl = gbase + C::OFF_KV + C::NS * C::TILEB;
+  uint8_t* ctl = gbase + C::OFF_CTL;
   const uint32_t bar0 = smem_u32(ctl);
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 8 * C::NBAR);
@@ -502,26 +510,59 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       tc_fence_after();
       const float inv = SOFTMAX ? 1.f / l_run : 1.f;
       const bool store = row < tl.rows;
-      __nv_bfloat16* orow = a.o + ((int64_t)(tl.row0 + row) * a.h + tl.head) * DH;
+      {
+        // Each lane owns one O row.  The warp passes its 32 rows through
+        // shared memory (64 columns at a time, rows swizzled by 16-byte
+        // chunk) so that every global store instruction writes whole rows:
+        // CPR lanes per row, 32 / CPR rows per instruction.
+        constexpr int PC = DH < 64 ? DH : 64;           // columns per pass
+        constexpr int CPR = PC / 8;                     // 16-byte chunks per row
+        constexpr int RPI = 32 / CPR;                   // rows per store instruction
+        const uint32_t ostg = base + C::OFF_OSTG + (uint32_t)(warp - 4) * C::OSTG_WARP;
+        auto chunk_addr = [&](int r, int j) -> uint32_t {
+          const int sw = CPR == 8 ? (r & 7) : ((r >> 1) & 3);
+          return ostg + (uint32_t)(r * CPR * 16) + ((uint32_t)(j ^ sw) << 4);
+        };
+        const int rl = lane / CPR, jl = lane % CPR;      // read-back: row in group, chunk
 #pragma unroll
-      for (int c = 0; c < DH; c += 16) {
-        uint32_t v[16];
-        tmem_ld_x16(my_o + c, v);
-        tmem_wait_ld();
-        uint32_t pk[8];
+        for (int c0 = 0; c0 < DH; c0 += PC) {
+          uint32_t v[PC];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv, __uint_as_float(v[2 * i + 1]) * inv);
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          for (int c = 0; c < PC; c += 16)
+            tmem_ld_x16(my_o + c0 + c, *reinterpret_cast<uint32_t(*)[16]>(&v[c]));
+          tmem_wait_ld();
+          if (c0 + PC == DH) {
+            tc_fence_before();
+            mbar_arrive(bar(C::B_OEMPTY + grp));        // the O accumulator is free
+          }
+#pragma unroll
+          for (int j = 0; j < CPR; ++j) {
+            const uint32_t p0 = pack_bf16x2(__uint_as_float(v[8 * j]) * inv, __uint_as_float(v[8 * j + 1]) * inv);
+            const uint32_t p1 = pack_bf16x2(__uint_as_float(v[8 * j + 2]) * inv, __uint_as_float(v[8 * j + 3]) * inv);
+            const uint32_t p2 = pack_bf16x2(__uint_as_float(v[8 * j + 4]) * inv, __uint_as_float(v[8 * j + 5]) * inv);
+            const uint32_t p3 = pack_bf16x2(__uint_as_float(v[8 * j + 6]) * inv, __uint_as_float(v[8 * j + 7]) * inv);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(chunk_addr(lane, j)),
+                         "r"(p0), "r"(p1), "r"(p2), "r"(p3)
+                         : "memory");
+          }
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < CPR; ++it) {
+            const int r = it * RPI + rl;                  // row within this warp's 32
+            uint4 val;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                         : "r"(chunk_addr(r, jl)));
+            const int tr = quad * 32 + r;                 // tile row
+            if (tr < tl.rows)
+              *reinterpret_cast<uint4*>(a.o + ((int64_t)(tl.row0 + tr) * a.h + tl.head) * DH + c0 +
+                                        jl * 8) = val;
+          }
+          __syncwarp();
         }
       }
       if (SOFTMAX && store && a.lse != nullptr)
         a.lse[(int64_t)tl.head * a.T + tl.row0 + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
-      tc_fence_before();
-      mbar_arrive(bar(C::B_OEMPTY + grp));
       ++oc;
     }
   }
