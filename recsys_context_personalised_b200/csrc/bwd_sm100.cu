@@ -48,27 +48,48 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // Zeroes the fp32 dQ workspace and, for softmax, writes D[head, t] =
 // sum_d dO[t, head, d] * O[t, head, d] (one warp per (t, head) row).
-__global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
-                                const __nv_bfloat16* __restrict__ g, float* __restrict__ dsum,
-                                float4* __restrict__ dq_acc, int64_t rows, int h, int dh,
-                                int64_t T, int softmax) {
-  const int64_t n4 = rows * dh / 4;
+template <int DH>
+__global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ g,
+                                float* __restrict__ dsum, float4* __restrict__ dq_acc,
+                                int64_t rows, int h, int64_t T, int softmax) {
+  const int64_t n4 = rows * DH / 4;
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t nth = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = tid; i < n4; i += nth) dq_acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (!softmax) return;
-  const int lane = threadIdx.x & 31;
-  for (int64_t row = tid >> 5; row < rows; row += nth >> 5) {
-    float acc = 0.f;
-    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(o + row * dh);
-    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(g + row * dh);
-    for (int d = lane; d < dh / 2; d += 32) {
-      const float2 a = __bfloat1622float2(o2[d]), b = __bfloat1622float2(g2[d]);
-      acc = fmaf(a.x, b.x, fmaf(a.y, b.y, acc));
+  // D of a (token, head) row: CPR lanes take one 16-byte piece of O and dO
+  // each; a warp covers RPW rows per step and U steps per iteration, so that
+  // 2U 16-byte loads per thread are in flight.
+  constexpr int CPR = DH / 8, RPW = 32 / CPR, U = 4;
+  const int lane = threadIdx.x & 31, sub = lane / CPR, piece = lane % CPR;
+  const int64_t warp = tid >> 5, nwarps = nth >> 5;
+  for (int64_t r0 = warp * (RPW * U); r0 < rows; r0 += nwarps * (RPW * U)) {
+    uint4 x[U], y[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t row = r0 + u * RPW + sub;
+      x[u] = y[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (row < rows) {
+        x[u] = o[row * CPR + piece];
+        y[u] = g[row * CPR + piece];
+      }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) dsum[(int64_t)(row % h) * T + row / h] = acc;
+    for (int u = 0; u < U; ++u) {
+      const uint32_t xa[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+      const uint32_t ya[4] = {y[u].x, y[u].y, y[u].z, y[u].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xa[e]));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ya[e]));
+        acc = fmaf(a.x, b.x, fmaf(a.y, b.y, acc));
+      }
+#pragma unroll
+      for (int off = CPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      const int64_t row = r0 + u * RPW + sub;
+      if (piece == 0 && row < rows) dsum[(int64_t)(row % h) * T + row / h] = acc;
+    }
   }
 }
 
@@ -1164,10 +1185,12 @@ cudaError_t launch_sm100_bwd(const gdpa_problem_t& p, const void* q, const int32
   const int sms = device_sm_count();
   if (rows > 0) {
     KernelScope ks_("gdpa_bwd_prep", st);
-    bwd_prep_kernel<<<sms * 8, 256, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dout),
-        dsum, reinterpret_cast<float4*>(dq_acc), rows, p.h, p.dh, p.total_tokens,
-        p.phi == GDPA_PHI_SOFTMAX ? 1 : 0);
+    auto prep = p.dh == 32 ? bwd_prep_kernel<32> : p.dh == 64 ? bwd_prep_kernel<64>
+                                                              : bwd_prep_kernel<128>;
+    prep<<<sms * 8, 256, 0, st>>>(reinterpret_cast<const uint4*>(o),
+                                  reinterpret_cast<const uint4*>(dout), dsum,
+                                  reinterpret_cast<float4*>(dq_acc), rows, p.h, p.total_tokens,
+                                  p.phi == GDPA_PHI_SOFTMAX ? 1 : 0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
