@@ -874,6 +874,9 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         return true;
       };
+      // LSE (natural log) and D of the next tile's rows: raw loads, consumed
+      // only when they are written to shared memory, so they stay in flight
+      // while the warp waits for and processes the current tile
       float nl[2] = {0.f, 0.f}, nd[2] = {0.f, 0.f};
       auto load_stats = [&](int ii) {
 #pragma unroll
@@ -883,8 +886,8 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
           nd[u] = 0.f;
           if (rg < n) {
             const int64_t at = (int64_t)it.head * a.T + t0 + rg;
-            nl[u] = a.lse[at] * 1.4426950408889634f;
-            nd[u] = a.dsum[at];
+            nl[u] = __ldg(a.lse + at);
+            nd[u] = __ldg(a.dsum + at);
           }
         }
       };
@@ -896,7 +899,7 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
           __syncwarp();
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            wst[32 * u + lane] = nl[u];
+            wst[32 * u + lane] = nl[u] * 1.4426950408889634f;   // log2 units
             wst[64 + 32 * u + lane] = nd[u];
           }
           __syncwarp();
