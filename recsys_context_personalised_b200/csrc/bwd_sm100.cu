@@ -17,15 +17,17 @@
 //   dV  += P^T dO_i         A = P^T (TMEM, bf16),   B = dO_i (smem, MN-major)
 //   dK  += dS^T Q_i         A = dS^T (smem, K-major), B = Q_i (MN-major)
 //   dQ_i = dS K             A = dS (the same smem bytes read MN-major), B = K (MN-major)
-// dQ_i (lane = query row) is added into an fp32 workspace with vector
-// reductions; a last kernel scales it by s and rounds it to bf16.
+// dQ_i (lane = query row) is added into an fp32 workspace; a last kernel
+// scales it by s and rounds it to bf16.
 //
-// CTA = 12 warps, one persistent CTA per SM, static round-robin over a work
-// list sorted by sample length (longest first):
-//   warp 0 TMA producer, warp 1 MMA issuer, warp 2 TMEM allocator,
-//   warps 4-7 and 8-11: the two activation groups, splitting each query tile's
-//   128 rows in halves; they also drain dQ_i and, at the end of an item, store
-//   dV (group 0) and dK (group 1).
+// One persistent CTA per SM, static round-robin over a work list sorted by
+// sample length (longest first).  Two kernels:
+//   - dh = 128 (gdpa_bwd_sm100_kernel, 12 warps): warp 0 TMA producer, warp 1
+//     MMA issuer, warp 2 TMEM allocator, warps 4-7 and 8-11 the activation
+//     groups (halves of each tile's 128 rows), which also drain dQ_i with
+//     vector reductions and store dV (group 0) and dK (group 1);
+//   - dh <= 64 (gdpa_bwd_half_kernel, 16 warps): a half-tile pipeline with a
+//     separate drain warpgroup and bulk tensor copies (described below).
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -549,7 +551,7 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   if (warp == 2) tmem_dealloc(tmem, 512);
 }
 
-// ---------------------------------------------------------------- half-tile pipeline (dh <= 64)
+// ---------------------------------------------------------------- half-tile kernel (dh <= 64)
 //
 // Same products as above, but each 128-row query tile is processed as two
 // 64-row halves with their own S^T/dP^T buffers in TMEM, so that activation
@@ -563,47 +565,73 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 // TMEM: S^T_h [128h, 128h+64), dP^T_h [128h+64, 128h+128) (P^T_h aliases the
 // first 32 columns of S^T_h), dV [256, 256+dh), dK [256+dh, 256+2dh),
 // dQ_c [256+2dh+c*dh, 256+3dh+c*dh).
+//
+// Schedule:
+//   - K/V have two slots, so the producer loads the next item's key block and
+//     query tiles while the current item runs, and the MMA thread issues the
+//     next item's first S^T/dP^T products right after the current item's dQ;
+//   - a fourth warpgroup (warps 12-15, one per TMEM lane quadrant) drains dQ
+//     (bulk reduce-add) and dV/dK (bulk store), and warp 2 loads the softmax
+//     row statistics one tile ahead, so the two activation groups only form
+//     P^T and dS^T.
+// The drain group stages each tile's dQ, and an item's dV/dK, in the tile's
+// own dS^T buffer: its readers are all in the completed products.  Before the
+// MMA thread issues the S^T products of the tile that will overwrite a buffer
+// (two tiles later), it waits on STGFREE of that buffer, which the drain group
+// arrives on once its bulk copies have read the staging area.
+// Registers (512 threads at 128 each): warps 0-3 drop to 72, the drain group
+// to 104, the activation groups rise to 168 (4 x 128 x (72+104+168+168) = 65536).
+constexpr int kHalfThreads = 512;
+
 template <int DH>
 struct BwdHalfCfg {
   static_assert(DH <= 64, "half-tile pipeline needs dh <= 64");
-  static constexpr int CH = DH;
-  static constexpr uint32_t ROWB = CH * 2;
+  static constexpr uint32_t ROWB = DH * 2;
   static constexpr uint32_t TILEB = 128 * ROWB;            // [128 x DH] bf16
   static constexpr uint32_t SW = DH < 64 ? kSw64 : kSw128;
   static constexpr uint32_t ATOM = 8 * ROWB;
-  static constexpr int NSTG = 2;
-  static constexpr uint32_t DSB = 2 * 128 * 128;           // one dS^T buffer
+  static constexpr int NSTG = 2, NKV = 2;
+  static constexpr uint32_t DSB = 2 * 128 * 128;           // one dS^T buffer, two 16 KB halves
   static constexpr uint32_t COL_DV = 256, COL_DK = 256 + DH, COL_DQ = 256 + 2 * DH;
-  static constexpr int B_KVFULL = 0, B_KVEMPTY = 1, B_SFULL = 2, B_PFULL = 4, B_DQFULL = 6,
-                       B_DQEMPTY = 8, B_ACCFULL = 10, B_ACCEMPTY = 11, B_DRAIN = 12,
-                       B_DQSYNC = 13, B_STFULL = 15, B_STEMPTY = 15 + NSTG,
-                       NBAR = 15 + 2 * NSTG;
-  static constexpr uint32_t OFF_K = 0, OFF_V = TILEB, OFF_STG = 2 * TILEB;
+  // staging rows: DH/2 fp32 (dQ box) or DH bf16 (dV/dK box), both 2*DH bytes
+  static constexpr uint32_t SROWB = 2 * DH;
+  static constexpr int B_KVFULL = 0, B_KVEMPTY = 2, B_SFULL = 4, B_PFULL = 6, B_DQFULL = 8,
+                       B_DQEMPTY = 10, B_ACCFULL = 12, B_ACCEMPTY = 13, B_DRAIN = 14,
+                       B_DSYNC = 15, B_STGFREE = 16, B_STFULL = 18, B_STEMPTY = 18 + NSTG,
+                       B_STATFULL = 18 + 2 * NSTG, B_STATEMPTY = 20 + 2 * NSTG,
+                       NBAR = 22 + 2 * NSTG;
+  static constexpr uint32_t OFF_KV = 0;                    // slot s: K at 2s TILEB, V at (2s+1) TILEB
+  static constexpr uint32_t OFF_STG = NKV * 2 * TILEB;
   static constexpr uint32_t OFF_DS = OFF_STG + NSTG * 2 * TILEB;
-  // dQ staging for the bulk reduce, one per group: [128 rows][DH/2 fp32], laid
-  // out with the swizzle of the reduce's tensor map (128 B rows: 128B, 64 B rows: 64B)
-  static constexpr uint32_t DQROWB = DH / 2 * 4;
-  static constexpr uint32_t DQSTGB = 128 * DQROWB;
-  static constexpr uint32_t OFF_DQS = OFF_DS + 2 * DSB;
-  static constexpr uint32_t OFF_CTL = OFF_DQS + 2 * DQSTGB;
-  static constexpr uint32_t CTL_BYTES = 1024 + 8 * 2 * 128 * 4;
+  static constexpr uint32_t OFF_CTL = OFF_DS + 2 * DSB;
+  // + a two-slot ring of row statistics: [slot][log2-scaled LSE, D][128 rows] fp32
+  static constexpr uint32_t CTL_BYTES = 1024 + 2 * 2 * 128 * 4;
   static constexpr uint32_t SMEM_USED = 1024 + OFF_CTL + CTL_BYTES;
   static constexpr uint32_t SMEM = SMEM_USED > 120u * 1024u ? SMEM_USED : 120u * 1024u;
   static_assert(SMEM <= 232448u, "exceeds the 227 KB of shared memory a CTA can have");
   static_assert(COL_DQ + 2 * DH <= 512, "TMEM columns");
-  static_assert(OFF_DQS % 1024 == 0 && DQSTGB % 1024 == 0, "swizzle atoms need 1024-B alignment");
-  static_assert(8 * NBAR <= 1016, "barriers, TMEM slot and abort flag share the first 1 KB");
+  static_assert(128 * SROWB <= DSB / 2, "a staging box fits in a dS^T half");
+  static_assert(OFF_STG % 1024 == 0 && OFF_DS % 1024 == 0, "swizzle atoms need 1024-B alignment");
+  static_assert(8 * NBAR + 8 <= 1024, "barriers, TMEM slot and abort flag share the first 1 KB");
 };
 
+// 16-byte chunk j of staging row r, swizzled like the bulk copies' maps
+// (128 B rows: 128B swizzle, 64 B rows: 64B swizzle)
+template <int DH>
+__device__ __forceinline__ uint32_t stage_chunk(uint32_t box, int r, int j) {
+  const int sw = DH == 64 ? (r & 7) : ((r >> 1) & 3);
+  return box + (uint32_t)(r * 2 * DH) + ((uint32_t)(j ^ sw) << 4);
+}
+
 template <int DH, int PHI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kHalfThreads, 1)
 gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
-                     const __grid_constant__ CUtensorMap tmG,
-                     const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV,
-                     const __grid_constant__ CUtensorMap tmDQ,
-                     const __grid_constant__ CUtensorMap tmDV,
-                     const __grid_constant__ CUtensorMap tmDK, const BwdArgs a) {
+                   const __grid_constant__ CUtensorMap tmG,
+                   const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV,
+                   const __grid_constant__ CUtensorMap tmDQ,
+                   const __grid_constant__ CUtensorMap tmDV,
+                   const __grid_constant__ CUtensorMap tmDK, const BwdArgs a) {
   using C = BwdHalfCfg<DH>;
   constexpr bool SOFTMAX = PHI == GDPA_PHI_SOFTMAX;
   constexpr uint32_t IDESC_T = idesc_bf16(128, 64, 0, 0);    // S^T, dP^T of a half: N = 64 rows
@@ -614,30 +642,31 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V, sStg = base + C::OFF_STG;
-  const uint32_t sDS = base + C::OFF_DS;
+  const uint32_t sKV = base + C::OFF_KV, sStg = base + C::OFF_STG, sDS = base + C::OFF_DS;
   uint8_t* ctl = gbase + C::OFF_CTL;
   const uint32_t bar0 = smem_u32(ctl);
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 8 * C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 8 * C::NBAR + 4);
-  float* stats = reinterpret_cast<float*>(ctl + 1024);   // [8 warps][2][128]
+  float* stats = reinterpret_cast<float*>(ctl + 1024);   // [2 slots][LSE, D][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    mbar_init(bar(C::B_KVFULL), 1);
-    mbar_init(bar(C::B_KVEMPTY), 1);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::B_KVFULL + i), 1);
+      mbar_init(bar(C::B_KVEMPTY + i), 1);
       mbar_init(bar(C::B_SFULL + i), 1);
       mbar_init(bar(C::B_PFULL + i), 128);
       mbar_init(bar(C::B_DQFULL + i), 1);
-      mbar_init(bar(C::B_DQEMPTY + i), 256);
+      mbar_init(bar(C::B_DQEMPTY + i), 128);
+      mbar_init(bar(C::B_STGFREE + i), 1);
+      mbar_init(bar(C::B_STATFULL + i), 1);
+      mbar_init(bar(C::B_STATEMPTY + i), 8);       // lane 0 of each activation warp
     }
     mbar_init(bar(C::B_ACCFULL), 1);
-    mbar_init(bar(C::B_ACCEMPTY), 256);
+    mbar_init(bar(C::B_ACCEMPTY), 128);
     mbar_init(bar(C::B_DRAIN), 1);
-    mbar_init(bar(C::B_DQSYNC + 0), 128);
-    mbar_init(bar(C::B_DQSYNC + 1), 128);
+    mbar_init(bar(C::B_DSYNC), 128);
     for (int i = 0; i < C::NSTG; ++i) {
       mbar_init(bar(C::B_STFULL + i), 1);
       mbar_init(bar(C::B_STEMPTY + i), 1);
@@ -663,21 +692,31 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int count = a.ws->status == GDPA_ERR_INVALID_ARG ? 0 : a.ws->tile_count;
+  const int wg = warp >> 2;
+  auto next_item = [&](int t) -> int {            // next item of this CTA with query rows
+    while (t < count && a.tiles[t].rows == 0) t += gridDim.x;
+    return t;
+  };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t ic = 0, stage = 0, sphase = 0;
+  if (wg == 0) {
+    setmaxnreg_dec<72>();
+    if (warp == 0 && lane == 0) {
+      // -------------------------------------------------------- producer
+      // runs up to one item ahead: K/V of the next item go to the other slot
+      uint32_t kvi = 0, stage = 0, sphase = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
         const Tile it = a.tiles[t];
         if (it.rows == 0) continue;
         const int nq = (it.rows + 127) >> 7;
         const int t0 = a.offsets[it.b];
-        if (!mbar_wait(bar(C::B_KVEMPTY), (ic & 1u) ^ 1u, abort_flag, kTimeoutNs)) break;
-        mbar_expect_tx(bar(C::B_KVFULL), 2 * C::TILEB);
-        tma_load_4d(sK, &tmK, bar(C::B_KVFULL), 0, it.row0, it.head, it.b);
-        tma_load_4d(sV, &tmV, bar(C::B_KVFULL), 0, it.row0, it.head, it.b);
+        const uint32_t slot = kvi & 1u;
+        if (!mbar_wait(bar(C::B_KVEMPTY + slot), ((kvi >> 1) & 1u) ^ 1u, abort_flag, kTimeoutNs))
+          break;
+        const uint32_t sK = sKV + slot * 2 * C::TILEB;
+        mbar_expect_tx(bar(C::B_KVFULL + slot), 2 * C::TILEB);
+        tma_load_4d(sK, &tmK, bar(C::B_KVFULL + slot), 0, it.row0, it.head, it.b);
+        tma_load_4d(sK + C::TILEB, &tmV, bar(C::B_KVFULL + slot), 0, it.row0, it.head, it.b);
         for (int i = 0; i < nq; ++i) {
           if (!mbar_wait(bar(C::B_STEMPTY + stage), sphase ^ 1u, abort_flag, kTimeoutNs)) {
             ok = false;
@@ -692,30 +731,41 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
             sphase ^= 1u;
           }
         }
-        ++ic;
+        ++kvi;
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t ic = 0, stage = 0, sphase = 0, qs = 0;
+    } else if (warp == 1 && lane == 0) {
+      // -------------------------------------------------------- MMA issuer
+      uint32_t stage = 0, sphase = 0, qs = 0, kvi = 0;
       bool ok = true;
-      const uint64_t dk0 = smem_desc(sK, 16, C::ATOM, C::SW), dv0 = smem_desc(sV, 16, C::ATOM, C::SW);
-      const uint64_t kmn0 = smem_desc(sK, C::TILEB, C::ATOM, C::SW);       // K, MN-major (dQ)
-      // ST(h): S^T_h = K Q[64h..64h+63]^T and dP^T_h = V dO[64h..64h+63]^T of the tile in `st`
-      auto issue_st = [&](uint32_t st, int h) {
+      // slot 0's descriptors; slot s starts s * 2 * TILEB bytes further
+      const uint64_t dk0 = smem_desc(sKV, 16, C::ATOM, C::SW);                 // K, K-major (S^T)
+      const uint64_t dv0 = smem_desc(sKV + C::TILEB, 16, C::ATOM, C::SW);      // V, K-major (dP^T)
+      const uint64_t kmn0 = smem_desc(sKV, C::TILEB, C::ATOM, C::SW);          // K, MN-major (dQ)
+      auto wait_bar = [&](int which, uint32_t ph) -> bool {
+        if (!mbar_wait(bar(which), ph, abort_flag, kTimeoutNs)) return false;
+        tc_fence_after();
+        return true;
+      };
+      // ST(q, h): S^T_h = K Q[64h..]^T and dP^T_h = V dO[64h..]^T of tile q, in stage `st`.
+      // Before half 0, the drain group must be done with tile q-2's staging in
+      // the dS^T buffer that tile q's activation will write.
+      auto issue_st = [&](uint32_t q, uint32_t st, int h, uint32_t slot) -> bool {
+        if (h == 0 && !wait_bar(C::B_STGFREE + (int)(q & 1u), ((q >> 1) & 1u) ^ 1u)) return false;
         const uint32_t qaddr = sStg + st * 2 * C::TILEB + 64 * h * C::ROWB;
         const uint64_t q0 = smem_desc(qaddr, 16, C::ATOM, C::SW);
         const uint64_t g0 = smem_desc(qaddr + C::TILEB, 16, C::ATOM, C::SW);
+        const uint64_t dk = desc_advance(dk0, slot * 2 * C::TILEB);
+        const uint64_t dv = desc_advance(dv0, slot * 2 * C::TILEB);
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k)
-          mma_ss(tmem + 128 * h, desc_advance(dk0, k * 32), desc_advance(q0, k * 32), IDESC_T,
+          mma_ss(tmem + 128 * h, desc_advance(dk, k * 32), desc_advance(q0, k * 32), IDESC_T,
                  k > 0 ? 1u : 0u);
 #pragma unroll
         for (int k = 0; k < DH / 16; ++k)
-          mma_ss(tmem + 128 * h + 64, desc_advance(dv0, k * 32), desc_advance(g0, k * 32), IDESC_T,
+          mma_ss(tmem + 128 * h + 64, desc_advance(dv, k * 32), desc_advance(g0, k * 32), IDESC_T,
                  k > 0 ? 1u : 0u);
         mma_commit(bar(C::B_SFULL + h));
+        return true;
       };
       // dVdK(h): dV += P^T_h dO[64h..], dK += dS^T[64h..] Q[64h..] of the tile in `st`
       auto issue_dvdk = [&](uint32_t st, int h, uint32_t c, bool first) {
@@ -732,193 +782,154 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
           mma_ss(tmem + C::COL_DK, desc_advance(dsk, k * 32), desc_advance(qmn, k * 2 * C::ATOM),
                  IDESC_KV, (first && k == 0) ? 0u : 1u);
       };
-      auto wait_stage = [&](uint32_t st, uint32_t ph) -> bool {
-        if (!mbar_wait(bar(C::B_STFULL + st), ph, abort_flag, kTimeoutNs)) return false;
-        tc_fence_after();
-        return true;
-      };
-      for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
-        const Tile it = a.tiles[t];
-        if (it.rows == 0) continue;
-        const int nq = (it.rows + 127) >> 7;
-        if (!mbar_wait(bar(C::B_KVFULL), ic & 1u, abort_flag, kTimeoutNs)) break;
-        tc_fence_after();
-        if (!wait_stage(stage, sphase)) break;
-        issue_st(stage, 0);
-        issue_st(stage, 1);
-        for (int i = 0; i < nq; ++i, ++qs) {
+      // One pass over every (item, query tile) of this CTA.
+      int t = next_item(blockIdx.x);
+      if (t < count) {
+        int nq = (a.tiles[t].rows + 127) >> 7;
+        uint32_t slot = 0;
+        ok = wait_bar(C::B_KVFULL + 0, 0) && wait_bar(C::B_STFULL + stage, sphase) &&
+             issue_st(0, stage, 0, slot) && issue_st(0, stage, 1, slot);
+        for (int i = 0; ok;) {
           const uint32_t c = qs & 1u;
+          const bool last = i + 1 == nq;
+          const int tn = last ? next_item(t + gridDim.x) : t;
+          const bool has_next = tn < count;
+          const uint32_t nslot = last ? slot ^ 1u : slot;
+          const uint32_t nkvi = last ? kvi + 1 : kvi;
           uint32_t nst = stage + 1, nph = sphase;
           if (nst == (uint32_t)C::NSTG) {
             nst = 0;
             nph ^= 1u;
           }
-          // half 0 of tile i, then the next tile's half-0 products
-          if (!mbar_wait(bar(C::B_PFULL + 0), qs & 1u, abort_flag, kTimeoutNs) ||
-              (i == 0 && !mbar_wait(bar(C::B_ACCEMPTY), (ic & 1u) ^ 1u, abort_flag, kTimeoutNs))) {
+          // half 0 of this tile, then (within an item) the next tile's half-0 products
+          if (!wait_bar(C::B_PFULL + 0, c) ||
+              (i == 0 && !wait_bar(C::B_ACCEMPTY, (kvi & 1u) ^ 1u))) {
             ok = false;
             break;
           }
-          tc_fence_after();
           issue_dvdk(stage, 0, c, i == 0);
-          if (i + 1 < nq) {
-            if (!wait_stage(nst, nph)) {
+          if (has_next && !last) {
+            if (!wait_bar(C::B_STFULL + nst, nph) || !issue_st(qs + 1, nst, 0, nslot)) {
               ok = false;
               break;
             }
-            issue_st(nst, 0);
           }
-          // half 1, the tile's dQ, then the next tile's half-1 products
-          if (!mbar_wait(bar(C::B_PFULL + 1), qs & 1u, abort_flag, kTimeoutNs)) {
+          // half 1 and the tile's dQ
+          if (!wait_bar(C::B_PFULL + 1, c)) {
             ok = false;
             break;
           }
-          tc_fence_after();
           issue_dvdk(stage, 1, c, false);
           mma_commit(bar(C::B_STEMPTY + stage));
-          if (!mbar_wait(bar(C::B_DQEMPTY + c), ((qs >> 1) & 1u) ^ 1u, abort_flag, kTimeoutNs)) {
+          if (!wait_bar(C::B_DQEMPTY + c, ((qs >> 1) & 1u) ^ 1u)) {
             ok = false;
             break;
           }
-          tc_fence_after();
           {
             const uint64_t dsm = smem_desc(sDS + c * C::DSB, 16384, 1024, kSw128);   // dS, MN-major
+            const uint64_t kmn = desc_advance(kmn0, slot * 2 * C::TILEB);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
               mma_ss(tmem + C::COL_DQ + c * DH, desc_advance(dsm, k * 2048),
-                     desc_advance(kmn0, k * 2 * C::ATOM), IDESC_Q, k > 0 ? 1u : 0u);
+                     desc_advance(kmn, k * 2 * C::ATOM), IDESC_Q, k > 0 ? 1u : 0u);
             mma_commit(bar(C::B_DQFULL + c));
           }
-          if (i + 1 < nq) issue_st(nst, 1);
+          if (last) {
+            mma_commit(bar(C::B_KVEMPTY + slot));
+            mma_commit(bar(C::B_ACCFULL));
+            // the next item's first products, once this item's are all issued
+            if (has_next &&
+                (!wait_bar(C::B_KVFULL + nslot, (nkvi >> 1) & 1u) ||
+                 !wait_bar(C::B_STFULL + nst, nph) || !issue_st(qs + 1, nst, 0, nslot))) {
+              ok = false;
+              break;
+            }
+          }
+          if (has_next && !issue_st(qs + 1, nst, 1, nslot)) {
+            ok = false;
+            break;
+          }
           stage = nst;
           sphase = nph;
+          ++qs;
+          if (!has_next) break;
+          if (last) {
+            t = tn;
+            nq = (a.tiles[t].rows + 127) >> 7;
+            slot = nslot;
+            kvi = nkvi;
+            i = 0;
+          } else {
+            ++i;
+          }
         }
-        if (!ok) break;
-        mma_commit(bar(C::B_KVEMPTY));
-        mma_commit(bar(C::B_ACCFULL));
-        ++ic;
       }
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ activation groups
-    const int grp = (warp - 4) >> 2;                   // the 64-row half this group owns
+    else if (warp == 2 && SOFTMAX) {
+      // -------------------------------------------------------- row statistics
+      // log2-scaled LSE and D of each query tile into the ring, one tile ahead
+      uint32_t q = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
+        const Tile it = a.tiles[t];
+        if (it.rows == 0) continue;
+        const int nq = (it.rows + 127) >> 7;
+        const int t0 = a.offsets[it.b];
+        for (int i = 0; i < nq; ++i, ++q) {
+          const uint32_t slot = q & 1u;
+          const bool w = mbar_wait(bar(C::B_STATEMPTY + (int)slot), ((q >> 1) & 1u) ^ 1u,
+                                   abort_flag, kTimeoutNs);
+          if (!__all_sync(0xffffffffu, w)) {
+            ok = false;
+            break;
+          }
+          float* ring = stats + slot * 256;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int r = 32 * u + lane, rg = 128 * i + r;
+            float l = 0.f, d = 0.f;
+            if (rg < it.rows) {
+              const int64_t at = (int64_t)it.head * a.T + t0 + rg;
+              l = __ldg(a.lse + at) * 1.4426950408889634f;
+              d = __ldg(a.dsum + at);
+            }
+            ring[r] = l;
+            ring[128 + r] = d;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(C::B_STATFULL + (int)slot));
+        }
+      }
+    }
+  } else if (wg <= 2) {
+    // ---------------------------------------------------------- activation groups
+    setmaxnreg_inc<168>();
+    const int grp = wg - 1;                            // the 64-row half this group owns
     const int quad = warp & 3;
-    const int lrow = quad * 32 + lane;                 // TMEM lane: key (S^T, dV, dK) or row (dQ)
+    const int lrow = quad * 32 + lane;                 // TMEM lane: key
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    float* wst = stats + (warp - 4) * 256;
     const float c2 = a.scale_log2, sc = a.scale, half_sc = 0.5f * a.scale;
-    const uint32_t sDQS = base + C::OFF_DQS + grp * C::DQSTGB;
-    uint32_t ic = 0, qs = 0, dq_sync_phase = 0;
-    // a dV/dK bulk store may still be reading the dS^T half of buffer acc_par
-    bool acc_pending = false;
-    uint32_t acc_par = 0;
+    uint32_t qs = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
       const Tile it = a.tiles[t];
       const int n = it.rows;
-      const int key = it.row0 + lrow;
-      __nv_bfloat16* kvout = (grp == 0 ? a.dv : a.dk) +
-                             (((int64_t)it.b * a.h + it.head) * a.m + key) * DH;
-      if (n == 0) {                                    // no tokens: dK = dV = 0
-        if (key < a.m) {
-          uint4* d4 = reinterpret_cast<uint4*>(kvout);
-#pragma unroll
-          for (int c = 0; c < DH / 8; ++c) d4[c] = make_uint4(0u, 0u, 0u, 0u);
-        }
-        continue;
-      }
+      if (n == 0) continue;
       const int nq = (n + 127) >> 7;
-      const int t0 = a.offsets[it.b];
-      // dQ of tile ii (buffer step & 1): lane = query row.  The group stages its
-      // half of the columns in shared memory and one thread adds the whole
-      // [128 x DH/2] box into the fp32 accumulator with one bulk reduce.  Rows
-      // past the sample carry exact zeros (their dS entries are zero), so the
-      // box may overlap the next sample; rows past T are clipped by the map.
-      auto group_sync = [&]() -> bool {
-        mbar_arrive(bar(C::B_DQSYNC + grp));
-        const bool w = mbar_wait(bar(C::B_DQSYNC + grp), dq_sync_phase, abort_flag, kTimeoutNs);
-        dq_sync_phase ^= 1u;
-        return __all_sync(0xffffffffu, w);
-      };
-      auto drain_dq = [&](int ii, uint32_t step) -> bool {
-        const uint32_t b = step & 1u;
-        const bool w = mbar_wait(bar(C::B_DQFULL + b), (step >> 1) & 1u, abort_flag, kTimeoutNs);
-        if (!__all_sync(0xffffffffu, w)) return false;
-        tc_fence_after();
-        uint32_t v[DH / 2];
-        const uint32_t src = tmem + lane_off + C::COL_DQ + b * DH + grp * (DH / 2);
-        if constexpr (DH == 64)
-          tmem_ld_x32(src, v);
-        else
-          tmem_ld_x16(src, v);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(C::B_DQEMPTY + b));
-        // the previous reduce from the staging area (and any dV/dK store) must
-        // have finished reading shared memory
-        if (lrow == 0) bulk_wait_group_read0();
-        if (!group_sync()) return false;
-        acc_pending = false;
-        const uint32_t line = sDQS + lrow * C::DQROWB;
-        const uint32_t sw = C::DQROWB == 128 ? (uint32_t)(lrow & 7) : (uint32_t)((lrow >> 1) & 3);
-#pragma unroll
-        for (int j = 0; j < (int)(C::DQROWB / 16); ++j)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(line + ((j ^ sw) << 4)),
-                       "r"(v[4 * j]), "r"(v[4 * j + 1]), "r"(v[4 * j + 2]), "r"(v[4 * j + 3])
-                       : "memory");
-        fence_proxy_async_smem();
-        if (!group_sync()) return false;
-        if (lrow == 0) {
-          tma_reduce_add_3d(&tmDQ, sDQS, grp * (DH / 2), it.head, t0 + 128 * ii);
-          bulk_commit_group();
-        }
-        return true;
-      };
-      // LSE (natural log) and D of the next tile's rows: raw loads, consumed
-      // only when they are written to shared memory, so they stay in flight
-      // while the warp waits for and processes the current tile
-      float nl[2] = {0.f, 0.f}, nd[2] = {0.f, 0.f};
-      auto load_stats = [&](int ii) {
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int rg = 128 * ii + 64 * grp + 32 * u + lane;
-          nl[u] = 0.f;
-          nd[u] = 0.f;
-          if (rg < n) {
-            const int64_t at = (int64_t)it.head * a.T + t0 + rg;
-            nl[u] = __ldg(a.lse + at);
-            nd[u] = __ldg(a.dsum + at);
-          }
-        }
-      };
-      if constexpr (SOFTMAX) load_stats(0);
       for (int i = 0; i < nq; ++i, ++qs) {
         const int rbase = 128 * i + 64 * grp;          // first sample row of this group's half
         const uint32_t dsb = sDS + (qs & 1u) * C::DSB + grp * 16384;
-        if constexpr (SOFTMAX) {
-          __syncwarp();
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            wst[32 * u + lane] = nl[u] * 1.4426950408889634f;   // log2 units
-            wst[64 + 32 * u + lane] = nd[u];
-          }
-          __syncwarp();
-          if (i + 1 < nq) load_stats(i + 1);
-        }
+        const float* st_l = stats + (qs & 1u) * 256 + 64 * grp;
+        const float* st_d = st_l + 128;
         bool w = mbar_wait(bar(C::B_SFULL + grp), qs & 1u, abort_flag, kTimeoutNs);
+        if constexpr (SOFTMAX)
+          w = w && mbar_wait(bar(C::B_STATFULL + (int)(qs & 1u)), (qs >> 1) & 1u, abort_flag,
+                             kTimeoutNs);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (acc_pending && (qs & 1u) == acc_par) {       // dS^T half below was a store's source
-          if (lrow == 0) bulk_wait_group_read0();
-          if (!group_sync()) {
-            ok = false;
-            break;
-          }
-          acc_pending = false;
-        }
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           uint32_t s[32], dp[32];
@@ -936,8 +947,8 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
               const float g = __uint_as_float(dp[c + e]);
               float p, ds;
               if constexpr (SOFTMAX) {
-                p = ex2_approx(fmaf(x, c2, -wst[r]));
-                ds = p * (g - wst[64 + r]);
+                p = ex2_approx(fmaf(x, c2, -st_l[r]));
+                ds = p * (g - st_d[r]);
               } else if constexpr (PHI == GDPA_PHI_SILU) {
                 const float hx = x * half_sc;
                 const float th = tanh_approx(hx);
@@ -971,69 +982,148 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar(C::B_PFULL + grp));
-        if (i > 0 && !drain_dq(i - 1, qs - 1)) {
+        if constexpr (SOFTMAX) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(C::B_STATEMPTY + (int)(qs & 1u)));
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------- drain group
+    setmaxnreg_dec<104>();
+    const int quad = warp & 3;
+    const int lrow = quad * 32 + lane;                 // TMEM lane: query row (dQ) or key (dV, dK)
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const float sc = a.scale;
+    uint32_t qs = 0, ic = 0, sync_phase = 0;
+    bool ok = true;
+    auto group_sync = [&]() -> bool {                 // the 128 threads of this group
+      mbar_arrive(bar(C::B_DSYNC));
+      const bool w = mbar_wait(bar(C::B_DSYNC), sync_phase, abort_flag, kTimeoutNs);
+      sync_phase ^= 1u;
+      return __all_sync(0xffffffffu, w);
+    };
+    // one row of 2*DH bytes from 16-column TMEM loads, packed as fp32 (dQ) or
+    // as bf16 times `mul` (dV, dK), into 16-byte chunks of a staging box
+    auto stage_f32 = [&](uint32_t src, uint32_t box) {
+#pragma unroll
+      for (int c = 0; c < DH / 2; c += 16) {
+        uint32_t v[16];
+        tmem_ld_x16(src + c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                       ::"r"(stage_chunk<DH>(box, lrow, c / 4 + j)), "r"(v[4 * j]),
+                       "r"(v[4 * j + 1]), "r"(v[4 * j + 2]), "r"(v[4 * j + 3])
+                       : "memory");
+      }
+    };
+    auto stage_bf16 = [&](uint32_t src, uint32_t box, float mul) {
+#pragma unroll
+      for (int c = 0; c < DH; c += 16) {
+        uint32_t v[16];
+        tmem_ld_x16(src + c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            pk[u] = pack_bf16x2(__uint_as_float(v[8 * j + 2 * u]) * mul,
+                                __uint_as_float(v[8 * j + 2 * u + 1]) * mul);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                       ::"r"(stage_chunk<DH>(box, lrow, c / 8 + j)), "r"(pk[0]), "r"(pk[1]),
+                       "r"(pk[2]), "r"(pk[3])
+                       : "memory");
+        }
+      }
+    };
+    for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
+      const Tile it = a.tiles[t];
+      const int n = it.rows;
+      if (n == 0) {                                    // no tokens: dK = dV = 0
+        const int key = it.row0 + lrow;
+        if (key < a.m) {
+          const int64_t row = (((int64_t)it.b * a.h + it.head) * a.m + key) * DH;
+          uint4* v4 = reinterpret_cast<uint4*>(a.dv + row);
+          uint4* k4 = reinterpret_cast<uint4*>(a.dk + row);
+#pragma unroll
+          for (int c = 0; c < DH / 8; ++c) {
+            v4[c] = make_uint4(0u, 0u, 0u, 0u);
+            k4[c] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        continue;
+      }
+      const int nq = (n + 127) >> 7;
+      const int t0 = a.offsets[it.b];
+      for (int i = 0; i < nq; ++i, ++qs) {
+        const uint32_t b = qs & 1u;
+        // dQ of tile qs.  Its dS^T buffer b is free: the tile's products are
+        // complete, and the bulk copies that last read it (tile qs-2) finished
+        // before STGFREE let the MMA thread start this tile.
+        bool w = mbar_wait(bar(C::B_DQFULL + (int)b), (qs >> 1) & 1u, abort_flag, kTimeoutNs);
+        if (!__all_sync(0xffffffffu, w)) {
           ok = false;
           break;
         }
-      }
-      if (ok && !drain_dq(nq - 1, qs - 1)) ok = false;
-      if (!ok) break;
-      // ---------------------------------------------------------- dV / dK of this key block
-      bool w = mbar_wait(bar(C::B_ACCFULL), ic & 1u, abort_flag, kTimeoutNs);
-      if (!__all_sync(0xffffffffu, w)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      {
-        // Group 0 writes dV, group 1 dK (times the scale): the rows go as bf16
-        // into this group's half of the last tile's dS^T buffer (its readers
-        // are all in the completed products), swizzled like the output's
-        // tensor map, and leave in one bulk tensor store; keys past m are
-        // clipped by the map.
-        const uint32_t src = tmem + lane_off + (grp == 0 ? C::COL_DV : C::COL_DK);
-        const float mul = grp == 0 ? 1.f : sc;
-        const uint32_t par = (qs - 1) & 1u;
-        const uint32_t stg = sDS + par * C::DSB + grp * 16384;
-        const uint32_t line = stg + lrow * (DH * 2);
-        const uint32_t sw = DH == 64 ? (uint32_t)(lrow & 7) : (uint32_t)((lrow >> 1) & 3);
-#pragma unroll
-        for (int c = 0; c < DH; c += 32) {
-          uint32_t v[32];
-          tmem_ld_x32(src + c, v);
-          tmem_wait_ld();
-          if (c + 32 == DH) {
-            tc_fence_before();
-            mbar_arrive(bar(C::B_ACCEMPTY));            // the accumulators are free
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              pk[u] = pack_bf16x2(__uint_as_float(v[8 * j + 2 * u]) * mul,
-                                  __uint_as_float(v[8 * j + 2 * u + 1]) * mul);
-            const uint32_t chunk = (uint32_t)(c / 8 + j);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(line + ((chunk ^ sw) << 4)),
-                         "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
-                         : "memory");
-          }
-        }
+        tc_fence_after();
+        const uint32_t stg = sDS + b * C::DSB;
+        const uint32_t src = tmem + lane_off + C::COL_DQ + b * DH;
+        stage_f32(src, stg);                           // columns [0, DH/2)
+        stage_f32(src + DH / 2, stg + 16384);          // columns [DH/2, DH)
+        tc_fence_before();
+        mbar_arrive(bar(C::B_DQEMPTY + (int)b));
         fence_proxy_async_smem();
         if (!group_sync()) {
           ok = false;
           break;
         }
         if (lrow == 0) {
-          tma_store_4d(grp == 0 ? &tmDV : &tmDK, stg, 0, it.row0, it.head, it.b);
+          // rows past the sample are exact zeros (their dS entries are zero);
+          // rows past T are clipped by the map
+          tma_reduce_add_3d(&tmDQ, stg, 0, it.head, t0 + 128 * i);
+          tma_reduce_add_3d(&tmDQ, stg + 16384, DH / 2, it.head, t0 + 128 * i);
           bulk_commit_group();
         }
-        acc_pending = true;
-        acc_par = par;
+        if (i + 1 == nq) {
+          // dV and s*dK of this key block, through the same buffer once the
+          // reduces have read it
+          w = mbar_wait(bar(C::B_ACCFULL), ic & 1u, abort_flag, kTimeoutNs);
+          if (!__all_sync(0xffffffffu, w)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lrow == 0) bulk_wait_group_read0();
+          if (!group_sync()) {
+            ok = false;
+            break;
+          }
+          stage_bf16(tmem + lane_off + C::COL_DV, stg, 1.f);
+          stage_bf16(tmem + lane_off + C::COL_DK, stg + 16384, sc);
+          tc_fence_before();
+          mbar_arrive(bar(C::B_ACCEMPTY));
+          fence_proxy_async_smem();
+          if (!group_sync()) {
+            ok = false;
+            break;
+          }
+          if (lrow == 0) {
+            tma_store_4d(&tmDV, stg, 0, it.row0, it.head, it.b);
+            tma_store_4d(&tmDK, stg + 16384, 0, it.row0, it.head, it.b);
+            bulk_commit_group();
+          }
+          ++ic;
+        }
+        if (lrow == 0) {                               // the staging area may be rewritten
+          bulk_wait_group_read0();
+          mbar_arrive(bar(C::B_STGFREE + (int)b));
+        }
       }
-      ++ic;
     }
-    if (lrow == 0) bulk_wait_group0();               // reduces done before the CTA exits
+    if (lrow == 0) bulk_wait_group0();                // copies done before the CTA exits
   }
 
   // ------------------------------------------------------------ teardown
@@ -1057,7 +1147,6 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
   tc_fence_after();
   if (warp == 2) tmem_dealloc(tmem, 512);
 }
-
 
 // ------------------------------------------------------------------ host side
 
@@ -1145,7 +1234,7 @@ cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* 
     e = cudaFuncSetAttribute(hk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H::SMEM);
     if (e != cudaSuccess) return e;
     KernelScope ks_("gdpa_bwd_sm100", st);
-    hk<<<device_sm_count(), kThreads, H::SMEM, st>>>(mq, mg, mk, mv, mdq, mdv, mdk, args);
+    hk<<<device_sm_count(), kHalfThreads, H::SMEM, st>>>(mq, mg, mk, mv, mdq, mdv, mdk, args);
     return cudaGetLastError();
   }
   KernelScope ks_("gdpa_bwd_sm100", st);
