@@ -35,6 +35,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOAD = 5
+E2E_CHUNKS = 8                          # sample groups of the end-to-end step
 FLOPS_FWD, FLOPS_BWD = 4, 8            # x T*h*m*dh
 # algorithmic FLOPs credited to each kernel, in units of T*h*m*dh
 KERNEL_FLOPS = {"gdpa_fwd_sm100": 4, "gdpa_bwd_sm100": 8, "gdpa_simt_fwd": 4,
@@ -347,35 +348,92 @@ def main():
                for k_, v_ in per_kernel.items()}
 
     # ---- end to end through host buffers ----
+    # The step again, through the public API, from pinned host memory: the
+    # batch is cut into E2E_CHUNKS equal groups of samples, each its own
+    # fwd + bwd call on views of the device tensors.  One stream copies chunk
+    # inputs in, one computes, one copies chunk outputs back, so the two PCIe
+    # directions and the compute overlap; per-chunk events order every reuse
+    # of a buffer (also from one step to the next).
     e2e = None
     if not args.no_e2e and args.e2e_steps > 0:
         hq, hk, hv, hg = (x.cpu().pin_memory() for x in (q, k, v, g))
         ho, hdq, hdk, hdv = (torch.empty(x.shape, dtype=x.dtype).pin_memory()
                              for x in (o, dq, dk, dv))
-        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg)) + off.numel() * 4
+        offs = [int(x) for x in d["offsets"]]
+        nb = len(offs) - 1
+        bounds = [nb * c // E2E_CHUNKS for c in range(E2E_CHUNKS + 1)]
+        chunks = []
+        for b0, b1 in zip(bounds[:-1], bounds[1:]):
+            if b1 <= b0:
+                continue
+            t0_, t1_ = offs[b0], offs[b1]
+            coff = [x - t0_ for x in offs[b0:b1 + 1]]
+            cp_ = pkg.problem_for(q[t0_:t1_], k[b0:b1], coff, wl.phi_name, wl.scale,
+                                  max_n=max(coff[i + 1] - coff[i] for i in range(b1 - b0)))
+            chunks.append(dict(
+                rows=(t0_, t1_), smp=(b0, b1), p=cp_,
+                hoff=torch.tensor(coff, dtype=torch.int32).pin_memory(),
+                off=torch.empty(len(coff), dtype=torch.int32, device=dev),
+                lse=torch.empty((wl.h, max(t1_ - t0_, 1)), dtype=torch.float32, device=dev),
+                wsf=pkg.workspace(pkg.fwd_workspace_bytes(cp_), dev),
+                wsb=pkg.workspace(pkg.bwd_workspace_bytes(cp_), dev),
+                loaded=torch.cuda.Event(), computed=torch.cuda.Event(), sent=torch.cuda.Event()))
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg)) + \
+            sum(c_["hoff"].numel() * 4 for c_ in chunks)
         d2h = sum(x.numel() * x.element_size() for x in (ho, hdq, hdk, hdv))
-        hoff = off.cpu().pin_memory()
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        first = [True]
 
         def e2e_step():
-            off.copy_(hoff, non_blocking=True)
-            for dst, src in ((q, hq), (k, hk), (v, hv), (g, hg)):
-                dst.copy_(src, non_blocking=True)
-            step()
-            for dst, src in ((ho, o), (hdq, dq), (hdk, dk), (hdv, dv)):
-                dst.copy_(src, non_blocking=True)
+            for c_ in chunks:
+                (t0_, t1_), (b0, b1) = c_["rows"], c_["smp"]
+                with torch.cuda.stream(s_in):
+                    if not first[0]:
+                        s_in.wait_event(c_["computed"])       # last step's compute read them
+                    c_["off"].copy_(c_["hoff"], non_blocking=True)
+                    for dst, src in ((q, hq), (g, hg)):
+                        dst[t0_:t1_].copy_(src[t0_:t1_], non_blocking=True)
+                    for dst, src in ((k, hk), (v, hv)):
+                        dst[b0:b1].copy_(src[b0:b1], non_blocking=True)
+                    c_["loaded"].record(s_in)
+            for c_ in chunks:
+                (t0_, t1_), (b0, b1) = c_["rows"], c_["smp"]
+                stream.wait_event(c_["loaded"])
+                if not first[0]:
+                    stream.wait_event(c_["sent"])             # last step's outputs copied out
+                cq, cg, co, cdq = q[t0_:t1_], g[t0_:t1_], o[t0_:t1_], dq[t0_:t1_]
+                ck, cv, cdk, cdv = k[b0:b1], v[b0:b1], dk[b0:b1], dv[b0:b1]
+                cl = c_["lse"][:, :t1_ - t0_]
+                G.fwd(c_["p"], cq, c_["off"], ck, cv, o=co, lse=cl, ws=c_["wsf"], stream=stream)
+                G.bwd(c_["p"], cq, c_["off"], ck, cv, co, cl, cg, dq=cdq, dk=cdk, dv=cdv,
+                      ws=c_["wsb"], stream=stream)
+                c_["computed"].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(c_["computed"])
+                    for dst, src in ((ho, o), (hdq, dq)):
+                        dst[t0_:t1_].copy_(src[t0_:t1_], non_blocking=True)
+                    for dst, src in ((hdk, dk), (hdv, dv)):
+                        dst[b0:b1].copy_(src[b0:b1], non_blocking=True)
+                    c_["sent"].record(s_out)
+            first[0] = False
 
         e2e_step()
         torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0 = time.perf_counter()
-        e0.record(stream)
+        e0.record(s_in)
         for _ in range(args.e2e_steps):
             e2e_step()
-        e1.record(stream)
+        s_out.wait_stream(stream)
+        s_out.wait_stream(s_in)
+        e1.record(s_out)
         torch.cuda.synchronize()
         wall = time.perf_counter() - t0
         barrier()
+        bad = [pkg.workspace_status(c_["wsf"]) or pkg.workspace_status(c_["wsb"]) for c_ in chunks]
+        if any(bad):
+            raise RuntimeError("device-side status error in the end-to-end steps")
         ea = aggregate(e0.elapsed_time(e1), (FLOPS_FWD + FLOPS_BWD) * unit_flops * args.e2e_steps,
                        0.0, 0.0, world, dist, dev)
         ems = ea["ms_max"]
@@ -383,8 +441,10 @@ def main():
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": args.e2e_steps, "ms_per_step": ems / args.e2e_steps,
                "wall_ms_per_step": 1e3 * wall / args.e2e_steps,
-               "api": "recsys_context_personalised_b200.gdpa fwd/bwd on tensors copied from pinned host memory"}
-        del hq, hk, hv, hg, ho, hdq, hdk, hdv
+               "api": (f"recsys_context_personalised_b200.gdpa fwd/bwd on {len(chunks)} sample "
+                       "chunks copied from and to pinned host memory; copy-in, compute and "
+                       "copy-out on three streams")}
+        del hq, hk, hv, hg, ho, hdq, hdk, hdv, chunks
 
     # ---- CPU oracle baseline (rank 0 at N=1 only) ----
     cpu = None
