@@ -44,12 +44,12 @@ TENSOR_KERNELS = {"gdpa_fwd_sm100", "gdpa_bwd_sm100"}
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per unit T*h*m*dh of
 # the fused kernels, from one ncu capture on the first 64 samples of this
 # workload (T = 20,846; `bench.py --samples 64 --steps 1 --warmup 1`):
-# backward 738,833,920 + 588,749,568 B, forward 580,582,144 + 35,432,960 B.
+# backward 743,162,880 + 589,410,048 B, forward 580,738,816 + 34,836,480 B.
 # A launch's traffic is this times its units; valid only for the kernels as
 # captured (set an entry to None when its kernel changes).
 _CAPTURE_UNITS = 20846 * 16 * 2048 * 64
-TRAFFIC_PER_UNIT = {"gdpa_bwd_sm100": None,   # changed since the capture
-                    "gdpa_fwd_sm100": (580582144 + 35432960) / _CAPTURE_UNITS}
+TRAFFIC_PER_UNIT = {"gdpa_bwd_sm100": (743162880 + 589410048) / _CAPTURE_UNITS,
+                    "gdpa_fwd_sm100": (580738816 + 34836480) / _CAPTURE_UNITS}
 # fp32 FFMA peak for the SIMT kernels: 148 SMs * 128 FMA/clk * 2 flop * 1.965 GHz
 SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
@@ -356,6 +356,7 @@ def main():
     # of a buffer (also from one step to the next).
     e2e = None
     if not args.no_e2e and args.e2e_steps > 0:
+        o_full = o.clone()          # O of the full-batch call (the forward is deterministic)
         hq, hk, hv, hg = (x.cpu().pin_memory() for x in (q, k, v, g))
         ho, hdq, hdk, hdv = (torch.empty(x.shape, dtype=x.dtype).pin_memory()
                              for x in (o, dq, dk, dv))
@@ -434,6 +435,8 @@ def main():
         bad = [pkg.workspace_status(c_["wsf"]) or pkg.workspace_status(c_["wsb"]) for c_ in chunks]
         if any(bad):
             raise RuntimeError("device-side status error in the end-to-end steps")
+        if not torch.equal(ho, o_full.cpu()):
+            raise RuntimeError("end-to-end O differs from the full-batch O")
         ea = aggregate(e0.elapsed_time(e1), (FLOPS_FWD + FLOPS_BWD) * unit_flops * args.e2e_steps,
                        0.0, 0.0, world, dist, dev)
         ems = ea["ms_max"]
@@ -444,7 +447,7 @@ def main():
                "api": (f"recsys_context_personalised_b200.gdpa fwd/bwd on {len(chunks)} sample "
                        "chunks copied from and to pinned host memory; copy-in, compute and "
                        "copy-out on three streams")}
-        del hq, hk, hv, hg, ho, hdq, hdk, hdv, chunks
+        del hq, hk, hv, hg, ho, hdq, hdk, hdv, chunks, o_full
 
     # ---- CPU oracle baseline (rank 0 at N=1 only) ----
     cpu = None
