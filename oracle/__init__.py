@@ -19,7 +19,7 @@ _SRC = os.path.join(_HERE, "gdpa_oracle.c")
 _LIB = os.path.join(_HERE, "libgdpa_oracle.so")
 _lib = None
 
-PHI = {"identity": 0, "silu": 1, "softmax": 2}
+PHI = {"identity": 0, "silu": 1, "softmax": 2, "relu": 3, "gelu": 4}
 
 
 def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:

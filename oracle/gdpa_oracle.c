@@ -16,7 +16,8 @@
  *   K^ = K[b, j], V^ = V[b, j]       (m x dh):
  *
  *   S  = s * Q^ K^T                  (n_b x m)
- *   P  = phi(S)                      phi in {identity, SiLU, row softmax}
+ *   P  = phi(S)                      phi in {identity, SiLU, row softmax,
+ *                                               ReLU, GELU}
  *   O  = P V^                        (n_b x dh)
  *   LSE_i = M_i + ln sum_k exp(S_ik - M_i),  M_i = max_k S_ik  (softmax)
  *
@@ -26,6 +27,9 @@
  *   dS = dP                                   (identity)
  *      = dP * sig(S) (1 + S (1 - sig(S)))     (SiLU, sig = logistic)
  *      = P * (dP - D),  D_i = sum_k P_ik dP_ik (softmax)
+ *      = dP * [S > 0]                          (ReLU)
+ *      = dP * (Phi(S) + S pdf(S))              (GELU = S Phi(S), Phi the standard
+ *                                               normal CDF, pdf its density)
  *   dQ^ = s dS K^,  dK^ = s dS^T Q^.
  *
  * Every dot product is a plain loop accumulated in double.  Inputs are float
@@ -34,7 +38,10 @@
  * blocked, fused or reordered.
  *
  * Layouts: q, o, dout, dq: [T, h, dh];  k, v, dk, dv: [B, h, m, dh];
- * offsets: int64 [B+1];  lse: [h, T].  phi: 0 identity, 1 SiLU, 2 softmax.
+ * offsets: int64 [B+1];  lse: [h, T].  phi: 0 identity, 1 SiLU, 2 softmax,
+ * 3 ReLU, 4 GELU.  ReLU and GELU are the "other phi" of the PFFN variants the
+ * Kunlun pages leave open; GELU is taken in its exact form x Phi(x) (reading:
+ * the pages name no approximation).
  */
 #include <math.h>
 #include <stdint.h>
@@ -47,6 +54,12 @@
 #define PHI_IDENTITY 0
 #define PHI_SILU 1
 #define PHI_SOFTMAX 2
+#define PHI_RELU 3
+#define PHI_GELU 4
+
+/* Standard normal CDF and density (for GELU): Phi(x) = (1 + erf(x / sqrt 2)) / 2. */
+static double normal_cdf(double x) { return 0.5 * (1.0 + erf(x * 0.70710678118654752440)); }
+static double normal_pdf(double x) { return 0.39894228040143267794 * exp(-0.5 * x * x); }
 
 static double logistic(double x) { return 1.0 / (1.0 + exp(-x)); }
 
@@ -73,6 +86,10 @@ static void activation(int n, int m, int phi, const double* S, double* P, double
       for (int k = 0; k < m; ++k) pi[k] = si[k];
     } else if (phi == PHI_SILU) {
       for (int k = 0; k < m; ++k) pi[k] = si[k] / (1.0 + exp(-si[k]));
+    } else if (phi == PHI_RELU) {
+      for (int k = 0; k < m; ++k) pi[k] = si[k] > 0.0 ? si[k] : 0.0;
+    } else if (phi == PHI_GELU) {
+      for (int k = 0; k < m; ++k) pi[k] = si[k] * normal_cdf(si[k]);
     } else {
       double mx = -INFINITY;
       for (int k = 0; k < m; ++k) mx = si[k] > mx ? si[k] : mx;
@@ -97,7 +114,7 @@ static int valid_args(int B, int h, int dh, int m, const int64_t* offsets) {
 int gdpa_oracle_fwd(int B, int h, int dh, int m, const int64_t* offsets,
                     const float* q, const float* k, const float* v, int phi,
                     double scale, double* o, double* lse, int nthreads) {
-  if (!valid_args(B, h, dh, m, offsets) || phi < 0 || phi > 2 || !q || !k || !v || !o)
+  if (!valid_args(B, h, dh, m, offsets) || phi < 0 || phi > 4 || !q || !k || !v || !o)
     return -1;
   const int64_t T = offsets[B];
   int failed = 0;
@@ -143,7 +160,7 @@ int gdpa_oracle_bwd(int B, int h, int dh, int m, const int64_t* offsets,
                     const float* q, const float* k, const float* v, const float* dout,
                     int phi, double scale, double* dq, double* dk, double* dv,
                     int nthreads) {
-  if (!valid_args(B, h, dh, m, offsets) || phi < 0 || phi > 2 || !q || !k || !v ||
+  if (!valid_args(B, h, dh, m, offsets) || phi < 0 || phi > 4 || !q || !k || !v ||
       !dout || !dq || !dk || !dv)
     return -1;
   int failed = 0;
@@ -199,6 +216,11 @@ int gdpa_oracle_bwd(int B, int h, int dh, int m, const int64_t* offsets,
           const double sg = logistic(si[kk]);
           dpi[kk] = dpi[kk] * sg * (1.0 + si[kk] * (1.0 - sg));
         }
+      } else if (phi == PHI_RELU) {
+        for (int kk = 0; kk < m; ++kk) dpi[kk] = si[kk] > 0.0 ? dpi[kk] : 0.0;
+      } else if (phi == PHI_GELU) {
+        for (int kk = 0; kk < m; ++kk)
+          dpi[kk] = dpi[kk] * (normal_cdf(si[kk]) + si[kk] * normal_pdf(si[kk]));
       } else if (phi == PHI_SOFTMAX) {
         double D = 0.0;
         for (int kk = 0; kk < m; ++kk) D += pi[kk] * dpi[kk];

@@ -35,6 +35,12 @@ MUTANTS = {
                       "acc += dP[(size_t)i * m + kk] * (double)qb[(size_t)i * dh + d];"),
     "dv_uses_logits": ("for (int i = 0; i < n; ++i) acc += P[(size_t)i * m + kk] * (double)gb[(size_t)i * h * dh + d];",
                        "for (int i = 0; i < n; ++i) acc += S[(size_t)i * m + kk] * (double)gb[(size_t)i * h * dh + d];"),
+    "relu_negative_half": ("pi[k] = si[k] > 0.0 ? si[k] : 0.0;", "pi[k] = si[k] > 0.0 ? si[k] : 0.01 * si[k];"),
+    "relu_grad_always": ("dpi[kk] = si[kk] > 0.0 ? dpi[kk] : 0.0;", "dpi[kk] = dpi[kk];"),
+    "gelu_cdf_scale": ("return 0.5 * (1.0 + erf(x * 0.70710678118654752440));",
+                       "return 0.5 * (1.0 + erf(x));"),
+    "gelu_grad_no_pdf": ("dpi[kk] = dpi[kk] * (normal_cdf(si[kk]) + si[kk] * normal_pdf(si[kk]));",
+                         "dpi[kk] = dpi[kk] * normal_cdf(si[kk]);"),
     "dp_uses_q": ("acc += (double)gb[(size_t)i * h * dh + d] * (double)vb[(size_t)kk * dh + d];",
                   "acc += (double)gb[(size_t)i * h * dh + d] * (double)kb[(size_t)kk * dh + d];"),
 }
@@ -47,6 +53,9 @@ PIN_CALLS = (
        (pins.test_silu_closed_forms, ()), (pins.test_identity_backward_closed_forms, ()),
        (pins.test_softmax_backward_invariants, ())]
     + [(pins.test_backward_matches_torch_autograd, (phi,)) for phi in pins.PHIS]
+    + [(pins.test_relu_gelu_closed_forms, ())]
+    + [(pins.test_matches_library_routines, (phi,)) for phi in ("relu", "gelu")]
+    + [(pins.test_backward_matches_torch_autograd, (phi,)) for phi in ("relu", "gelu")]
 )
 
 

@@ -23,6 +23,10 @@ from synthetic import random_problem
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 PHIS = ["identity", "silu", "softmax"]
+# the PFFN variants' other activations (ReLU, and GELU in its exact form x Phi(x))
+PHIS_ALL = PHIS + ["relu", "gelu"]
+_LIB_PHI = {"identity": lambda x: x, "silu": F.silu, "softmax": lambda x: torch.softmax(x, dim=-1),
+            "relu": F.relu, "gelu": lambda x: F.gelu(x, approximate="none")}
 
 
 def _f64(x):
@@ -46,8 +50,7 @@ def _lib_forward(q, k, v, off, phi, s):
         for j in range(h):
             qh = _f64(q[t0:t1, j])
             S = s * (qh @ _f64(k[b, j]).T)
-            P = {"identity": lambda x: x, "silu": F.silu,
-                 "softmax": lambda x: torch.softmax(x, dim=-1)}[phi](S)
+            P = _LIB_PHI[phi](S)
             out[t0:t1, j] = P @ _f64(v[b, j])
     return out.numpy()
 
@@ -99,7 +102,7 @@ def test_identity_equals_other_association():
             np.testing.assert_allclose(o[t0:t1, j], s * (Q @ (K.T @ V)), rtol=1e-12, atol=1e-12)
 
 
-@pytest.mark.parametrize("phi", PHIS)
+@pytest.mark.parametrize("phi", PHIS_ALL)
 def test_matches_library_routines(phi):
     p = _problem(2, B=4, h=3, dh=16, m=11, n=(1, 9, 0, 13))
     s = 0.3 if phi != "softmax" else 0.25
@@ -177,6 +180,35 @@ def test_silu_closed_forms():
     assert np.abs(o).max() == 0.0
 
 
+def test_relu_gelu_closed_forms():
+    # one token, three keys with logits S = [1, -1, 1/2] (s = 1, q = e1, k_k = S_k e1),
+    # values v = [e1, e2, e1 + e2]:  O = sum_k phi(S_k) v_k
+    q = np.array([[[1.0, 0.0]]], np.float32)
+    k = np.array([[[[1.0, 0.0], [-1.0, 0.0], [0.5, 0.0]]]], np.float32)
+    v = np.array([[[[1.0, 0.0], [0.0, 1.0], [1.0, 1.0]]]], np.float32)
+    off = np.array([0, 1], np.int64)
+    o, _ = oracle.fwd(q, k, v, off, "relu", 1.0)
+    np.testing.assert_allclose(o[0, 0], [1.5, 0.5], rtol=0, atol=1e-15)
+    # standard normal CDF from printed tables: Phi(1), Phi(-1), Phi(1/2)
+    c1, cm1, ch = 0.8413447460685429, 0.15865525393145707, 0.6914624612740131
+    g1, gm1, gh = c1, -cm1, 0.5 * ch
+    o, _ = oracle.fwd(q, k, v, off, "gelu", 1.0)
+    np.testing.assert_allclose(o[0, 0], [g1 + gh, gm1 + gh], rtol=1e-14)
+    # derivatives: ReLU' = [S > 0]; GELU'(x) = Phi(x) + x pdf(x), pdf(1) = pdf(-1) =
+    # 0.24197072451914337, pdf(1/2) = 0.3520653267642995 (tables); with dO = e1,
+    # dP_k = v_k . e1 = [1, 0, 1] and dV_k = phi(S_k) e1
+    dout = np.array([[[1.0, 0.0]]], np.float32)
+    dq, dk, dv = oracle.bwd(q, k, v, dout, off, "relu", 1.0)
+    np.testing.assert_allclose(dq[0, 0], [1.0 * 1 * 1.0 + 1.0 * 0.5, 0.0], atol=1e-15)
+    np.testing.assert_allclose(dv[0, 0, :, 0], [1.0, 0.0, 0.5], atol=1e-15)
+    d1, dh_ = c1 + 0.24197072451914337, ch + 0.5 * 0.3520653267642995
+    dq, dk, dv = oracle.bwd(q, k, v, dout, off, "gelu", 1.0)
+    # dQ = sum_k dS_k k_k with dS = dP * GELU'(S); dK_k = dS_k q
+    np.testing.assert_allclose(dq[0, 0, 0], d1 * 1.0 + dh_ * 0.5, rtol=1e-14)
+    np.testing.assert_allclose(dk[0, 0, :, 0], [d1, 0.0, dh_], rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(dv[0, 0, :, 0], [g1, gm1, gh], rtol=1e-14)
+
+
 def test_identity_backward_closed_forms():
     p = _problem(6, dh=5, m=7, n=(6, 2, 3))
     s = 1.3
@@ -209,7 +241,7 @@ def test_softmax_backward_invariants():
 # invariances
 
 
-@pytest.mark.parametrize("phi", PHIS)
+@pytest.mark.parametrize("phi", PHIS_ALL)
 def test_key_permutation_invariance(phi):
     p = _problem(8, B=2, h=2, dh=4, m=10, n=(6, 3))
     perm = torch.from_numpy(np.random.default_rng(0).permutation(10))
@@ -224,7 +256,7 @@ def test_key_permutation_invariance(phi):
     np.testing.assert_allclose(g1[2][:, :, perm.numpy()], g2[2], rtol=1e-12, atol=1e-13)
 
 
-@pytest.mark.parametrize("phi", PHIS)
+@pytest.mark.parametrize("phi", PHIS_ALL)
 def test_token_equivariance_and_independence(phi):
     p = _problem(9, B=3, h=2, dh=4, m=6, n=(5, 2, 4))
     off = p["offsets"]
@@ -271,7 +303,7 @@ def test_bad_arguments_rejected():
 # gradients: finite differences (brute force over every input element)
 
 
-@pytest.mark.parametrize("phi", PHIS)
+@pytest.mark.parametrize("phi", PHIS_ALL)
 def test_backward_matches_central_differences(phi):
     p = random_problem(12, 2, 2, 3, 4, (3, 2), dtype=torch.float32)
     q, k, v, g = (p[x].double().numpy() for x in ("q", "k", "v", "dout"))
@@ -305,7 +337,7 @@ def test_backward_matches_central_differences(phi):
         assert _rel(grad, fd) < 2e-5, (name, _rel(grad, fd))
 
 
-@pytest.mark.parametrize("phi", PHIS)
+@pytest.mark.parametrize("phi", PHIS_ALL)
 def test_backward_matches_torch_autograd(phi):
     p = random_problem(13, 3, 2, 8, 6, (4, 0, 5), dtype=torch.float32)
     off = p["offsets"]
@@ -320,8 +352,7 @@ def test_backward_matches_torch_autograd(phi):
             if t1 == t0:
                 continue
             S = s * (q[t0:t1, j] @ k[b, j].T)
-            P = {"identity": lambda x: x, "silu": F.silu,
-                 "softmax": lambda x: torch.softmax(x, -1)}[phi](S)
+            P = _LIB_PHI[phi](S)
             outs.append(((t0, t1, j), P @ v[b, j]))
     L = sum((o * g[t0:t1, j]).sum() for (t0, t1, j), o in outs)
     L.backward()
