@@ -21,6 +21,7 @@ same workload (rank 0 only), in the same units.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import json
 import math
@@ -66,7 +67,20 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--samples", type=int, default=0,
                     help="run only the first N samples of the workload (small profiling case)")
+    ap.add_argument("--phi", default=None,
+                    choices=["identity", "silu", "softmax", "relu", "gelu"],
+                    help="the same workload with another activation (the PFFN variants' phi)")
     return ap.parse_args()
+
+
+def workload(args):
+    """The benchmarked workload, with its activation replaced when --phi is given."""
+    import synthetic as syn
+    wl = syn.WORKLOADS[WORKLOAD]
+    if args.phi and args.phi != wl.phi_name:
+        code = {v_: k_ for k_, v_ in syn.PHI_NAMES.items()}[args.phi]
+        wl = dataclasses.replace(wl, phi=code, name=wl.name.replace(wl.phi_name, args.phi))
+    return wl
 
 
 def peaks():
@@ -215,7 +229,7 @@ def run_reference(args, rank):
     if rank != 0:
         return
     import synthetic as syn
-    wl = syn.WORKLOADS[WORKLOAD]
+    wl = workload(args)
     lengths = syn.lengths(wl)
     total = args.steps + args.warmup
     per_step = max(1.0, min(8.0, 150.0 / max(total, 1)))
@@ -272,7 +286,7 @@ def main():
         if world > 1:
             dist.barrier()
 
-    wl = syn.WORKLOADS[WORKLOAD]
+    wl = workload(args)
     subset = list(range(args.samples)) if 0 < args.samples < wl.B else None
     d = syn.make_inputs(WORKLOAD, device=dev, seed=rank, backward=True, samples=subset)
     q, k, v, g = d["q"], d["k"], d["v"], d["dout"]
@@ -338,7 +352,7 @@ def main():
     else:
         roof = {"bound": "alu", "peak": SIMT_PEAK_TFLOPS,
                 "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz"}
-    tpu = TRAFFIC_PER_UNIT.get(name) if WORKLOAD == 5 else None
+    tpu = TRAFFIC_PER_UNIT.get(name) if WORKLOAD == 5 and wl.phi_name == "softmax" else None
     roof.update(kernel=name, achieved=achieved, unit="TFLOP/s", frac=achieved / roof["peak"],
                 traffic=tpu * unit_flops if tpu else None,
                 traffic_source=("ncu DRAM bytes of a 64-sample capture, scaled by T*h*m*dh"

@@ -59,10 +59,15 @@
 extern "C" {
 #endif
 
+/* phi applied to the scaled logits x = s * q.k: identity, SiLU x*logistic(x),
+ * row softmax, and the PFFN variants' other activations ReLU max(x, 0) and
+ * GELU in its exact form x * Phi(x) (Phi the standard normal CDF). */
 typedef enum {
   GDPA_PHI_IDENTITY = 0,
   GDPA_PHI_SILU = 1,
-  GDPA_PHI_SOFTMAX = 2
+  GDPA_PHI_SOFTMAX = 2,
+  GDPA_PHI_RELU = 3,
+  GDPA_PHI_GELU = 4
 } gdpa_phi_t;
 
 typedef enum {

@@ -72,7 +72,7 @@ gdpa_status_t check_problem(const gdpa_problem_t* p) {
       p->total_tokens >= (int64_t)1 << 31)
     return GDPA_ERR_INVALID_ARG;
   if ((int64_t)p->max_n * p->B < p->total_tokens) return GDPA_ERR_INVALID_ARG;
-  if (p->phi < GDPA_PHI_IDENTITY || p->phi > GDPA_PHI_SOFTMAX) return GDPA_ERR_INVALID_ARG;
+  if (p->phi < GDPA_PHI_IDENTITY || p->phi > GDPA_PHI_GELU) return GDPA_ERR_INVALID_ARG;
   if (p->dtype != GDPA_DTYPE_F32 && p->dtype != GDPA_DTYPE_BF16) return GDPA_ERR_INVALID_ARG;
   if (!(p->scale == p->scale) || p->scale > 3.0e38f || p->scale < -3.0e38f)
     return GDPA_ERR_INVALID_ARG;

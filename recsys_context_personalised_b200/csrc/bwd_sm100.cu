@@ -458,6 +458,14 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 const float sg = fmaf(0.5f, th, 0.5f);          // logistic(x s)
                 p = fmaf(hx, th, hx);                             // x s * logistic(x s)
                 ds = g * sg * fmaf(x * sc, 1.f - sg, 1.f);
+              } else if constexpr (PHI == GDPA_PHI_RELU) {
+                const float u = x * sc;
+                p = relu_f(u);
+                ds = g * relu_grad(u);
+              } else if constexpr (PHI == GDPA_PHI_GELU) {
+                const float u = x * sc;
+                p = gelu_f(u);
+                ds = g * gelu_grad(u);
               } else {
                 p = x * sc;
                 ds = g;
@@ -955,6 +963,14 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                 const float sg = fmaf(0.5f, th, 0.5f);          // logistic(x s)
                 p = fmaf(hx, th, hx);                             // x s * logistic(x s)
                 ds = g * sg * fmaf(x * sc, 1.f - sg, 1.f);
+              } else if constexpr (PHI == GDPA_PHI_RELU) {
+                const float u = x * sc;
+                p = relu_f(u);
+                ds = g * relu_grad(u);
+              } else if constexpr (PHI == GDPA_PHI_GELU) {
+                const float u = x * sc;
+                p = gelu_f(u);
+                ds = g * gelu_grad(u);
               } else {
                 p = x * sc;
                 ds = g;
@@ -1252,6 +1268,10 @@ cudaError_t launch_bwd_dh(const gdpa_problem_t& p, const void* q, const int32_t*
       return launch_bwd_t<DH, GDPA_PHI_SOFTMAX>(p, q, offsets, k, v, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st);
     case GDPA_PHI_SILU:
       return launch_bwd_t<DH, GDPA_PHI_SILU>(p, q, offsets, k, v, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st);
+    case GDPA_PHI_RELU:
+      return launch_bwd_t<DH, GDPA_PHI_RELU>(p, q, offsets, k, v, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st);
+    case GDPA_PHI_GELU:
+      return launch_bwd_t<DH, GDPA_PHI_GELU>(p, q, offsets, k, v, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st);
     default:
       return launch_bwd_t<DH, GDPA_PHI_IDENTITY>(p, q, offsets, k, v, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st);
   }

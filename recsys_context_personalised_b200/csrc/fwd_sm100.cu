@@ -486,6 +486,12 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
               if constexpr (PHI == GDPA_PHI_SILU) {
                 p0 = silu_tanh(x0, half_scale);
                 p1 = silu_tanh(x1, half_scale);
+              } else if constexpr (PHI == GDPA_PHI_RELU) {
+                p0 = relu_f(x0 * a.scale);
+                p1 = relu_f(x1 * a.scale);
+              } else if constexpr (PHI == GDPA_PHI_GELU) {
+                p0 = gelu_f(x0 * a.scale);
+                p1 = gelu_f(x1 * a.scale);
               } else {
                 p0 = x0 * a.scale;
                 p1 = x1 * a.scale;
@@ -652,6 +658,8 @@ cudaError_t launch_fwd_dh(const gdpa_problem_t& p, const void* q, const void* k,
   switch (p.phi) {
     case GDPA_PHI_SOFTMAX: return launch_fwd_t<DH, GDPA_PHI_SOFTMAX>(p, q, k, v, o, lse, ws, tiles, st);
     case GDPA_PHI_SILU: return launch_fwd_t<DH, GDPA_PHI_SILU>(p, q, k, v, o, lse, ws, tiles, st);
+    case GDPA_PHI_RELU: return launch_fwd_t<DH, GDPA_PHI_RELU>(p, q, k, v, o, lse, ws, tiles, st);
+    case GDPA_PHI_GELU: return launch_fwd_t<DH, GDPA_PHI_GELU>(p, q, k, v, o, lse, ws, tiles, st);
     default: return launch_fwd_t<DH, GDPA_PHI_IDENTITY>(p, q, k, v, o, lse, ws, tiles, st);
   }
 }

@@ -85,4 +85,33 @@ struct KernelScope {
   cudaStream_t st;
 };
 
+// Elementwise phi of the PFFN variants on a scaled logit x, and dphi/dx:
+// ReLU max(x, 0); GELU in its exact form x * Phi(x), Phi(x) = (1 + erf(x/sqrt 2))/2,
+// with derivative Phi(x) + x * exp(-x^2/2) / sqrt(2 pi).
+__device__ __forceinline__ float relu_f(float x) { return fmaxf(x, 0.f); }
+__device__ __forceinline__ float relu_grad(float x) { return x > 0.f ? 1.f : 0.f; }
+// Phi(x) and exp(-x^2/2), with erf from Abramowitz & Stegun, Handbook of
+// Mathematical Functions, formula 7.1.26 (|error| <= 1.5e-7): for z >= 0,
+// erf(z) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2), t = 1 / (1 + p z).
+__device__ __forceinline__ void normal_cdf_gauss(float x, float& cdf, float& gauss) {
+  const float z = fabsf(x) * 0.7071067811865476f;
+  const float t = __fdividef(1.f, fmaf(0.3275911f, z, 1.f));
+  const float poly =
+      t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, 1.061405429f, -1.453152027f), 1.421413741f),
+                       -0.284496736f),
+               0.254829592f);
+  gauss = __expf(-z * z);
+  cdf = 0.5f + copysignf(0.5f * (1.f - poly * gauss), x);
+}
+__device__ __forceinline__ float gelu_f(float x) {
+  float cdf, gauss;
+  normal_cdf_gauss(x, cdf, gauss);
+  return x * cdf;
+}
+__device__ __forceinline__ float gelu_grad(float x) {
+  float cdf, gauss;
+  normal_cdf_gauss(x, cdf, gauss);
+  return fmaf(x * 0.3989422804014327f, gauss, cdf);
+}
+
 }  // namespace gdpa

@@ -102,6 +102,12 @@ simt_fwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     } else if (phi == GDPA_PHI_SILU) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) s[i] = silu_f(s[i]);
+    } else if (phi == GDPA_PHI_RELU) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s[i] = relu_f(s[i]);
+    } else if (phi == GDPA_PHI_GELU) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s[i] = gelu_f(s[i]);
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) Ps[r * PL + c * 8 + i] = s[i];
@@ -157,6 +163,14 @@ __device__ __forceinline__ float dlogit(int phi, float s, float dp, float lse_r,
   if (phi == GDPA_PHI_SILU) {
     *p_out = silu_f(s);
     return dp * silu_grad(s);
+  }
+  if (phi == GDPA_PHI_RELU) {
+    *p_out = relu_f(s);
+    return dp * relu_grad(s);
+  }
+  if (phi == GDPA_PHI_GELU) {
+    *p_out = gelu_f(s);
+    return dp * gelu_grad(s);
   }
   *p_out = s;
   return dp;

@@ -16,8 +16,9 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdpa.so")
 
-PHI_IDENTITY, PHI_SILU, PHI_SOFTMAX = 0, 1, 2
-PHI = {"identity": PHI_IDENTITY, "silu": PHI_SILU, "softmax": PHI_SOFTMAX}
+PHI_IDENTITY, PHI_SILU, PHI_SOFTMAX, PHI_RELU, PHI_GELU = 0, 1, 2, 3, 4
+PHI = {"identity": PHI_IDENTITY, "silu": PHI_SILU, "softmax": PHI_SOFTMAX, "relu": PHI_RELU,
+       "gelu": PHI_GELU}
 DTYPE_F32, DTYPE_BF16 = 0, 1
 STATUS = {0: "GDPA_OK", 1: "GDPA_ERR_INVALID_ARG", 2: "GDPA_ERR_UNSUPPORTED",
           3: "GDPA_ERR_CUDA", 4: "GDPA_ERR_TIMEOUT", 5: "GDPA_ERR_WORKSPACE"}

@@ -36,7 +36,8 @@ import numpy as np
 import torch
 
 PHI_IDENTITY, PHI_SILU, PHI_SOFTMAX = 0, 1, 2
-PHI_NAMES = {PHI_IDENTITY: "identity", PHI_SILU: "silu", PHI_SOFTMAX: "softmax"}
+PHI_NAMES = {PHI_IDENTITY: "identity", PHI_SILU: "silu", PHI_SOFTMAX: "softmax", 3: "relu",
+             4: "gelu"}
 
 _GAMMA = 0x9E3779B97F4A7C15
 _M1 = 0xBF58476D1CE4E5B9

@@ -57,6 +57,9 @@ def check(out, d, phi, scale, backward, dtype, label=""):
     return errs
 
 
+# identity, SiLU, softmax and the PFFN variants' other activations
+PHIS = ["identity", "silu", "softmax", "relu", "gelu"]
+
 SMALL = [
     # (n per sample, m)
     ([130, 0, 17, 256], 200),
@@ -71,7 +74,7 @@ SMALL = [
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("dh", [32, 64, 128])
-@pytest.mark.parametrize("phi", ["identity", "silu", "softmax"])
+@pytest.mark.parametrize("phi", PHIS)
 @pytest.mark.parametrize("case", range(len(SMALL)))
 def test_small_jagged(case, phi, dh, dtype):
     n, m = SMALL[case]
@@ -84,7 +87,7 @@ def test_small_jagged(case, phi, dh, dtype):
     check(out, d, phi, scale, True, dtype, f"n={n} m={m}")
 
 
-@pytest.mark.parametrize("phi", ["identity", "silu", "softmax"])
+@pytest.mark.parametrize("phi", PHIS)
 @pytest.mark.parametrize("n", [[100], [300, 7], [129, 0, 640]])
 def test_odd_head_count(n, phi):
     """h = 3: the work list can hold an odd number of tiles and mixes tiles of
@@ -112,7 +115,7 @@ def test_softmax_row_max_growth(dh):
     check(out, d, "softmax", scale, True, torch.bfloat16, f"growth dh={dh}")
 
 
-@pytest.mark.parametrize("phi", ["identity", "silu", "softmax"])
+@pytest.mark.parametrize("phi", PHIS)
 def test_negative_scale(phi):
     """A negative scale flips the logits (the softmax kernels then track a row
     minimum of the raw dot products)."""
