@@ -98,6 +98,20 @@ def test_odd_head_count(n, phi):
     check(out, d, phi, scale, True, torch.bfloat16, f"h=3 n={n}")
 
 
+@pytest.mark.parametrize("phi", ["softmax", "silu"])
+@pytest.mark.parametrize("dh", [64, 128])
+def test_many_samples_unsorted_work_list(phi, dh):
+    """B = 4500 > 4096: the backward's work list is not sorted by length, and
+    thousands of one-tile items, a third of them without tokens, pass through
+    each CTA's K/V slots, staging buffers and statistics ring."""
+    rng = np.random.default_rng(7)
+    n = rng.choice([0, 1, 2, 50, 130], size=4500, p=[0.3, 0.2, 0.2, 0.2, 0.1]).tolist()
+    d = syn.random_problem(61, len(n), 2, dh, 64, n, dtype=torch.bfloat16, std=0.6)
+    scale = 1.0 / dh ** 0.5 if phi == "softmax" else 0.5
+    out = run_gpu(d, phi, scale, True)
+    check(out, d, phi, scale, True, torch.bfloat16, f"B=4500 dh={dh}")
+
+
 @pytest.mark.parametrize("dh", [32, 64, 128])
 def test_softmax_row_max_growth(dh):
     """Logits that grow from one key block to the next (and one that jumps by
