@@ -1170,7 +1170,7 @@ template <int DH>
 bool make_bwd_maps(const gdpa_problem_t& p, const void* q, const void* g, const void* k,
                    const void* v, CUtensorMap* mq, CUtensorMap* mg, CUtensorMap* mk,
                    CUtensorMap* mv) {
-  using C = BwdCfg<DH>;
+  constexpr int CH = DH < 64 ? DH : 64;                 // columns of one swizzled box row
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   const CUtensorMapSwizzle sw = DH < 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
@@ -1178,7 +1178,7 @@ bool make_bwd_maps(const gdpa_problem_t& p, const void* q, const void* g, const 
   const cuuint64_t qd[3] = {(cuuint64_t)DH, (cuuint64_t)p.h,
                             (cuuint64_t)(p.total_tokens > 0 ? p.total_tokens : 1)};
   const cuuint64_t qs[2] = {(cuuint64_t)DH * 2, (cuuint64_t)p.h * DH * 2};
-  const cuuint32_t qb[3] = {(cuuint32_t)C::CH, 1, 128};
+  const cuuint32_t qb[3] = {(cuuint32_t)CH, 1, 128};
   for (int i = 0; i < 2; ++i)
     if (enc(i ? mg : mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(i ? g : q), qd, qs,
             qb, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1187,7 +1187,7 @@ bool make_bwd_maps(const gdpa_problem_t& p, const void* q, const void* g, const 
   const cuuint64_t kd[4] = {(cuuint64_t)DH, (cuuint64_t)p.m, (cuuint64_t)p.h, (cuuint64_t)p.B};
   const cuuint64_t ks[3] = {(cuuint64_t)DH * 2, (cuuint64_t)p.m * DH * 2,
                             (cuuint64_t)p.h * p.m * DH * 2};
-  const cuuint32_t kb[4] = {(cuuint32_t)C::CH, 128, 1, 1};
+  const cuuint32_t kb[4] = {(cuuint32_t)CH, 128, 1, 1};
   for (int i = 0; i < 2; ++i)
     if (enc(i ? mv : mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(i ? v : k), kd, ks,
             kb, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1218,13 +1218,10 @@ cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* 
                          const void* k, const void* v, const float* lse, const float* dsum,
                          const void* g, void* dk, void* dv, float* dq_acc, WsHeader* ws,
                          const Tile* tiles, cudaStream_t st) {
-  using C = BwdCfg<DH>;
   CUtensorMap mq, mg, mk, mv;
   if (p.total_tokens == 0) q = g = k;   // no query rows: the maps are never read
   if (!make_bwd_maps<DH>(p, q, g, k, v, &mq, &mg, &mk, &mv)) return cudaErrorInvalidValue;
-  auto kern = gdpa_bwd_sm100_kernel<DH, PHI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
   BwdArgs args;
   args.tiles = tiles;
   args.ws = ws;
@@ -1252,10 +1249,15 @@ cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* 
     KernelScope ks_("gdpa_bwd_sm100", st);
     hk<<<device_sm_count(), kHalfThreads, H::SMEM, st>>>(mq, mg, mk, mv, mdq, mdv, mdk, args);
     return cudaGetLastError();
+  } else {
+    using C = BwdCfg<DH>;
+    auto kern = gdpa_bwd_sm100_kernel<DH, PHI>;     // dh = 128 only
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+    if (e != cudaSuccess) return e;
+    KernelScope ks_("gdpa_bwd_sm100", st);
+    kern<<<device_sm_count(), kThreads, C::SMEM, st>>>(mq, mg, mk, mv, args);
+    return cudaGetLastError();
   }
-  KernelScope ks_("gdpa_bwd_sm100", st);
-  kern<<<device_sm_count(), kThreads, C::SMEM, st>>>(mq, mg, mk, mv, args);
-  return cudaGetLastError();
 }
 
 template <int DH>
