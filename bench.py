@@ -73,6 +73,16 @@ def parse():
     return ap.parse_args()
 
 
+def e2e_chunks(offsets, nchunks):
+    """Equal groups of consecutive samples for the end-to-end step: a list of
+    ((first sample, end sample), (first token row, end token row)), non-empty,
+    in order, covering every sample once."""
+    nb = len(offsets) - 1
+    bounds = [nb * c // nchunks for c in range(nchunks + 1)]
+    return [((b0, b1), (offsets[b0], offsets[b1]))
+            for b0, b1 in zip(bounds[:-1], bounds[1:]) if b1 > b0]
+
+
 def workload(args):
     """The benchmarked workload, with its activation replaced when --phi is given."""
     import synthetic as syn
@@ -375,13 +385,8 @@ def main():
         ho, hdq, hdk, hdv = (torch.empty(x.shape, dtype=x.dtype).pin_memory()
                              for x in (o, dq, dk, dv))
         offs = [int(x) for x in d["offsets"]]
-        nb = len(offs) - 1
-        bounds = [nb * c // E2E_CHUNKS for c in range(E2E_CHUNKS + 1)]
         chunks = []
-        for b0, b1 in zip(bounds[:-1], bounds[1:]):
-            if b1 <= b0:
-                continue
-            t0_, t1_ = offs[b0], offs[b1]
+        for (b0, b1), (t0_, t1_) in e2e_chunks(offs, E2E_CHUNKS):
             coff = [x - t0_ for x in offs[b0:b1 + 1]]
             cp_ = pkg.problem_for(q[t0_:t1_], k[b0:b1], coff, wl.phi_name, wl.scale,
                                   max_n=max(coff[i + 1] - coff[i] for i in range(b1 - b0)))

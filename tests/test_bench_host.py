@@ -20,3 +20,17 @@ def test_phi_override_keeps_shapes_and_scale():
         assert (wl.B, wl.h, wl.dh, wl.m, wl.scale, wl.lengths) == \
             (base.B, base.h, base.dh, base.m, base.scale, base.lengths)
     assert bench.workload(argparse.Namespace(phi="softmax")) is base
+
+
+def test_e2e_chunks_cover_every_sample_once():
+    import numpy as np
+    for B, nchunks in ((1024, 8), (5, 8), (7, 3), (1, 1)):
+        n = np.random.default_rng(B).integers(0, 50, size=B)
+        off = [0] + np.cumsum(n).tolist()
+        ch = bench.e2e_chunks(off, nchunks)
+        assert ch[0][0][0] == 0 and ch[-1][0][1] == B
+        assert all(b1 > b0 for (b0, b1), _ in ch)
+        for ((_, e0), (_, r0)), ((s1, _), (t1, _)) in zip(ch, ch[1:]):
+            assert e0 == s1 and r0 == t1                      # contiguous samples and rows
+        assert all(t0 == off[b0] and t1 == off[b1] for (b0, b1), (t0, t1) in ch)
+        assert len(ch) == min(nchunks, B)
