@@ -145,7 +145,11 @@ struct BwdCfg {
                        B_STFULL = 11, B_STEMPTY = 11 + NSTG, NBAR = 11 + 2 * NSTG;
   static constexpr uint32_t OFF_K = 0, OFF_V = TILEB, OFF_STG = 2 * TILEB;
   static constexpr uint32_t OFF_DS = OFF_STG + NSTG * 2 * TILEB;
-  static constexpr uint32_t OFF_CTL = OFF_DS + DSB;
+  // dV/dK epilogue: per activation warp, 32 rows x 64 columns of bf16 (128 B
+  // rows), to turn its key rows into whole-row global stores
+  static constexpr uint32_t KSTG_WARP = 32 * 128;
+  static constexpr uint32_t OFF_KSTG = OFF_DS + DSB;
+  static constexpr uint32_t OFF_CTL = OFF_KSTG + 8 * KSTG_WARP;
   static constexpr uint32_t CTL_BYTES = 1024 + 8 * 2 * 128 * 4;  // barriers + per-warp row stats
   static constexpr uint32_t SMEM_USED = 1024 + OFF_CTL + CTL_BYTES;
   static constexpr uint32_t SMEM = SMEM_USED > 120u * 1024u ? SMEM_USED : 120u * 1024u;
@@ -158,6 +162,7 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmG,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const BwdArgs a) {
+  static_assert(DH == 128, "dh <= 64 runs gdpa_bwd_half_kernel");
   using C = BwdCfg<DH>;
   constexpr bool SOFTMAX = PHI == GDPA_PHI_SOFTMAX;
   constexpr uint32_t IDESC_T = idesc_bf16(128, 128, 0, 0);   // S^T, dP^T
@@ -513,26 +518,55 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
       tc_fence_after();
       {
+        // Group 0 writes dV, group 1 s*dK.  Each lane owns one key row; the
+        // warp passes its 32 rows through its own shared-memory area (64
+        // columns at a time, 16-byte chunks swizzled by row) so that every
+        // global store instruction writes 4 whole 128-byte row pieces.
         const uint32_t src = tmem + lane_off + (grp == 0 ? C::COL_DV : C::COL_DK);
         const float mul = grp == 0 ? 1.f : sc;
+        const uint32_t kstg = base + C::OFF_KSTG + (uint32_t)(warp - 4) * C::KSTG_WARP;
+        __nv_bfloat16* blk = (grp == 0 ? a.dv : a.dk) +
+                             (((int64_t)it.b * a.h + it.head) * a.m + it.row0 + quad * 32) * DH;
+        const int rl = lane >> 3, jl = lane & 7;         // read-back: row in group of 4, chunk
 #pragma unroll
-        for (int c = 0; c < DH; c += 16) {
-          uint32_t v[16];
-          tmem_ld_x16(src + c, v);
-          tmem_wait_ld();
-          uint32_t pk[8];
+        for (int c0 = 0; c0 < DH; c0 += 64) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            pk[u] = pack_bf16x2(__uint_as_float(v[2 * u]) * mul, __uint_as_float(v[2 * u + 1]) * mul);
-          if (key < a.m) {
-            uint4* d4 = reinterpret_cast<uint4*>(kvout + c);
-            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          for (int c = 0; c < 64; c += 16) {
+            uint32_t v[16];
+            tmem_ld_x16(src + c0 + c, v);
+            tmem_wait_ld();
+            if (c0 + c + 16 == DH) {
+              tc_fence_before();
+              mbar_arrive(bar(C::B_ACCEMPTY));          // the accumulators are free
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                pk[u] = pack_bf16x2(__uint_as_float(v[8 * j + 2 * u]) * mul,
+                                    __uint_as_float(v[8 * j + 2 * u + 1]) * mul);
+              const uint32_t chunk = (uint32_t)(c / 8 + j);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                           ::"r"(kstg + lane * 128 + ((chunk ^ (uint32_t)(lane & 7)) << 4)),
+                           "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                           : "memory");
+            }
           }
+          __syncwarp();
+#pragma unroll
+          for (int it4 = 0; it4 < 8; ++it4) {
+            const int r = it4 * 4 + rl;                  // row within this warp's 32
+            uint4 val;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                         : "r"(kstg + r * 128 + (((uint32_t)jl ^ (uint32_t)(r & 7)) << 4)));
+            if (it.row0 + quad * 32 + r < a.m)
+              *reinterpret_cast<uint4*>(blk + (int64_t)r * DH + c0 + jl * 8) = val;
+          }
+          __syncwarp();
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(C::B_ACCEMPTY));
       ++ic;
     }
   }
