@@ -385,22 +385,46 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         const bool w = mbar_wait(bar(C::B_DQFULL + b), par, abort_flag, kTimeoutNs);
         if (!__all_sync(0xffffffffu, w)) return false;
         tc_fence_after();
-        const int rg = 128 * ii + lrow;
-        float* dst = a.dq_acc + ((int64_t)(t0 + rg) * a.h + it.head) * DH + grp * (DH / 2);
+        // Lane = query row.  This group's DH/2 columns go through the warp's
+        // shared-memory area, 32 fp32 columns (128 B of a row) at a time, so
+        // that each vector reduction instruction covers 4 whole row pieces.
+        const uint32_t kstg = base + C::OFF_KSTG + (uint32_t)(warp - 4) * C::KSTG_WARP;
+        const int rl = lane >> 3, jl = lane & 7;
+        float* rows = a.dq_acc + ((int64_t)(t0 + 128 * ii + quad * 32) * a.h + it.head) * DH +
+                      grp * (DH / 2);
 #pragma unroll
-        for (int c = 0; c < DH / 2; c += 16) {
-          uint32_t v[16];
-          tmem_ld_x16(tmem + lane_off + C::COL_DQ + b * DH + grp * (DH / 2) + c, v);
-          tmem_wait_ld();
-          if (rg < n) {
+        for (int c0 = 0; c0 < DH / 2; c0 += 32) {
 #pragma unroll
-            for (int u = 0; u < 16; u += 4)
-              red_add_v4(dst + c + u, __uint_as_float(v[u]), __uint_as_float(v[u + 1]),
-                         __uint_as_float(v[u + 2]), __uint_as_float(v[u + 3]));
+          for (int c = 0; c < 32; c += 16) {
+            uint32_t v[16];
+            tmem_ld_x16(tmem + lane_off + C::COL_DQ + b * DH + grp * (DH / 2) + c0 + c, v);
+            tmem_wait_ld();
+            if (c0 + c + 16 == DH / 2) {
+              tc_fence_before();
+              mbar_arrive(bar(C::B_DQEMPTY + b));       // the dQ columns are free
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t chunk = (uint32_t)(c / 4 + j);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                           ::"r"(kstg + lane * 128 + ((chunk ^ (uint32_t)(lane & 7)) << 4)),
+                           "r"(v[4 * j]), "r"(v[4 * j + 1]), "r"(v[4 * j + 2]), "r"(v[4 * j + 3])
+                           : "memory");
+            }
           }
+          __syncwarp();
+#pragma unroll
+          for (int it4 = 0; it4 < 8; ++it4) {
+            const int r = it4 * 4 + rl;                  // row within this warp's 32
+            float4 val;
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(val.x), "=f"(val.y), "=f"(val.z), "=f"(val.w)
+                         : "r"(kstg + r * 128 + (((uint32_t)jl ^ (uint32_t)(r & 7)) << 4)));
+            if (128 * ii + quad * 32 + r < n)
+              red_add_v4(rows + (int64_t)r * a.h * DH + c0 + jl * 4, val.x, val.y, val.z, val.w);
+          }
+          __syncwarp();
         }
-        tc_fence_before();
-        mbar_arrive(bar(C::B_DQEMPTY + b));
         return true;
       };
       // softmax row statistics of a query tile, loaded one step ahead
