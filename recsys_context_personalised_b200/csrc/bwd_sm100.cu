@@ -437,8 +437,8 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           nd[u] = 0.f;
           if (rg < n) {
             const int64_t at = (int64_t)it.head * a.T + t0 + rg;
-            nl[u] = a.lse[at] * 1.4426950408889634f;
-            nd[u] = a.dsum[at];
+            nl[u] = __ldg(a.lse + at);                 // raw: consumed a tile later
+            nd[u] = __ldg(a.dsum + at);
           }
         }
       };
@@ -449,7 +449,7 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           __syncwarp();
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            wst[32 * u + lane] = nl[u];
+            wst[32 * u + lane] = nl[u] * 1.4426950408889634f;   // log2 units
             wst[64 + 32 * u + lane] = nd[u];
           }
           __syncwarp();
