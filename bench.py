@@ -1,31 +1,36 @@
 #!/usr/bin/env python
-"""GDPA benchmark: forward + backward TFLOP/s on one B200 (or N replicas).
+"""GDPA benchmark: TFLOP/s of the fused hot path on one B200 (or N replicas).
 
 One step = the whole GDPA hot path over one synthetic batch: tile scheduling,
-the fused forward (S = s Q K^T, P = phi(S), O = P V, softmax statistics) and
-the fused backward (dQ, dK, dV).  The workload is the largest jagged bf16
-softmax problem: B = 1024 samples with power-law (alpha = 1.5) history lengths
-on [32, 4096], h = 16 heads, dh = 64, m = 2048 context keys per sample and
-head, scale 1/sqrt(dh).
+the fused forward (S = s Q K^T, P = phi(S), O = P V, softmax statistics) and,
+for the workloads that train (4 and 5), the fused backward (dQ, dK, dV).  The
+default workload is the largest jagged bf16 softmax problem: B = 1024 samples
+with power-law (alpha = 1.5) history lengths on [32, 4096], h = 16 heads,
+dh = 64, m = 2048 context keys per sample and head, scale 1/sqrt(dh).
+``--workload 1..5`` runs any of the five problem shapes.
 
 Throughput counts algorithmic FLOPs only: forward 4*T*h*m*dh, backward
-8*T*h*m*dh (the recomputation of S in the backward is not credited).
+8*T*h*m*dh (the recomputation of S in the backward is not credited).  Every
+step is bracketed by its own CUDA events, and the L2 is flushed (a 256 MB
+write) between steps, outside the events.
 
 Multi-GPU: samples are independent and the op has no exchange step, so N
 ranks run N independent batches (weak scaling, no collective on the data
-path; a barrier and one max-reduction of the timings only).
+path; a barrier and one max-reduction of the timings only).  ``--gpus N``
+without a torchrun environment relaunches itself under torchrun.
 
-``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
-same workload (rank 0 only), in the same units.
+``--impl reference`` times the fp64 CPU oracle on a fixed seeded sample of
+the same workload (rank 0 only), in the same units.
 """
 from __future__ import annotations
 
 import argparse
 import dataclasses
 import datetime
+import hashlib
 import json
-import math
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -34,43 +39,51 @@ import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
+CSRC = os.path.join(ROOT, "recsys_context_personalised_b200", "csrc")
 
-WORKLOAD = 5
+DEFAULT_WORKLOAD = 5
 E2E_CHUNKS = 8                          # sample groups of the end-to-end step
 FLOPS_FWD, FLOPS_BWD = 4, 8            # x T*h*m*dh
+L2_FLUSH_BYTES = 256 << 20              # > the 126 MB L2
 # algorithmic FLOPs credited to each kernel, in units of T*h*m*dh
 KERNEL_FLOPS = {"gdpa_fwd_sm100": 4, "gdpa_bwd_sm100": 8, "gdpa_simt_fwd": 4,
                 "gdpa_simt_bwd_dq": 4, "gdpa_simt_bwd_dkdv": 4}
 TENSOR_KERNELS = {"gdpa_fwd_sm100", "gdpa_bwd_sm100"}
+FWD_KERNELS = {"gdpa_fwd_sm100", "gdpa_simt_fwd"}
+# Source files whose contents decide each fused kernel's DRAM traffic.
+KERNEL_SOURCES = {"gdpa_fwd_sm100": ("fwd_sm100.cu", "sm100.cuh", "gdpa_internal.cuh"),
+                  "gdpa_bwd_sm100": ("bwd_sm100.cu", "sm100.cuh", "gdpa_internal.cuh")}
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per unit T*h*m*dh of
-# the fused kernels, from one ncu capture on the first 64 samples of this
-# workload (T = 20,846; `bench.py --samples 64 --steps 1 --warmup 1`):
-# backward 743,162,880 + 589,410,048 B, forward 580,738,816 + 34,836,480 B.
-# A launch's traffic is this times its units; valid only for the kernels as
-# captured (set an entry to None when its kernel changes).
-_CAPTURE_UNITS = 20846 * 16 * 2048 * 64
-TRAFFIC_PER_UNIT = {"gdpa_bwd_sm100": (743162880 + 589410048) / _CAPTURE_UNITS,
-                    "gdpa_fwd_sm100": (580738816 + 34836480) / _CAPTURE_UNITS}
+# a fused kernel, from one ncu capture: {kernel: {workload id: (bytes per unit,
+# sha16 of the kernel's sources at capture time)}}.  An entry whose hash no
+# longer matches the sources is not used (the traffic is then reported null).
+TRAFFIC_PER_UNIT = {}
 # fp32 FFMA peak for the SIMT kernels: 148 SMs * 128 FMA/clk * 2 flop * 1.965 GHz
 SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# dense bf16 tcgen05 rate of one SM (flop per clock), for the clock-scaled nominal peak
+MMA_FLOP_PER_CLK_SM = 8192
+# oracle sample per reference step / per cpu_baseline pass: this many fp64 FLOPs
+ORACLE_STEP_FLOPS = 6.0e10
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-passes", type=int, default=3,
+                    help="passes of the oracle over its fixed sample for cpu_baseline")
     ap.add_argument("--samples", type=int, default=0,
                     help="run only the first N samples of the workload (small profiling case)")
     ap.add_argument("--phi", default=None,
                     choices=["identity", "silu", "softmax", "relu", "gelu"],
                     help="the same workload with another activation (the PFFN variants' phi)")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def e2e_chunks(offsets, nchunks):
@@ -86,11 +99,56 @@ def e2e_chunks(offsets, nchunks):
 def workload(args):
     """The benchmarked workload, with its activation replaced when --phi is given."""
     import synthetic as syn
-    wl = syn.WORKLOADS[WORKLOAD]
+    wl = syn.WORKLOADS[getattr(args, "workload", DEFAULT_WORKLOAD)]
     if args.phi and args.phi != wl.phi_name:
         code = {v_: k_ for k_, v_ in syn.PHI_NAMES.items()}[args.phi]
         wl = dataclasses.replace(wl, phi=code, name=wl.name.replace(wl.phi_name, args.phi))
     return wl
+
+
+def metric_name(wl):
+    return "GDPA fwd+bwd TFLOP/s" if wl.backward else "GDPA fwd TFLOP/s"
+
+
+def step_flop_units(wl):
+    """Algorithmic FLOPs of one step in units of T*h*m*dh."""
+    return FLOPS_FWD + (FLOPS_BWD if wl.backward else 0)
+
+
+def fwd_bytes(wl, T):
+    """Algorithmic HBM bytes of one forward: Q, K, V read once, O written, LSE."""
+    e = 2 if wl.dtype.itemsize == 2 else 4
+    b = e * (2 * T * wl.h * wl.dh + 2 * wl.B * wl.h * wl.m * wl.dh)
+    return b + (4 * T * wl.h if wl.phi_name == "softmax" else 0)
+
+
+def config_dict(wl, T, n_gpus, subset=None):
+    """The `config` object of the JSON line (identical in both arms)."""
+    return {"workload": wl.name if subset is None else
+            f"{wl.name} (first {len(subset)} samples only: profiling case)",
+            "B": wl.B if subset is None else len(subset), "h": wl.h, "dh": wl.dh, "m": wl.m,
+            "phi": wl.phi_name, "scale": wl.scale, "lengths": wl.lengths,
+            "backward": wl.backward, "tokens_per_rank": int(T),
+            "parallelism": f"replicas x{n_gpus} (samples independent)",
+            "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write outside the "
+                  "per-step events)"}
+
+
+def sources_sha16(kernel):
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kernel, ()):
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel, wid, units):
+    """DRAM bytes of one launch from the recorded capture, or None when no
+    capture exists for this kernel and workload or its sources changed since."""
+    ent = TRAFFIC_PER_UNIT.get(kernel, {}).get(wid)
+    if not ent or ent[1] != sources_sha16(kernel):
+        return None
+    return ent[0] * units
 
 
 def peaks():
@@ -98,38 +156,50 @@ def peaks():
     try:
         with open(path) as f:
             d = json.load(f)
-        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
-                    bf16_sustained=d["bf16_tflops_sustained"], source="measured")
-    except (OSError, KeyError, ValueError):
-        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+        out = dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                   bf16_sustained=float(d.get("bf16_tflops_sustained") or d["bf16_tflops"]),
+                   source="measured", sustained_mhz=None)
+        cl = d.get("clocks_under_load") or d.get("sustained_clocks") or {}
+        if isinstance(cl, dict):
+            for k_ in ("sm_mhz_median", "sm_mhz", "median_sm_mhz"):
+                if isinstance(cl.get(k_), (int, float)):
+                    out["sustained_mhz"] = float(cl[k_])
+                    break
+        return out
+    except (OSError, KeyError, ValueError, TypeError):
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback",
+                    sustained_mhz=1300.0)
+
+
+def choose_bf16_peak(pk, clk):
+    """Burst or sustained dense bf16 peak, from the SM clock this run saw.
+
+    The sustained figure was taken over a seconds-long GEMM loop that settled
+    at a lower clock under the power cap; the burst figure applies while the
+    clocks stay near their maximum.  The run's median SM clock decides."""
+    med = clk.get("sm_mhz") if clk else None
+    mx = clk.get("sm_max_mhz") if clk else None
+    if med and pk.get("sustained_mhz") and med <= 1.05 * pk["sustained_mhz"]:
+        return pk["bf16_sustained"], (f"{pk['source']} bf16 dense, sustained: median SM clock "
+                                      f"{med:.0f} MHz is at the sustained run's "
+                                      f"{pk['sustained_mhz']:.0f} MHz")
+    why = (f"median SM clock {med:.0f} of {mx:.0f} MHz" if med and mx else "no clock record")
+    return pk["bf16"], f"{pk['source']} bf16 dense, burst ({why})"
 
 
 # --------------------------------------------------------------------------
-# CPU oracle timing (the reported baseline; the oracle as it stands)
+# CPU oracle (the reported baseline; the oracle as it stands)
 
 
 def _oracle_unit_flops(n, wl):
-    return (FLOPS_FWD + FLOPS_BWD) * int(n) * wl.h * wl.m * wl.dh
+    return step_flop_units(wl) * int(n) * wl.h * wl.m * wl.dh
 
 
-def time_oracle(wl, lengths, seconds, seed=0):
-    """Time the oracle's fwd+bwd on a seeded sample of samples (~`seconds`)."""
+def oracle_sample(wl, lengths, budget=ORACLE_STEP_FLOPS):
+    """A fixed seeded choice of samples whose oracle FLOPs fill `budget`
+    (the same choice in the cpu_baseline leg and the reference arm)."""
     import numpy as np
-
-    import oracle
-    import synthetic as syn
-    rng = np.random.default_rng(1234)
-    order = rng.permutation(len(lengths))
-    threads = oracle.max_threads()
-    # calibrate on one short sample (its h units keep min(h, threads) cores busy)
-    probe = [int(next(b for b in order if lengths[b] <= 256))]
-    d = syn.make_inputs(wl.wid, samples=probe, backward=True, seed=seed)
-    t = time.perf_counter()
-    oracle.fwd(d["q"], d["k"], d["v"], d["offsets"], wl.phi_name, wl.scale)
-    oracle.bwd(d["q"], d["k"], d["v"], d["dout"], d["offsets"], wl.phi_name, wl.scale)
-    dt = max(time.perf_counter() - t, 1e-3)
-    per_core = _oracle_unit_flops(lengths[probe[0]], wl) / dt / min(threads, wl.h)
-    budget = per_core * threads * seconds
+    order = np.random.default_rng(1234).permutation(len(lengths))
     pick, acc = [], 0
     for b in order:
         f = _oracle_unit_flops(lengths[b], wl)
@@ -137,21 +207,33 @@ def time_oracle(wl, lengths, seconds, seed=0):
             continue
         pick.append(int(b))
         acc += f
-        if acc >= 0.8 * budget:
+        if acc >= 0.9 * budget:
             break
-    return pick, threads
+    return sorted(pick)
 
 
-def run_oracle_sample(wl, samples, seed=0):
+def run_oracle_sample(wl, inputs):
     import oracle
-    import synthetic as syn
-    d = syn.make_inputs(wl.wid, samples=samples, backward=True, seed=seed)
+    d = inputs
     t = time.perf_counter()
     oracle.fwd(d["q"], d["k"], d["v"], d["offsets"], wl.phi_name, wl.scale)
-    oracle.bwd(d["q"], d["k"], d["v"], d["dout"], d["offsets"], wl.phi_name, wl.scale)
+    if wl.backward:
+        oracle.bwd(d["q"], d["k"], d["v"], d["dout"], d["offsets"], wl.phi_name, wl.scale)
     dt = time.perf_counter() - t
     flops = sum(_oracle_unit_flops(n, wl) for n in d["lengths"])
     return flops, dt, int(d["lengths"].sum())
+
+
+def oracle_inputs(wl, samples):
+    """Host inputs of the chosen samples (the activation does not change them)."""
+    import synthetic as syn
+    return syn.make_inputs(wl.wid, samples=samples, backward=wl.backward)
+
+
+def oracle_desc(wl, samples, tokens):
+    return (f"{len(samples)} of {wl.B} samples ({tokens} tokens, all {wl.h} heads), "
+            f"{'fwd+bwd' if wl.backward else 'fwd'}, fixed seeded choice of "
+            f"~{ORACLE_STEP_FLOPS / 1e9:.0f} GFLOP")
 
 
 # --------------------------------------------------------------------------
@@ -234,6 +316,29 @@ def aggregate(ms, flops, tokens, launches, world, dist=None, device=None):
             "tokens_per_s": tokens / (ms / 1e3) if ms > 0 else 0.0}
 
 
+def torchrun_command(args_list, n, port):
+    """The torchrun command line that runs this script on n local ranks."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__), *args_list]
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def world_from_env(args):
+    """(rank, world, local_rank); raises when a torchrun world disagrees with --gpus."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if "WORLD_SIZE" in os.environ and world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}")
+    return rank, world, local_rank
+
+
 def run_reference(args, rank):
     """The oracle, as it stands, on the host cores; rank 0 only."""
     if rank != 0:
@@ -241,44 +346,43 @@ def run_reference(args, rank):
     import synthetic as syn
     wl = workload(args)
     lengths = syn.lengths(wl)
-    total = args.steps + args.warmup
-    per_step = max(1.0, min(8.0, 150.0 / max(total, 1)))
-    samples, threads = time_oracle(wl, lengths, per_step)
+    samples = oracle_sample(wl, lengths)
+    inputs = oracle_inputs(wl, samples)
+    import oracle
+    threads = oracle.max_threads()
     for _ in range(args.warmup):
-        run_oracle_sample(wl, samples)
+        run_oracle_sample(wl, inputs)
     flops = secs = 0.0
     tokens = 0
     for _ in range(args.steps):
-        f, dt, tk = run_oracle_sample(wl, samples)
+        f, dt, tk = run_oracle_sample(wl, inputs)
         flops += f
         secs += dt
         tokens += tk
     value = flops / secs / 1e12
-    sample_desc = (f"{len(samples)} of {wl.B} samples per step ({tokens // max(args.steps, 1)} "
-                   f"tokens, all {wl.h} heads), fwd+bwd, seeded choice")
-    emit({"impl": "reference", "metric": "GDPA fwd+bwd TFLOP/s", "value": value,
+    emit({"impl": "reference", "metric": metric_name(wl), "value": value,
           "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
           "ms_per_step": 1e3 * secs / max(args.steps, 1), "higher_is_better": True,
           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-          "config": {"workload": wl.name, "B": wl.B, "h": wl.h, "dh": wl.dh, "m": wl.m,
-                     "phi": wl.phi_name, "lengths": wl.lengths, "parallelism": "none (CPU)"},
+          "config": config_dict(wl, int(lengths.sum()), args.gpus),
           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                           "sample": sample_desc},
+                           "sample": oracle_desc(wl, samples, tokens // max(args.steps, 1))},
           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                   "d2h_bytes_per_step": 0},
           "tokens_per_s": tokens / secs})
 
 
-def main():
-    args = parse()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+def main(argv=None):
+    args = parse(argv)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        argv = sys.argv[1:] if argv is None else list(argv)
+        cmd = torchrun_command(argv, args.gpus, _free_port())
+        raise SystemExit(subprocess.call(cmd))
+    rank, world, local_rank = world_from_env(args)
     if args.impl == "reference":
         run_reference(args, rank)
         return
 
-    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -298,33 +402,36 @@ def main():
 
     wl = workload(args)
     subset = list(range(args.samples)) if 0 < args.samples < wl.B else None
-    d = syn.make_inputs(WORKLOAD, device=dev, seed=rank, backward=True, samples=subset)
-    q, k, v, g = d["q"], d["k"], d["v"], d["dout"]
+    d = syn.make_inputs(wl.wid, device=dev, seed=rank, backward=wl.backward, samples=subset)
+    q, k, v, g = d["q"], d["k"], d["v"], d.get("dout")
     T = int(d["offsets"][-1])
     off = torch.tensor(d["offsets"], dtype=torch.int32, device=dev)
     p = pkg.problem_for(q, k, d["offsets"], wl.phi_name, wl.scale,
                         max_n=int(d["lengths"].max()))
     o = torch.empty_like(q)
     lse = torch.empty((wl.h, T), dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dq, dk, dv = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)) \
+        if wl.backward else (None, None, None)
     ws_f = pkg.workspace(pkg.fwd_workspace_bytes(p), dev)
-    ws_b = pkg.workspace(pkg.bwd_workspace_bytes(p), dev)
+    ws_b = pkg.workspace(pkg.bwd_workspace_bytes(p), dev) if wl.backward else None
     stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     launches = [0]
 
     def step():
         G.fwd(p, q, off, k, v, o=o, lse=lse, ws=ws_f, stream=stream)
         launches[0] += G.last_launch_count()
-        G.bwd(p, q, off, k, v, o, lse, g, dq=dq, dk=dk, dv=dv, ws=ws_b, stream=stream)
-        launches[0] += G.last_launch_count()
+        if wl.backward:
+            G.bwd(p, q, off, k, v, o, lse, g, dq=dq, dk=dk, dv=dv, ws=ws_b, stream=stream)
+            launches[0] += G.last_launch_count()
 
     for _ in range(max(args.warmup, 0)):
         step()
     torch.cuda.synchronize()
-    if pkg.workspace_status(ws_f) or pkg.workspace_status(ws_b):
+    if pkg.workspace_status(ws_f) or (ws_b is not None and pkg.workspace_status(ws_b)):
         raise RuntimeError("device-side status error during warm-up")
 
-    # ---- timed region (device events; inputs are far larger than L2) ----
+    # ---- timed region: per-step device events, L2 flushed between steps ----
     clocks = ClockSampler(local_rank)
     barrier()
     torch.cuda.synchronize()
@@ -332,58 +439,85 @@ def main():
     time.sleep(0.3)
     G.timing_enable(True)
     launches[0] = 0
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for _ in range(args.steps):
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
         step()
-    ev1.record(stream)
+        e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     per_kernel = G.timing_read()
     G.timing_enable(False)
     clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in evs)
     unit_flops = float(T) * wl.h * wl.m * wl.dh
-    agg = aggregate(ms, (FLOPS_FWD + FLOPS_BWD) * unit_flops * args.steps, float(T) * args.steps,
+    agg = aggregate(ms, step_flop_units(wl) * unit_flops * args.steps, float(T) * args.steps,
                     float(launches[0]), world, dist, dev)
     ms_max, value, n_launch = agg["ms_max"], agg["tflops"], agg["launches"]
 
-    # ---- dominant kernel roofline ----
+    # ---- rooflines: dominant kernel, and the forward kernel on its own ----
     pk = peaks()
-    credited = {k_: v_ for k_, v_ in per_kernel.items() if KERNEL_FLOPS.get(k_, 0)}
-    top = max((credited or per_kernel).items(), key=lambda kv: kv[1][1])
-    name, (nl, tot_ms) = top
-    avg_ms = tot_ms / max(nl, 1)
-    per_launch_flops = KERNEL_FLOPS.get(name, 0) * unit_flops
-    achieved = per_launch_flops / (avg_ms / 1e3) / 1e12
-    if name in TENSOR_KERNELS:
-        roof = {"bound": "tensor", "peak": pk["bf16_sustained"],
-                "peak_source": f"{pk['source']} bf16 dense, sustained (kernel timed inside a long step loop)"}
-    else:
-        roof = {"bound": "alu", "peak": SIMT_PEAK_TFLOPS,
-                "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz"}
-    tpu = TRAFFIC_PER_UNIT.get(name) if WORKLOAD == 5 and wl.phi_name == "softmax" else None
-    roof.update(kernel=name, achieved=achieved, unit="TFLOP/s", frac=achieved / roof["peak"],
-                traffic=tpu * unit_flops if tpu else None,
-                traffic_source=("ncu DRAM bytes of a 64-sample capture, scaled by T*h*m*dh"
-                                if tpu else None),
-                launches=nl, avg_ms=avg_ms)
+    bf16_peak, peak_why = choose_bf16_peak(pk, clk)
+    fp32 = wl.dtype == torch.float32
+    nominal = None
+    if clk and clk.get("sm_mhz"):
+        nominal = 148 * MMA_FLOP_PER_CLK_SM * clk["sm_mhz"] * 1e6 / 1e12
+
+    def roofline(name):
+        nl, tot_ms = per_kernel[name]
+        avg_ms = tot_ms / max(nl, 1)
+        flops = KERNEL_FLOPS.get(name, 0) * unit_flops
+        tflops = flops / (avg_ms / 1e3) / 1e12
+        if name in FWD_KERNELS and not fp32 and wl.wid == 2:
+            # m = 256: below the ridge (171 flop/B); judged on HBM bytes
+            nbytes = fwd_bytes(wl, T)
+            gbs = nbytes / (avg_ms / 1e3) / 1e9
+            r = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                 "frac": gbs / pk["hbm"], "peak_source": f"{pk['source']} HBM copy",
+                 "algorithmic_bytes": nbytes, "tflops": tflops,
+                 "frac_of_bf16_peak": tflops / bf16_peak}
+        elif name in TENSOR_KERNELS:
+            r = {"bound": "tensor", "achieved": tflops, "peak": bf16_peak, "unit": "TFLOP/s",
+                 "frac": tflops / bf16_peak, "peak_source": peak_why,
+                 "frac_of_sustained": tflops / pk["bf16_sustained"],
+                 "frac_of_nominal_at_clock": tflops / nominal if nominal else None}
+        else:
+            r = {"bound": "alu", "achieved": tflops, "peak": SIMT_PEAK_TFLOPS, "unit": "TFLOP/s",
+                 "frac": tflops / SIMT_PEAK_TFLOPS,
+                 "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz"}
+        t_ = traffic_for(name, wl.wid, unit_flops) if subset is None else None
+        r.update(kernel=name, traffic=t_, launches=nl, avg_ms=avg_ms,
+                 traffic_source=("ncu DRAM bytes per T*h*m*dh of a capture of this kernel "
+                                 "source, scaled to the launch" if t_ else
+                                 "null: no capture of the current kernel source"))
+        return r
+
+    credited = [k_ for k_ in per_kernel if KERNEL_FLOPS.get(k_, 0)]
+    top = max(credited or per_kernel, key=lambda k_: per_kernel[k_][1])
+    roof = roofline(top)
+    fwd_name = next((k_ for k_ in per_kernel if k_ in FWD_KERNELS), None)
+    roof_fwd = roofline(fwd_name) if fwd_name else None
     kernels = {k_: {"launches": v_[0], "ms": v_[1], "share": v_[1] / max(ms, 1e-9)}
                for k_, v_ in per_kernel.items()}
 
     # ---- end to end through host buffers ----
     # The step again, through the public API, from pinned host memory: the
     # batch is cut into E2E_CHUNKS equal groups of samples, each its own
-    # fwd + bwd call on views of the device tensors.  One stream copies chunk
+    # fwd (+ bwd) call on views of the device tensors.  One stream copies chunk
     # inputs in, one computes, one copies chunk outputs back, so the two PCIe
     # directions and the compute overlap; per-chunk events order every reuse
     # of a buffer (also from one step to the next).
     e2e = None
     if not args.no_e2e and args.e2e_steps > 0:
         o_full = o.clone()          # O of the full-batch call (the forward is deterministic)
-        hq, hk, hv, hg = (x.cpu().pin_memory() for x in (q, k, v, g))
-        ho, hdq, hdk, hdv = (torch.empty(x.shape, dtype=x.dtype).pin_memory()
-                             for x in (o, dq, dk, dv))
+        ins = [q, k, v] + ([g] if wl.backward else [])
+        outs = [o] + ([dq, dk, dv] if wl.backward else [])
+        h_in = [x.cpu().pin_memory() for x in ins]
+        h_out = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in outs]
+        token_major_in = [True, False, False, True]
+        token_major_out = [True, True, False, False]
         offs = [int(x) for x in d["offsets"]]
         chunks = []
         for (b0, b1), (t0_, t1_) in e2e_chunks(offs, E2E_CHUNKS):
@@ -396,44 +530,43 @@ def main():
                 off=torch.empty(len(coff), dtype=torch.int32, device=dev),
                 lse=torch.empty((wl.h, max(t1_ - t0_, 1)), dtype=torch.float32, device=dev),
                 wsf=pkg.workspace(pkg.fwd_workspace_bytes(cp_), dev),
-                wsb=pkg.workspace(pkg.bwd_workspace_bytes(cp_), dev),
+                wsb=pkg.workspace(pkg.bwd_workspace_bytes(cp_), dev) if wl.backward else None,
                 loaded=torch.cuda.Event(), computed=torch.cuda.Event(), sent=torch.cuda.Event()))
-        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg)) + \
+        h2d = sum(x.numel() * x.element_size() for x in h_in) + \
             sum(c_["hoff"].numel() * 4 for c_ in chunks)
-        d2h = sum(x.numel() * x.element_size() for x in (ho, hdq, hdk, hdv))
+        d2h = sum(x.numel() * x.element_size() for x in h_out)
         s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
         first = [True]
 
+        def rng(c_, tok):
+            (t0_, t1_), (b0, b1) = c_["rows"], c_["smp"]
+            return slice(t0_, t1_) if tok else slice(b0, b1)
+
         def e2e_step():
             for c_ in chunks:
-                (t0_, t1_), (b0, b1) = c_["rows"], c_["smp"]
                 with torch.cuda.stream(s_in):
                     if not first[0]:
                         s_in.wait_event(c_["computed"])       # last step's compute read them
                     c_["off"].copy_(c_["hoff"], non_blocking=True)
-                    for dst, src in ((q, hq), (g, hg)):
-                        dst[t0_:t1_].copy_(src[t0_:t1_], non_blocking=True)
-                    for dst, src in ((k, hk), (v, hv)):
-                        dst[b0:b1].copy_(src[b0:b1], non_blocking=True)
+                    for dst, src, tok in zip(ins, h_in, token_major_in):
+                        dst[rng(c_, tok)].copy_(src[rng(c_, tok)], non_blocking=True)
                     c_["loaded"].record(s_in)
             for c_ in chunks:
-                (t0_, t1_), (b0, b1) = c_["rows"], c_["smp"]
                 stream.wait_event(c_["loaded"])
                 if not first[0]:
                     stream.wait_event(c_["sent"])             # last step's outputs copied out
-                cq, cg, co, cdq = q[t0_:t1_], g[t0_:t1_], o[t0_:t1_], dq[t0_:t1_]
-                ck, cv, cdk, cdv = k[b0:b1], v[b0:b1], dk[b0:b1], dv[b0:b1]
-                cl = c_["lse"][:, :t1_ - t0_]
-                G.fwd(c_["p"], cq, c_["off"], ck, cv, o=co, lse=cl, ws=c_["wsf"], stream=stream)
-                G.bwd(c_["p"], cq, c_["off"], ck, cv, co, cl, cg, dq=cdq, dk=cdk, dv=cdv,
-                      ws=c_["wsb"], stream=stream)
+                tr, sr = rng(c_, True), rng(c_, False)
+                cl = c_["lse"][:, :c_["rows"][1] - c_["rows"][0]]
+                G.fwd(c_["p"], q[tr], c_["off"], k[sr], v[sr], o=o[tr], lse=cl, ws=c_["wsf"],
+                      stream=stream)
+                if wl.backward:
+                    G.bwd(c_["p"], q[tr], c_["off"], k[sr], v[sr], o[tr], cl, g[tr], dq=dq[tr],
+                          dk=dk[sr], dv=dv[sr], ws=c_["wsb"], stream=stream)
                 c_["computed"].record(stream)
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(c_["computed"])
-                    for dst, src in ((ho, o), (hdq, dq)):
-                        dst[t0_:t1_].copy_(src[t0_:t1_], non_blocking=True)
-                    for dst, src in ((hdk, dk), (hdv, dv)):
-                        dst[b0:b1].copy_(src[b0:b1], non_blocking=True)
+                    for dst, src, tok in zip(h_out, outs, token_major_out):
+                        dst[rng(c_, tok)].copy_(src[rng(c_, tok)], non_blocking=True)
                     c_["sent"].record(s_out)
             first[0] = False
 
@@ -451,48 +584,57 @@ def main():
         torch.cuda.synchronize()
         wall = time.perf_counter() - t0
         barrier()
-        bad = [pkg.workspace_status(c_["wsf"]) or pkg.workspace_status(c_["wsb"]) for c_ in chunks]
+        bad = [pkg.workspace_status(c_["wsf"]) or
+               (wl.backward and pkg.workspace_status(c_["wsb"])) for c_ in chunks]
         if any(bad):
             raise RuntimeError("device-side status error in the end-to-end steps")
-        if not torch.equal(ho, o_full.cpu()):
+        if not torch.equal(h_out[0], o_full.cpu()):
             raise RuntimeError("end-to-end O differs from the full-batch O")
-        ea = aggregate(e0.elapsed_time(e1), (FLOPS_FWD + FLOPS_BWD) * unit_flops * args.e2e_steps,
-                       0.0, 0.0, world, dist, dev)
+        ea = aggregate(e0.elapsed_time(e1),
+                       step_flop_units(wl) * unit_flops * args.e2e_steps, 0.0, 0.0, world, dist,
+                       dev)
         ems = ea["ms_max"]
         e2e = {"value": ea["tflops"], "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "steps": args.e2e_steps, "ms_per_step": ems / args.e2e_steps,
                "wall_ms_per_step": 1e3 * wall / args.e2e_steps,
-               "api": (f"recsys_context_personalised_b200.gdpa fwd/bwd on {len(chunks)} sample "
-                       "chunks copied from and to pinned host memory; copy-in, compute and "
-                       "copy-out on three streams")}
-        del hq, hk, hv, hg, ho, hdq, hdk, hdv, chunks, o_full
+               "api": (f"recsys_context_personalised_b200.gdpa fwd"
+                       f"{'/bwd' if wl.backward else ''} on {len(chunks)} sample chunks copied "
+                       "from and to pinned host memory; copy-in, compute and copy-out on three "
+                       "streams")}
+        del h_in, h_out, chunks, o_full
 
     # ---- CPU oracle baseline (rank 0 at N=1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        samples, threads = time_oracle(wl, syn.lengths(wl), args.cpu_seconds)
-        f, dt, tk = run_oracle_sample(wl, samples)
-        cpu = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": f"{len(samples)} of {wl.B} samples ({tk} tokens, all {wl.h} heads), "
-                         f"fwd+bwd, seeded choice, {dt:.1f} s"}
+        import oracle
+        samples = oracle_sample(wl, syn.lengths(wl))
+        inputs = oracle_inputs(wl, samples)
+        f = dt = 0.0
+        tk = 0
+        for _ in range(max(args.cpu_passes, 1)):
+            f_, dt_, tk = run_oracle_sample(wl, inputs)
+            f += f_
+            dt += dt_
+        cpu = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+               "kind": "oracle",
+               "sample": oracle_desc(wl, samples, tk) + f", {args.cpu_passes} passes, "
+                                                       f"{dt:.1f} s"}
 
     if rank == 0:
-        emit({"metric": "GDPA fwd+bwd TFLOP/s", "value": value, "unit": "TFLOP/s",
+        emit({"metric": metric_name(wl), "value": value, "unit": "TFLOP/s",
               "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
               "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
-              "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-              "config": {"workload": wl.name if subset is None else
-                         f"{wl.name} (first {len(subset)} samples only: profiling case)",
-                         "B": wl.B if subset is None else len(subset), "h": wl.h, "dh": wl.dh,
-                         "m": wl.m, "phi": wl.phi_name, "scale": wl.scale, "lengths": wl.lengths,
-                         "tokens_per_rank": T, "parallelism": f"replicas x{world} (samples independent)",
-                         "l2": "inputs (K, V 4.3 GB each) far larger than the 126 MB L2; no flush"},
-              "pct_of_bf16_peak": 100.0 * value / (world * pk["bf16_sustained"]),
+              "vs_baseline": None, "dtype": "f32" if fp32 else "bf16", "data": "synthetic",
+              "config": config_dict(wl, T, world, subset),
+              "pct_of_bf16_peak": None if fp32 else 100.0 * value / (world * bf16_peak),
+              "bf16_peak": None if fp32 else {"value": bf16_peak, "source": peak_why,
+                                              "nominal_at_median_clock": nominal},
               "tokens_per_s": agg["tokens_per_s"],
-              "fwd_flops_per_step": FLOPS_FWD * unit_flops, "bwd_flops_per_step": FLOPS_BWD * unit_flops,
+              "fwd_flops_per_step": FLOPS_FWD * unit_flops,
+              "bwd_flops_per_step": FLOPS_BWD * unit_flops if wl.backward else 0.0,
               "gpu_launches": n_launch, "kernels": kernels, "roofline": roof,
-              "cpu_baseline": cpu, "e2e": e2e, "clocks": clk})
+              "roofline_fwd": roof_fwd, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk})
     if world > 1:
         dist.destroy_process_group()
 

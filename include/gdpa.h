@@ -16,9 +16,10 @@
  *
  *     S = scale * Q_bj K_bj^T,    P = phi(S),    O_bj = P V_bj
  *
- * with phi = identity, SiLU (x * logistic(x)) or a row softmax, and its
- * gradient.  Heads and samples are independent; there is no normalisation
- * for the elementwise phi, no bias and no head mixing.
+ * with phi = identity, SiLU (x * logistic(x)), a row softmax, ReLU or GELU
+ * (the PFFN variants' other activations), and its gradient.  Heads and
+ * samples are independent; there is no normalisation for the elementwise phi,
+ * no bias and no head mixing.
  *
  * Layouts (row-major, contiguous, every base pointer 16-byte aligned):
  *   q, o, dout, dq : [T, h, dh]      jagged tokens, T = offsets[B]
@@ -196,11 +197,21 @@ GDPA_API gdpa_status_t gdpa_selftest_wait_timeout(void* workspace, size_t worksp
  *   routine.  All calls share the one array, so calls that overlap on the GPU
  *   (different streams, or different host threads, without ordering between
  *   them) race on it and must be serialised by the caller.  The device status
- *   of the last call is not readable through gdpa_workspace_status.
+ *   of the last call is read with gdpa_fwd_no_alloc_status, not with
+ *   gdpa_workspace_status.
  */
 GDPA_API gdpa_status_t gdpa_fwd_no_alloc(const gdpa_problem_t* p, const void* q,
                                          const int32_t* offsets, const void* k, const void* v,
                                          void* o, float* lse, void* stream);
+
+/*
+ * Device-detected status (GDPA_OK, GDPA_ERR_INVALID_ARG for inconsistent
+ * device offsets, GDPA_ERR_TIMEOUT) of the last gdpa_fwd_no_alloc call on the
+ * current device, read from the header of its static scratch.  Copies four
+ * bytes on `stream`, synchronises it, and writes the code to *status (host).
+ * Allocates nothing.  The Kunlun pages have no counterpart of this call.
+ */
+GDPA_API gdpa_status_t gdpa_fwd_no_alloc_status(void* stream, int32_t* status);
 
 #ifdef __cplusplus
 }

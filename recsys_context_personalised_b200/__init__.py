@@ -3,7 +3,7 @@
 GDPA is the Kunlun recommendation model's Personalized FFN recast as a
 multi-head attention operator: jagged user-history tokens are the queries,
 per-sample context-generated weights are the keys and values, and
-O = phi(s Q K^T) V with phi in {identity, SiLU, softmax}.  The compute runs in
+O = phi(s Q K^T) V with phi in {identity, SiLU, softmax, ReLU, GELU}.  The compute runs in
 libgdpa.so (CUDA C++ for sm_100a behind a C ABI, ``include/gdpa.h``);
 ``gdpa`` is its ctypes binding.
 """

@@ -47,10 +47,9 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         for log in ex.map(run, jobs):
             if verbose and log.strip():
                 print(log)
-    # drop objects of sources that no longer exist
     if force or jobs or _stale(OUT, objs):
-        run([NVCC, *ARCH, "-shared", "-o", OUT, *objs, "-lcuda" if False else "-lcudart_static",
-             "-ldl", "-lrt", "-lpthread"])
+        run([NVCC, *ARCH, "-shared", "-o", OUT, *objs, "-lcudart_static", "-ldl", "-lrt",
+             "-lpthread"])
     return OUT
 
 

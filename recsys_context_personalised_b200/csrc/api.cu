@@ -50,8 +50,6 @@ cudaError_t launch_sm100_bwd(const gdpa_problem_t& p, const void* q, const int32
                              const void* dout, void* dq, void* dk, void* dv, float* dq_acc,
                              float* dsum, WsHeader* ws, Tile* tiles, cudaStream_t st);
 int64_t sm100_bwd_items(const gdpa_problem_t& p);
-bool sm100_fwd_available();
-bool sm100_bwd_available();
 
 namespace {
 
@@ -83,12 +81,10 @@ gdpa_status_t check_problem(const gdpa_problem_t* p) {
   return GDPA_OK;
 }
 
-int fwd_bm(const gdpa_problem_t& p) {
-  return (p.dtype == GDPA_DTYPE_BF16 && sm100_fwd_available()) ? kMmaBM : kSimtBM;
-}
-int bwd_bm(const gdpa_problem_t& p) {
-  return (p.dtype == GDPA_DTYPE_BF16 && sm100_bwd_available()) ? kMmaBM : kSimtBM;
-}
+// One backend per element type: bf16 runs on the tcgen05 kernels (128-row
+// tiles), fp32 on the exact SIMT kernels (64-row tiles).
+int fwd_bm(const gdpa_problem_t& p) { return p.dtype == GDPA_DTYPE_BF16 ? kMmaBM : kSimtBM; }
+int bwd_bm(const gdpa_problem_t& p) { return p.dtype == GDPA_DTYPE_BF16 ? kMmaBM : kSimtBM; }
 
 FwdLayout fwd_layout(const gdpa_problem_t& p) {
   FwdLayout L;

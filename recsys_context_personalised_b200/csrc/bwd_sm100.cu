@@ -1339,8 +1339,6 @@ cudaError_t launch_bwd_dh(const gdpa_problem_t& p, const void* q, const int32_t*
 
 }  // namespace
 
-bool sm100_bwd_available() { return true; }
-
 int64_t sm100_bwd_items(const gdpa_problem_t& p) {
   return (int64_t)p.B * p.h * ((p.m + 127) / 128);
 }

@@ -57,3 +57,17 @@ extern "C" gdpa_status_t gdpa_fwd_no_alloc(const gdpa_problem_t* p, const void* 
   // rewrites the header and the tile list at the start of every call.
   return gdpa_fwd(p, q, offsets, k, v, o, lse, scratch, gdpa::kFwdScratchBytes, stream);
 }
+
+// Device-detected status of the last gdpa_fwd_no_alloc call on the current
+// device (the header's status word in the static scratch): GDPA_OK, or
+// GDPA_ERR_INVALID_ARG for inconsistent device offsets, or GDPA_ERR_TIMEOUT.
+// Copies four bytes on `stream` and synchronises it; allocates nothing.
+extern "C" gdpa_status_t gdpa_fwd_no_alloc_status(void* stream, int32_t* status) {
+  if (!status) return GDPA_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= gdpa::kMaxDevices)
+    return GDPA_ERR_CUDA;
+  void* scratch = gdpa::scratch_address(dev);
+  if (!scratch) return GDPA_ERR_CUDA;
+  return gdpa_workspace_status(scratch, stream, status);
+}

@@ -666,8 +666,6 @@ cudaError_t launch_fwd_dh(const gdpa_problem_t& p, const void* q, const void* k,
 
 }  // namespace
 
-bool sm100_fwd_available() { return true; }
-
 cudaError_t launch_sm100_fwd(const gdpa_problem_t& p, const void* q, const void* k,
                              const void* v, void* o, float* lse, WsHeader* ws, const Tile* tiles,
                              cudaStream_t st) {

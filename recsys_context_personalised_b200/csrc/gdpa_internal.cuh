@@ -61,7 +61,7 @@ cudaError_t launch_schedule(const gdpa_problem_t& p, const int32_t* offsets, int
 cudaError_t launch_schedule_kv(const gdpa_problem_t& p, const int32_t* offsets, WsHeader* ws,
                                Tile* tiles, cudaStream_t st);
 
-// SIMT kernels (fp32 or bf16 elements; fp32 math).
+// SIMT kernels (fp32 problems only; fp32 math).
 cudaError_t launch_simt_fwd(const gdpa_problem_t& p, const void* q, const void* k,
                             const void* v, void* o, float* lse, WsHeader* ws,
                             const Tile* tiles, int64_t tile_cap, cudaStream_t st);

@@ -1,9 +1,11 @@
-// SIMT (CUDA-core FFMA) GDPA kernels: the exact-fp32 path, used for fp32
-// problems, where tensor-core formats are too coarse for fp32 parity.
+// SIMT (CUDA-core FFMA) GDPA kernels: the exact-fp32 path, the only path of
+// fp32 problems (tensor-core formats are too coarse for fp32 parity); bf16
+// problems run on the tcgen05 kernels only.
 //
 // Operator (Kunlun summary, section 2.2, GDPA bullet; RecSysChannel review
 // "Kunlun ... [2/2]", items 1-2): per sample b and head j,
-//   S = s Q K^T, P = phi(S), O = P V, with phi in {identity, SiLU, softmax};
+//   S = s Q K^T, P = phi(S), O = P V, with phi in {identity, SiLU, softmax,
+//   ReLU, GELU};
 // backward: dV = P^T dO, dP = dO V^T, dS = dP * phi'(S) (softmax:
 // P * (dP - D), D = rowsum(dO * O)), dQ = s dS K, dK = s dS^T Q.
 //
@@ -429,11 +431,8 @@ cudaError_t dkdv_t(const gdpa_problem_t& p, const void* q, const int32_t* offset
   }
 
 template <int DH> cudaError_t fwd_f32(const gdpa_problem_t& p, const void* q, const void* k, const void* v, void* o, float* lse, WsHeader* ws, const Tile* t, int64_t cap, cudaStream_t st) { return fwd_t<float, DH>(p, q, k, v, o, lse, ws, t, cap, st); }
-template <int DH> cudaError_t fwd_bf16(const gdpa_problem_t& p, const void* q, const void* k, const void* v, void* o, float* lse, WsHeader* ws, const Tile* t, int64_t cap, cudaStream_t st) { return fwd_t<__nv_bfloat16, DH>(p, q, k, v, o, lse, ws, t, cap, st); }
 template <int DH> cudaError_t dq_f32(const gdpa_problem_t& p, const void* q, const void* k, const void* v, const float* l, const float* ds, const void* g, void* dq, WsHeader* ws, const Tile* t, int64_t cap, cudaStream_t st) { return dq_t<float, DH>(p, q, k, v, l, ds, g, dq, ws, t, cap, st); }
-template <int DH> cudaError_t dq_bf16(const gdpa_problem_t& p, const void* q, const void* k, const void* v, const float* l, const float* ds, const void* g, void* dq, WsHeader* ws, const Tile* t, int64_t cap, cudaStream_t st) { return dq_t<__nv_bfloat16, DH>(p, q, k, v, l, ds, g, dq, ws, t, cap, st); }
 template <int DH> cudaError_t dkdv_f32(const gdpa_problem_t& p, const void* q, const int32_t* off, const void* k, const void* v, const float* l, const float* ds, const void* g, void* dk, void* dv, WsHeader* ws, cudaStream_t st) { return dkdv_t<float, DH>(p, q, off, k, v, l, ds, g, dk, dv, ws, st); }
-template <int DH> cudaError_t dkdv_bf16(const gdpa_problem_t& p, const void* q, const int32_t* off, const void* k, const void* v, const float* l, const float* ds, const void* g, void* dk, void* dv, WsHeader* ws, cudaStream_t st) { return dkdv_t<__nv_bfloat16, DH>(p, q, off, k, v, l, ds, g, dk, dv, ws, st); }
 
 }  // namespace
 
@@ -441,8 +440,8 @@ cudaError_t launch_simt_fwd(const gdpa_problem_t& p, const void* q, const void* 
                             void* o, float* lse, WsHeader* ws, const Tile* tiles, int64_t cap,
                             cudaStream_t st) {
   if (cap <= 0) return cudaSuccess;
-  if (p.dtype == GDPA_DTYPE_F32) { GDPA_DISPATCH_DH(p.dh, fwd_f32, p, q, k, v, o, lse, ws, tiles, cap, st); }
-  GDPA_DISPATCH_DH(p.dh, fwd_bf16, p, q, k, v, o, lse, ws, tiles, cap, st);
+  if (p.dtype != GDPA_DTYPE_F32) return cudaErrorInvalidValue;
+  GDPA_DISPATCH_DH(p.dh, fwd_f32, p, q, k, v, o, lse, ws, tiles, cap, st);
 }
 
 cudaError_t launch_row_dot(const gdpa_problem_t& p, const void* o, const void* g, float* dsum,
@@ -452,13 +451,10 @@ cudaError_t launch_row_dot(const gdpa_problem_t& p, const void* o, const void* g
   const int threads = 256;
   int64_t blocks = (rows * 32 + threads - 1) / threads;
   if (blocks > 148 * 64) blocks = 148 * 64;
+  if (p.dtype != GDPA_DTYPE_F32) return cudaErrorInvalidValue;
   KernelScope ks_("gdpa_row_dot", st);
-  if (p.dtype == GDPA_DTYPE_F32)
-    row_dot_kernel<float><<<(unsigned)blocks, threads, 0, st>>>((const float*)o, (const float*)g,
-                                                                dsum, rows, p.h, p.dh, p.total_tokens);
-  else
-    row_dot_kernel<__nv_bfloat16><<<(unsigned)blocks, threads, 0, st>>>(
-        (const __nv_bfloat16*)o, (const __nv_bfloat16*)g, dsum, rows, p.h, p.dh, p.total_tokens);
+  row_dot_kernel<float><<<(unsigned)blocks, threads, 0, st>>>((const float*)o, (const float*)g,
+                                                              dsum, rows, p.h, p.dh, p.total_tokens);
   return cudaGetLastError();
 }
 
@@ -467,16 +463,16 @@ cudaError_t launch_simt_bwd_dq(const gdpa_problem_t& p, const void* q, const voi
                                const void* g, void* dq, WsHeader* ws, const Tile* tiles,
                                int64_t cap, cudaStream_t st) {
   if (cap <= 0) return cudaSuccess;
-  if (p.dtype == GDPA_DTYPE_F32) { GDPA_DISPATCH_DH(p.dh, dq_f32, p, q, k, v, lse, dsum, g, dq, ws, tiles, cap, st); }
-  GDPA_DISPATCH_DH(p.dh, dq_bf16, p, q, k, v, lse, dsum, g, dq, ws, tiles, cap, st);
+  if (p.dtype != GDPA_DTYPE_F32) return cudaErrorInvalidValue;
+  GDPA_DISPATCH_DH(p.dh, dq_f32, p, q, k, v, lse, dsum, g, dq, ws, tiles, cap, st);
 }
 
 cudaError_t launch_simt_bwd_dkdv(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
                                  const void* k, const void* v, const float* lse,
                                  const float* dsum, const void* g, void* dk, void* dv,
                                  WsHeader* ws, cudaStream_t st) {
-  if (p.dtype == GDPA_DTYPE_F32) { GDPA_DISPATCH_DH(p.dh, dkdv_f32, p, q, offsets, k, v, lse, dsum, g, dk, dv, ws, st); }
-  GDPA_DISPATCH_DH(p.dh, dkdv_bf16, p, q, offsets, k, v, lse, dsum, g, dk, dv, ws, st);
+  if (p.dtype != GDPA_DTYPE_F32) return cudaErrorInvalidValue;
+  GDPA_DISPATCH_DH(p.dh, dkdv_f32, p, q, offsets, k, v, lse, dsum, g, dk, dv, ws, st);
 }
 
 }  // namespace gdpa

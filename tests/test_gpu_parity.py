@@ -174,21 +174,50 @@ def check_single_key_softmax(out, d, scale, tol):
     assert np.abs(out["dk"].float().cpu().numpy()).max(initial=0.0) <= tol * scale * dp * qmax
 
 
-def test_outputs_untouched_outside_rows():
-    """Guard region: rows of o beyond T and the lse tail stay as they were."""
-    n, m, dh = [129, 3], 70, 64
-    d = syn.random_problem(7, 2, 2, dh, m, n, dtype=torch.bfloat16)
-    q, k, v = (d[x].to(DEV) for x in ("q", "k", "v"))
+@pytest.mark.parametrize("dh", [64, 128])
+@pytest.mark.parametrize("phi", ["softmax", "silu"])
+def test_outputs_untouched_outside_their_ranges(phi, dh):
+    """Guard regions around every output of the forward and the backward.
+
+    o, lse and dq sit 64 rows (lse: 64 values) into larger sentinel-filled
+    buffers, dk and dv one sample in, and the workspaces are 4 KB longer than
+    asked for.  Ragged lengths and m = 70 (not a multiple of the 128-key
+    block) put partial tiles at both ends.  Every sentinel before and after
+    each output must be untouched, and the outputs inside must still match
+    the oracle.
+    """
+    n, m, h = [129, 3, 0, 200], 70, 2
+    B = len(n)
+    d = syn.random_problem(7, B, h, dh, m, n, dtype=torch.bfloat16, std=0.6)
+    q, k, v, g = (d[x].to(DEV) for x in ("q", "k", "v", "dout"))
     off = torch.tensor(d["offsets"], dtype=torch.int32, device=DEV)
     T = int(d["offsets"][-1])
-    big = torch.full((T + 64, 2, dh), 7.0, dtype=torch.bfloat16, device=DEV)
-    o = big[:T]
-    p = pkg.problem_for(q, k, d["offsets"], "softmax", 0.125)
-    lse_big = torch.full((2, T + 64), 3.0, device=DEV)
-    pkg.fwd(p, q, off, k, v, o=o, lse=None)
+    scale = 1.0 / dh ** 0.5 if phi == "softmax" else 0.5
+    p = pkg.problem_for(q, k, d["offsets"], phi, scale)
+    bf = torch.bfloat16
+    o_big = torch.full((T + 128, h, dh), 7.0, dtype=bf, device=DEV)
+    dq_big = torch.full((T + 128, h, dh), 5.0, dtype=bf, device=DEV)
+    dk_big = torch.full((B + 2, h, m, dh), 9.0, dtype=bf, device=DEV)
+    dv_big = torch.full((B + 2, h, m, dh), 11.0, dtype=bf, device=DEV)
+    lse_big = torch.full((h * T + 128,), 3.0, dtype=torch.float32, device=DEV)
+    o, dq = o_big[64:64 + T], dq_big[64:64 + T]
+    dk, dv = dk_big[1:B + 1], dv_big[1:B + 1]
+    lse = lse_big[64:64 + h * T].view(h, T)
+    nf, nb = pkg.fwd_workspace_bytes(p), pkg.bwd_workspace_bytes(p)
+    wsf = torch.full((nf + 4096,), 0xAB, dtype=torch.uint8, device=DEV)
+    wsb = torch.full((nb + 4096,), 0xAB, dtype=torch.uint8, device=DEV)
+    pkg.fwd(p, q, off, k, v, o=o, lse=lse, ws=wsf)
+    pkg.bwd(p, q, off, k, v, o, lse, g, dq=dq, dk=dk, dv=dv, ws=wsb)
     torch.cuda.synchronize()
-    assert (big[T:] == 7.0).all()
-    del lse_big
+    assert pkg.workspace_status(wsf) == 0 and pkg.workspace_status(wsb) == 0
+    for name, big, lo, hi, val in (("o", o_big, 64, 64 + T, 7.0), ("dq", dq_big, 64, 64 + T, 5.0),
+                                   ("dk", dk_big, 1, B + 1, 9.0), ("dv", dv_big, 1, B + 1, 11.0),
+                                   ("lse", lse_big, 64, 64 + h * T, 3.0)):
+        assert (big[:lo] == val).all(), f"{name}: written before its range"
+        assert (big[hi:] == val).all(), f"{name}: written past its range"
+    assert (wsf[nf:] == 0xAB).all() and (wsb[nb:] == 0xAB).all(), "workspace overrun"
+    out = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+    check(out, d, phi, scale, True, torch.bfloat16, f"guarded {phi} dh={dh}")
 
 
 def test_bad_device_offsets_reported_not_crashing():
