@@ -45,6 +45,12 @@ def load(path: str = None):
     lib.gdpa_oracle_bwd.argtypes = [i32, i32, i32, i32, i64p, fp, fp, fp, fp, i32, f64,
                                     dp, dp, dp, i32]
     lib.gdpa_oracle_bwd.restype = i32
+    lib.gdpa_oracle_fwd_bias.argtypes = [i32, i32, i32, i32, i64p, fp, fp, fp, fp, fp, i32, f64,
+                                         dp, dp, i32]
+    lib.gdpa_oracle_fwd_bias.restype = i32
+    lib.gdpa_oracle_bwd_bias.argtypes = [i32, i32, i32, i32, i64p, fp, fp, fp, fp, fp, i32, f64,
+                                         dp, dp, dp, dp, dp, i32]
+    lib.gdpa_oracle_bwd_bias.restype = i32
     lib.gdpa_oracle_max_threads.restype = i32
     if path is None:
         _lib = lib
@@ -70,41 +76,70 @@ def max_threads(lib=None) -> int:
     return (lib or load()).gdpa_oracle_max_threads()
 
 
-def fwd(q, k, v, offsets, phi, scale, nthreads: int = 0, lib=None):
-    """O [T,h,dh] float64 and LSE [h,T] float64 (NaN-free only for softmax)."""
+def _opt(x, shape):
+    """Exact float32 copy of an optional bias, checked against its shape."""
+    if x is None:
+        return None
+    x = _f32(x)
+    assert x.shape == shape, (x.shape, shape)
+    return x
+
+
+def _optp(x, ct):
+    return None if x is None else _ptr(x, ct)
+
+
+def fwd(q, k, v, offsets, phi, scale, nthreads: int = 0, lib=None, b1=None, b2=None):
+    """O [T,h,dh] float64 and LSE [h,T] float64 (NaN-free only for softmax).
+
+    ``b1`` [B,h,m] and ``b2`` [B,h,dh] are the optional biases of
+    phi(s Q K^T + b1) V + b2."""
     lib = lib or load()
     q, k, v = _f32(q), _f32(k), _f32(v)
     off = np.ascontiguousarray(offsets, dtype=np.int64)
     B, h, m, dh = k.shape
     T = int(off[-1])
     assert q.shape == (T, h, dh) and v.shape == k.shape and off.shape == (B + 1,)
+    b1, b2 = _opt(b1, (B, h, m)), _opt(b2, (B, h, dh))
     o = np.zeros((T, h, dh), dtype=np.float64)
     lse = np.zeros((h, T), dtype=np.float64)
-    rc = lib.gdpa_oracle_fwd(B, h, dh, m, _ptr(off, ctypes.c_int64), _ptr(q, ctypes.c_float),
-                             _ptr(k, ctypes.c_float), _ptr(v, ctypes.c_float), _phi(phi),
-                             float(scale), _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double),
-                             int(nthreads))
+    rc = lib.gdpa_oracle_fwd_bias(B, h, dh, m, _ptr(off, ctypes.c_int64),
+                                  _ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                  _ptr(v, ctypes.c_float), _optp(b1, ctypes.c_float),
+                                  _optp(b2, ctypes.c_float), _phi(phi), float(scale),
+                                  _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double),
+                                  int(nthreads))
     if rc != 0:
         raise RuntimeError(f"gdpa_oracle_fwd failed with code {rc}")
     return o, lse
 
 
-def bwd(q, k, v, dout, offsets, phi, scale, nthreads: int = 0, lib=None):
-    """(dQ [T,h,dh], dK [B,h,m,dh], dV [B,h,m,dh]) in float64."""
+def bwd(q, k, v, dout, offsets, phi, scale, nthreads: int = 0, lib=None, b1=None,
+        bias_grads: bool = False):
+    """(dQ [T,h,dh], dK [B,h,m,dh], dV [B,h,m,dh]) in float64, and with
+    ``bias_grads`` also (dB1 [B,h,m], dB2 [B,h,dh]).  ``b1`` is the optional
+    key bias (the output bias b2 does not enter the gradients)."""
     lib = lib or load()
     q, k, v, g = _f32(q), _f32(k), _f32(v), _f32(dout)
     off = np.ascontiguousarray(offsets, dtype=np.int64)
     B, h, m, dh = k.shape
     T = int(off[-1])
     assert q.shape == (T, h, dh) and g.shape == q.shape and v.shape == k.shape
+    b1 = _opt(b1, (B, h, m))
     dq = np.zeros((T, h, dh), dtype=np.float64)
     dk = np.zeros((B, h, m, dh), dtype=np.float64)
     dv = np.zeros((B, h, m, dh), dtype=np.float64)
-    rc = lib.gdpa_oracle_bwd(B, h, dh, m, _ptr(off, ctypes.c_int64), _ptr(q, ctypes.c_float),
-                             _ptr(k, ctypes.c_float), _ptr(v, ctypes.c_float),
-                             _ptr(g, ctypes.c_float), _phi(phi), float(scale),
-                             _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double),
-                             _ptr(dv, ctypes.c_double), int(nthreads))
+    db1 = np.zeros((B, h, m), dtype=np.float64) if bias_grads else None
+    db2 = np.zeros((B, h, dh), dtype=np.float64) if bias_grads else None
+    rc = lib.gdpa_oracle_bwd_bias(B, h, dh, m, _ptr(off, ctypes.c_int64),
+                                  _ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                  _ptr(v, ctypes.c_float), _optp(b1, ctypes.c_float),
+                                  _ptr(g, ctypes.c_float), _phi(phi), float(scale),
+                                  _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double),
+                                  _ptr(dv, ctypes.c_double), _optp(db1, ctypes.c_double),
+                                  _optp(db2, ctypes.c_double), int(nthreads))
     if rc != 0:
         raise RuntimeError(f"gdpa_oracle_bwd failed with code {rc}")
+    if bias_grads:
+        return dq, dk, dv, db1, db2
     return dq, dk, dv

@@ -37,7 +37,17 @@
  * (b, j) are independent and run under OpenMP; inside a unit nothing is
  * blocked, fused or reordered.
  *
+ * Biased variant (the PFFN with biases, phi(s Q K^T + b1) V + b2; the pages
+ * leave the PFFN's biases open, this is reading R19): per sample and head a
+ * key bias b1^ = b1[b, j] (m) added to every row of the scaled logits before
+ * phi, and an output bias b2^ = b2[b, j] (dh) added to every row of O:
+ *
+ *   S  = s * Q^ K^T + 1 b1^T,   O = phi(S) V^ + 1 b2^T,
+ *   db1^ = sum_i dS_i.,  db2^ = sum_i dO^_i.   (the other gradients unchanged
+ *                                               in form, with this S)
+ *
  * Layouts: q, o, dout, dq: [T, h, dh];  k, v, dk, dv: [B, h, m, dh];
+ * b1, db1: [B, h, m];  b2, db2: [B, h, dh];
  * offsets: int64 [B+1];  lse: [h, T].  phi: 0 identity, 1 SiLU, 2 softmax,
  * 3 ReLU, 4 GELU.  ReLU and GELU are the "other phi" of the PFFN variants the
  * Kunlun pages leave open; GELU is taken in its exact form x Phi(x) (reading:
@@ -63,16 +73,17 @@ static double normal_pdf(double x) { return 0.39894228040143267794 * exp(-0.5 * 
 
 static double logistic(double x) { return 1.0 / (1.0 + exp(-x)); }
 
-/* S = s Q^ K^T for one unit; S is n x m, row-major. */
+/* S = s Q^ K^T (+ b1^ on every row when b1b is not NULL) for one unit; S is
+ * n x m, row-major. */
 static void logits(int n, int m, int dh, int h, const float* qb, const float* kb,
-                   double scale, double* S) {
+                   const float* b1b, double scale, double* S) {
   for (int i = 0; i < n; ++i) {
     const float* qi = qb + (size_t)i * h * dh;
     for (int k = 0; k < m; ++k) {
       const float* kk = kb + (size_t)k * dh;
       double acc = 0.0;
       for (int d = 0; d < dh; ++d) acc += (double)qi[d] * (double)kk[d];
-      S[(size_t)i * m + k] = scale * acc;
+      S[(size_t)i * m + k] = scale * acc + (b1b ? (double)b1b[k] : 0.0);
     }
   }
 }
@@ -109,11 +120,13 @@ static int valid_args(int B, int h, int dh, int m, const int64_t* offsets) {
   return 1;
 }
 
-/* Forward.  o: [T,h,dh] (required), lse: [h,T] (softmax only; may be NULL).
+/* Forward.  o: [T,h,dh] (required), lse: [h,T] (softmax only; may be NULL);
+ * b1 [B,h,m] and b2 [B,h,dh] may be NULL (no bias).
  * Returns 0 on success, -1 on bad arguments, -2 if memory ran out. */
-int gdpa_oracle_fwd(int B, int h, int dh, int m, const int64_t* offsets,
-                    const float* q, const float* k, const float* v, int phi,
-                    double scale, double* o, double* lse, int nthreads) {
+int gdpa_oracle_fwd_bias(int B, int h, int dh, int m, const int64_t* offsets,
+                         const float* q, const float* k, const float* v, const float* b1,
+                         const float* b2, int phi, double scale, double* o, double* lse,
+                         int nthreads) {
   if (!valid_args(B, h, dh, m, offsets) || phi < 0 || phi > 4 || !q || !k || !v || !o)
     return -1;
   const int64_t T = offsets[B];
@@ -138,14 +151,16 @@ int gdpa_oracle_fwd(int B, int h, int dh, int m, const int64_t* offsets,
     const float* qb = q + ((size_t)t0 * h + j) * dh;
     const float* kb = k + ((size_t)b * h + j) * (size_t)m * dh;
     const float* vb = v + ((size_t)b * h + j) * (size_t)m * dh;
-    logits(n, m, dh, h, qb, kb, scale, S);
+    const float* b1b = b1 ? b1 + ((size_t)b * h + j) * (size_t)m : NULL;
+    const float* b2b = b2 ? b2 + ((size_t)b * h + j) * (size_t)dh : NULL;
+    logits(n, m, dh, h, qb, kb, b1b, scale, S);
     activation(n, m, phi, S, P, L);
     for (int i = 0; i < n; ++i) {
       double* oi = o + ((size_t)(t0 + i) * h + j) * dh;
       for (int d = 0; d < dh; ++d) {
         double acc = 0.0;
         for (int kk = 0; kk < m; ++kk) acc += P[(size_t)i * m + kk] * (double)vb[(size_t)kk * dh + d];
-        oi[d] = acc;
+        oi[d] = acc + (b2b ? (double)b2b[d] : 0.0);
       }
       if (lse && phi == PHI_SOFTMAX) lse[(size_t)j * T + t0 + i] = L[i];
     }
@@ -155,11 +170,13 @@ int gdpa_oracle_fwd(int B, int h, int dh, int m, const int64_t* offsets,
 }
 
 /* Backward.  dout: [T,h,dh]; dq: [T,h,dh]; dk, dv: [B,h,m,dh] (all required).
+ * b1 [B,h,m] may be NULL (no key bias; b2 does not enter the gradients);
+ * db1 [B,h,m] and db2 [B,h,dh] are written when not NULL.
  * P is recomputed from its definition; no forward state is taken. */
-int gdpa_oracle_bwd(int B, int h, int dh, int m, const int64_t* offsets,
-                    const float* q, const float* k, const float* v, const float* dout,
-                    int phi, double scale, double* dq, double* dk, double* dv,
-                    int nthreads) {
+int gdpa_oracle_bwd_bias(int B, int h, int dh, int m, const int64_t* offsets,
+                         const float* q, const float* k, const float* v, const float* b1,
+                         const float* dout, int phi, double scale, double* dq, double* dk,
+                         double* dv, double* db1, double* db2, int nthreads) {
   if (!valid_args(B, h, dh, m, offsets) || phi < 0 || phi > 4 || !q || !k || !v ||
       !dout || !dq || !dk || !dv)
     return -1;
@@ -178,9 +195,21 @@ int gdpa_oracle_bwd(int B, int h, int dh, int m, const int64_t* offsets,
     const float* gb = dout + ((size_t)t0 * h + j) * dh;
     double* dkb = dk + ((size_t)b * h + j) * (size_t)m * dh;
     double* dvb = dv + ((size_t)b * h + j) * (size_t)m * dh;
+    const float* b1b = b1 ? b1 + ((size_t)b * h + j) * (size_t)m : NULL;
+    double* db1b = db1 ? db1 + ((size_t)b * h + j) * (size_t)m : NULL;
+    double* db2b = db2 ? db2 + ((size_t)b * h + j) * (size_t)dh : NULL;
     memset(dkb, 0, sizeof(double) * (size_t)m * dh);
     memset(dvb, 0, sizeof(double) * (size_t)m * dh);
+    if (db1b) memset(db1b, 0, sizeof(double) * (size_t)m);
+    if (db2b) memset(db2b, 0, sizeof(double) * (size_t)dh);
     if (n == 0) continue;
+    /* db2^ = sum_i dO^_i. */
+    if (db2b)
+      for (int d = 0; d < dh; ++d) {
+        double acc = 0.0;
+        for (int i = 0; i < n; ++i) acc += (double)gb[(size_t)i * h * dh + d];
+        db2b[d] = acc;
+      }
     double* S = (double*)malloc(sizeof(double) * (size_t)n * m);
     double* P = (double*)malloc(sizeof(double) * (size_t)n * m);
     double* dP = (double*)malloc(sizeof(double) * (size_t)n * m);
@@ -189,7 +218,7 @@ int gdpa_oracle_bwd(int B, int h, int dh, int m, const int64_t* offsets,
       failed |= 1;
       continue;
     }
-    logits(n, m, dh, h, qb, kb, scale, S);
+    logits(n, m, dh, h, qb, kb, b1b, scale, S);
     activation(n, m, phi, S, P, NULL);
     /* dP = dO^ V^T */
     for (int i = 0; i < n; ++i)
@@ -227,6 +256,13 @@ int gdpa_oracle_bwd(int B, int h, int dh, int m, const int64_t* offsets,
         for (int kk = 0; kk < m; ++kk) dpi[kk] = pi[kk] * (dpi[kk] - D);
       }
     }
+    /* db1^ = sum_i dS_i. */
+    if (db1b)
+      for (int kk = 0; kk < m; ++kk) {
+        double acc = 0.0;
+        for (int i = 0; i < n; ++i) acc += dP[(size_t)i * m + kk];
+        db1b[kk] = acc;
+      }
     /* dQ^ = s dS K^ */
     for (int i = 0; i < n; ++i) {
       double* dqi = dq + ((size_t)(t0 + i) * h + j) * dh;
@@ -246,6 +282,21 @@ int gdpa_oracle_bwd(int B, int h, int dh, int m, const int64_t* offsets,
     free(S); free(P); free(dP);
   }
   return failed ? -2 : 0;
+}
+
+/* The operator without biases. */
+int gdpa_oracle_fwd(int B, int h, int dh, int m, const int64_t* offsets, const float* q,
+                    const float* k, const float* v, int phi, double scale, double* o,
+                    double* lse, int nthreads) {
+  return gdpa_oracle_fwd_bias(B, h, dh, m, offsets, q, k, v, NULL, NULL, phi, scale, o, lse,
+                              nthreads);
+}
+
+int gdpa_oracle_bwd(int B, int h, int dh, int m, const int64_t* offsets, const float* q,
+                    const float* k, const float* v, const float* dout, int phi, double scale,
+                    double* dq, double* dk, double* dv, int nthreads) {
+  return gdpa_oracle_bwd_bias(B, h, dh, m, offsets, q, k, v, NULL, dout, phi, scale, dq, dk, dv,
+                              NULL, NULL, nthreads);
 }
 
 int gdpa_oracle_max_threads(void) {

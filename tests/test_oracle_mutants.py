@@ -20,13 +20,29 @@ MUTANTS = {
     "silu_sign": ("pi[k] = si[k] / (1.0 + exp(-si[k]));", "pi[k] = si[k] / (1.0 + exp(si[k]));"),
     "softmax_no_max": ("pi[k] = exp(si[k] - mx) / sum;", "pi[k] = exp(si[k]) / sum;"),
     "lse_no_max": ("lse_rows[i] = mx + log(sum);", "lse_rows[i] = log(sum);"),
-    "logit_no_scale": ("S[(size_t)i * m + k] = scale * acc;", "S[(size_t)i * m + k] = acc;"),
+    "logit_no_scale": ("S[(size_t)i * m + k] = scale * acc + (b1b ? (double)b1b[k] : 0.0);",
+                       "S[(size_t)i * m + k] = acc + (b1b ? (double)b1b[k] : 0.0);"),
     "logit_k_transposed": ("acc += (double)qi[d] * (double)kk[d];",
                            "acc += (double)qi[d] * (double)kb[(size_t)d * m + k];"),
     "pv_v_transposed": ("acc += P[(size_t)i * m + kk] * (double)vb[(size_t)kk * dh + d];",
                         "acc += P[(size_t)i * m + kk] * (double)vb[(size_t)d * m + kk];"),
-    "q_head_offset": ("const float* qb = q + ((size_t)t0 * h + j) * dh;\n    const float* kb = k + ((size_t)b * h + j) * (size_t)m * dh;\n    const float* vb = v + ((size_t)b * h + j) * (size_t)m * dh;\n    logits",
-                      "const float* qb = q + ((size_t)t0 * h) * dh;\n    const float* kb = k + ((size_t)b * h + j) * (size_t)m * dh;\n    const float* vb = v + ((size_t)b * h + j) * (size_t)m * dh;\n    logits"),
+    "q_head_offset": ("const float* qb = q + ((size_t)t0 * h + j) * dh;\n    const float* kb = k + ((size_t)b * h + j) * (size_t)m * dh;\n    const float* vb = v + ((size_t)b * h + j) * (size_t)m * dh;\n    const float* b1b = b1 ? b1 + ((size_t)b * h + j) * (size_t)m : NULL;\n    const float* b2b",
+                      "const float* qb = q + ((size_t)t0 * h) * dh;\n    const float* kb = k + ((size_t)b * h + j) * (size_t)m * dh;\n    const float* vb = v + ((size_t)b * h + j) * (size_t)m * dh;\n    const float* b1b = b1 ? b1 + ((size_t)b * h + j) * (size_t)m : NULL;\n    const float* b2b"),
+    # the biased variant
+    "b1_ignored": ("S[(size_t)i * m + k] = scale * acc + (b1b ? (double)b1b[k] : 0.0);",
+                   "S[(size_t)i * m + k] = scale * acc;"),
+    "b1_per_token": ("S[(size_t)i * m + k] = scale * acc + (b1b ? (double)b1b[k] : 0.0);",
+                     "S[(size_t)i * m + k] = scale * acc + (b1b ? (double)b1b[i % m] : 0.0);"),
+    "b1_unscaled_twice": ("S[(size_t)i * m + k] = scale * acc + (b1b ? (double)b1b[k] : 0.0);",
+                          "S[(size_t)i * m + k] = scale * (acc + (b1b ? (double)b1b[k] : 0.0));"),
+    "b2_dropped": ("oi[d] = acc + (b2b ? (double)b2b[d] : 0.0);", "oi[d] = acc;"),
+    "b2_wrong_head": ("const float* b2b = b2 ? b2 + ((size_t)b * h + j) * (size_t)dh : NULL;",
+                      "const float* b2b = b2 ? b2 + ((size_t)b * h) * (size_t)dh : NULL;"),
+    "db1_sums_p": ("for (int i = 0; i < n; ++i) acc += dP[(size_t)i * m + kk];\n        db1b[kk] = acc;",
+                   "for (int i = 0; i < n; ++i) acc += P[(size_t)i * m + kk];\n        db1b[kk] = acc;"),
+    "db1_scaled": ("db1b[kk] = acc;", "db1b[kk] = scale * acc;"),
+    "db2_row_stride": ("for (int i = 0; i < n; ++i) acc += (double)gb[(size_t)i * h * dh + d];",
+                       "for (int i = 0; i < n; ++i) acc += (double)gb[(size_t)i * dh + d];"),
     "silu_grad_term": ("dpi[kk] = dpi[kk] * sg * (1.0 + si[kk] * (1.0 - sg));",
                        "dpi[kk] = dpi[kk] * sg * (1.0 + si[kk] * sg);"),
     "softmax_grad_sign": ("dpi[kk] = pi[kk] * (dpi[kk] - D);", "dpi[kk] = pi[kk] * (dpi[kk] + D);"),
@@ -56,6 +72,11 @@ PIN_CALLS = (
     + [(pins.test_relu_gelu_closed_forms, ())]
     + [(pins.test_matches_library_routines, (phi,)) for phi in ("relu", "gelu")]
     + [(pins.test_backward_matches_torch_autograd, (phi,)) for phi in ("relu", "gelu")]
+    + [(pins.test_bias_hand_derived_golden, (phi,)) for phi in pins.PHIS]
+    + [(pins.test_key_bias_is_an_extra_head_dim_column, (phi,)) for phi in ("silu", "softmax")]
+    + [(pins.test_output_bias_shifts_o_and_its_gradient_is_the_token_sum, ("silu",))]
+    + [(pins.test_softmax_key_bias_shift_invariance, ())]
+    + [(pins.test_biased_operator_matches_torch_autograd, (phi,)) for phi in ("silu", "softmax")]
 )
 
 

@@ -360,3 +360,176 @@ def test_backward_matches_torch_autograd(phi):
     assert _rel(dq, q.grad.numpy()) < 1e-12
     assert _rel(dk, k.grad.numpy()) < 1e-12
     assert _rel(dv, v.grad.numpy()) < 1e-12
+
+
+# --------------------------------------------------------------------------
+# the biased variant phi(s Q K^T + b1) V + b2 (reading R19)
+
+
+def _biases(seed, B, h, m, dh, scale=1.0):
+    rng = np.random.default_rng(seed)
+    b1 = (rng.standard_normal((B, h, m)) * scale).astype(np.float32)
+    b2 = (rng.standard_normal((B, h, dh)) * scale).astype(np.float32)
+    return b1, b2
+
+
+@pytest.mark.parametrize("phi", PHIS)
+def test_bias_hand_derived_golden(phi):
+    g = json.load(open(os.path.join(HERE, "golden", "gdpa_bias_hand_derived.json")))
+    inp = g["inputs"]
+    ev = lambda e: eval(e, {"log": math.log})    # noqa: E731
+    q, k, v, dout = (np.array(inp[x], np.float32) for x in ("q", "k", "v", "dout"))
+    b1 = np.array([[[ev(e) for e in row] for row in blk] for blk in inp["b1"]], np.float32)
+    b2 = np.array([[[ev(e) for e in row] for row in blk] for blk in inp["b2"]], np.float32)
+    off = np.array(inp["offsets"], np.int64)
+    scale = float(np.float32(ev(inp["scale"])))
+    # the exact inputs are fp32 roundings of ln3; the derivation uses ln3 itself
+    want = {key: np.array([ev(e) for e in vals]) for key, vals in g["cases"][phi].items()}
+    o, lse = oracle.fwd(q, k, v, off, phi, scale, b1=b1, b2=b2)
+    dq, dk, dv, db1, db2 = oracle.bwd(q, k, v, dout, off, phi, scale, b1=b1, bias_grads=True)
+    got = {"o": o, "dq": dq, "dk": dk, "dv": dv, "db1": db1, "db2": db2, "lse": lse}
+    for key, w in want.items():
+        np.testing.assert_allclose(got[key].reshape(-1), w, rtol=2e-7, atol=2e-7, err_msg=key)
+
+
+@pytest.mark.parametrize("phi", PHIS_ALL)
+def test_zero_biases_reproduce_the_unbiased_operator(phi):
+    p = _problem(31, B=3, h=2, dh=8, m=7, n=(5, 0, 3))
+    z1, z2 = np.zeros((3, 2, 7), np.float32), np.zeros((3, 2, 8), np.float32)
+    s = 0.6
+    a = oracle.fwd(p["q"], p["k"], p["v"], p["offsets"], phi, s)
+    b = oracle.fwd(p["q"], p["k"], p["v"], p["offsets"], phi, s, b1=z1, b2=z2)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    ga = oracle.bwd(p["q"], p["k"], p["v"], p["dout"], p["offsets"], phi, s)
+    gb = oracle.bwd(p["q"], p["k"], p["v"], p["dout"], p["offsets"], phi, s, b1=z1,
+                    bias_grads=True)
+    for x, y in zip(ga, gb[:3]):
+        assert np.array_equal(x, y)
+
+
+@pytest.mark.parametrize("phi", PHIS_ALL)
+def test_key_bias_is_an_extra_head_dim_column(phi):
+    """s (Q K^T) + b1 = s [Q, 1] [K, b1 / s]^T: the unbiased operator on inputs
+    with one more head-dim column gives the biased O, dQ, dK, and s * db1 as
+    the gradient of that column of K.  s = 1/2 keeps b1 / s exact in fp32."""
+    p = _problem(32, B=3, h=2, dh=6, m=5, n=(4, 3, 0))
+    s = 0.5
+    b1, b2 = _biases(5, 3, 2, 5, 6)
+    T = int(p["offsets"][-1])
+    qa = np.concatenate([p["q"].numpy(), np.ones((T, 2, 1), np.float32)], -1)
+    ka = np.concatenate([p["k"].numpy(), (b1 / s)[..., None]], -1)
+    va = np.concatenate([p["v"].numpy(), np.zeros((3, 2, 5, 1), np.float32)], -1)
+    ga = np.concatenate([p["dout"].numpy(), np.zeros((T, 2, 1), np.float32)], -1)
+    o, lse = oracle.fwd(p["q"], p["k"], p["v"], p["offsets"], phi, s, b1=b1)
+    oa, lsea = oracle.fwd(qa, ka, va, p["offsets"], phi, s)
+    assert _rel(o, oa[..., :6]) < 1e-13
+    if phi == "softmax":
+        assert np.abs(lse - lsea).max() < 1e-12
+    dq, dk, dv, db1, _ = oracle.bwd(p["q"], p["k"], p["v"], p["dout"], p["offsets"], phi, s,
+                                    b1=b1, bias_grads=True)
+    dqa, dka, dva = oracle.bwd(qa, ka, va, ga, p["offsets"], phi, s)
+    assert _rel(dq, dqa[..., :6]) < 1e-12
+    assert _rel(dk, dka[..., :6]) < 1e-12
+    assert _rel(dv, dva[..., :6]) < 1e-12
+    assert _rel(db1, dka[..., 6] / s) < 1e-12
+
+
+@pytest.mark.parametrize("phi", PHIS_ALL)
+def test_output_bias_shifts_o_and_its_gradient_is_the_token_sum(phi):
+    p = _problem(33, B=3, h=2, dh=8, m=6, n=(7, 0, 2))
+    s = 0.4
+    b1, b2 = _biases(6, 3, 2, 6, 8)
+    o1, l1 = oracle.fwd(p["q"], p["k"], p["v"], p["offsets"], phi, s, b1=b1)
+    o2, l2 = oracle.fwd(p["q"], p["k"], p["v"], p["offsets"], phi, s, b1=b1, b2=b2)
+    off = p["offsets"]
+    for b in range(3):
+        for j in range(2):
+            d = o2[off[b]:off[b + 1], j] - o1[off[b]:off[b + 1], j]
+            np.testing.assert_allclose(d, np.broadcast_to(b2[b, j], d.shape), atol=1e-14)
+    assert np.array_equal(l1, l2)
+    *_, db2 = oracle.bwd(p["q"], p["k"], p["v"], p["dout"], off, phi, s, b1=b1, bias_grads=True)
+    g = p["dout"].double().numpy()
+    for b in range(3):
+        np.testing.assert_allclose(db2[b], g[off[b]:off[b + 1]].sum(0), atol=1e-12)
+
+
+def test_softmax_key_bias_shift_invariance():
+    """Adding c to every key bias of a (sample, head) leaves softmax O, dQ, dK,
+    dV and db1 unchanged and moves LSE by c; db1 sums to zero over the keys."""
+    p = _problem(34, B=2, h=2, dh=8, m=9, n=(6, 4))
+    s = 0.35
+    b1, _ = _biases(7, 2, 2, 9, 8)
+    b1 = (np.round(b1 * 1024) / 1024).astype(np.float32)    # so that b1 + c is exact in fp32
+    c = np.float32(1.25)
+    a = oracle.fwd(p["q"], p["k"], p["v"], p["offsets"], "softmax", s, b1=b1)
+    b = oracle.fwd(p["q"], p["k"], p["v"], p["offsets"], "softmax", s, b1=b1 + c)
+    assert _rel(a[0], b[0]) < 1e-13
+    assert np.abs((b[1] - a[1]) - c).max() < 1e-12
+    ga = oracle.bwd(p["q"], p["k"], p["v"], p["dout"], p["offsets"], "softmax", s, b1=b1,
+                    bias_grads=True)
+    gb = oracle.bwd(p["q"], p["k"], p["v"], p["dout"], p["offsets"], "softmax", s, b1=b1 + c,
+                    bias_grads=True)
+    for x, y in zip(ga, gb):
+        assert _rel(x, y) < 1e-11
+    assert np.abs(ga[3].sum(-1)).max() < 1e-12
+
+
+@pytest.mark.parametrize("phi", PHIS_ALL)
+def test_biased_operator_matches_torch_autograd(phi):
+    p = random_problem(35, 3, 2, 8, 6, (4, 0, 5), dtype=torch.float32)
+    off = p["offsets"]
+    s = 0.45
+    b1n, b2n = _biases(8, 3, 2, 6, 8)
+    q, k, v = (p[x].double().requires_grad_(True) for x in ("q", "k", "v"))
+    b1 = torch.from_numpy(b1n).double().requires_grad_(True)
+    b2 = torch.from_numpy(b2n).double().requires_grad_(True)
+    g = p["dout"].double()
+    L = 0.0
+    ref_o = torch.zeros_like(q)
+    for b in range(3):
+        t0, t1 = int(off[b]), int(off[b + 1])
+        for j in range(2):
+            if t1 == t0:
+                continue
+            x = s * (q[t0:t1, j] @ k[b, j].T) + b1[b, j]
+            o = _LIB_PHI[phi](x) @ v[b, j] + b2[b, j]
+            ref_o[t0:t1, j] = o.detach()
+            L = L + (o * g[t0:t1, j]).sum()
+    L.backward()
+    o, _ = oracle.fwd(p["q"], p["k"], p["v"], off, phi, s, b1=b1n, b2=b2n)
+    assert _rel(o, ref_o.numpy()) < 1e-12
+    dq, dk, dv, db1, db2 = oracle.bwd(p["q"], p["k"], p["v"], p["dout"], off, phi, s, b1=b1n,
+                                      bias_grads=True)
+    for got, ref in ((dq, q.grad), (dk, k.grad), (dv, v.grad), (db1, b1.grad), (db2, b2.grad)):
+        assert _rel(got, ref.numpy()) < 1e-12
+
+
+@pytest.mark.parametrize("phi", PHIS_ALL)
+def test_bias_gradients_match_central_differences(phi):
+    p = random_problem(36, 2, 2, 3, 4, (3, 2), dtype=torch.float32)
+    off = p["offsets"]
+    s = 0.7
+    g = p["dout"].double().numpy()
+    b1, b2 = (x.astype(np.float64) for x in _biases(9, 2, 2, 4, 3, scale=0.5))
+
+    def loss(bb1, bb2):
+        o, _ = oracle.fwd(p["q"], p["k"], p["v"], off, phi, s, b1=bb1.astype(np.float32),
+                          b2=bb2.astype(np.float32))
+        return float((o * g).sum())
+
+    *_, db1, db2 = oracle.bwd(p["q"], p["k"], p["v"], p["dout"], off, phi, s,
+                              b1=b1.astype(np.float32), bias_grads=True)
+    eps = 2.0 ** -10
+    for which, x, grad in (("b1", b1, db1), ("b2", b2, db2)):
+        fd = np.zeros_like(x)
+        flat = x.reshape(-1)
+        for i in range(flat.size):
+            xp, xm = flat.copy(), flat.copy()
+            xp[i] += eps
+            xm[i] -= eps
+            if which == "b1":
+                lp, lm = loss(xp.reshape(x.shape), b2), loss(xm.reshape(x.shape), b2)
+            else:
+                lp, lm = loss(b1, xp.reshape(x.shape)), loss(b1, xm.reshape(x.shape))
+            fd.reshape(-1)[i] = (lp - lm) / (2 * eps)
+        assert _rel(grad, fd) < 2e-5, (which, _rel(grad, fd))
