@@ -131,6 +131,44 @@ GDPA_API gdpa_status_t gdpa_bwd(const gdpa_problem_t* p, const void* q, const in
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The PFFN variant with biases (reading of the Kunlun summary, section 2.2,
+ * GDPA bullet: GDPA is the Personalized FFN y = W2 phi(W1 x + b1) + b2 with
+ * per-sample weights, recast as attention; the pages print neither the
+ * formula nor the biases):
+ *
+ *     O_bj = phi(scale * Q_bj K_bj^T + 1 b1_bj^T) V_bj + 1 b2_bj^T
+ *
+ *   b1 fp32 [B, h, m]: per-sample, per-head key bias, added to every row of
+ *     the scaled logits before phi (softmax: inside the exponent).
+ *   b2 fp32 [B, h, dh]: per-sample, per-head output bias, added to every row
+ *     of O (and not to LSE).
+ *   Either may be NULL (a zero bias); with both NULL this is gdpa_fwd.  Device
+ *   pointers, 4-byte aligned.  Every other argument, the workspace size and
+ *   the error behaviour are those of gdpa_fwd.
+ */
+GDPA_API gdpa_status_t gdpa_fwd_bias(const gdpa_problem_t* p, const void* q,
+                                     const int32_t* offsets, const void* k, const void* v,
+                                     const float* b1, const float* b2, void* o, float* lse,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward of gdpa_fwd_bias for an upstream gradient dout of o.
+ *   b1, b2: the forward's biases (either may be NULL).  o: the biased
+ *   forward output (read for phi = softmax, whose row sums D = rowsum(dout *
+ *   (o - b2)) need it).
+ *   dq, dk, dv: as gdpa_bwd.  db1 fp32 [B, h, m] = the sum over each sample's
+ *   tokens of dS (the gradient of the biased logits); db2 fp32 [B, h, dh] = the
+ *   sum over each sample's tokens of dout.  Either may be NULL (not computed);
+ *   a sample with no tokens gets zeros.  Same workspace as gdpa_bwd.
+ */
+GDPA_API gdpa_status_t gdpa_bwd_bias(const gdpa_problem_t* p, const void* q,
+                                     const int32_t* offsets, const void* k, const void* v,
+                                     const float* b1, const float* b2, const void* o,
+                                     const float* lse, const void* dout, void* dq, void* dk,
+                                     void* dv, float* db1, float* db2, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/*
  * Device-detected status of the last gdpa_fwd/gdpa_bwd that used `workspace`
  * (GDPA_OK, GDPA_ERR_INVALID_ARG for inconsistent offsets, GDPA_ERR_TIMEOUT).
  * Synchronises `stream`; writes the code to *status (host).
@@ -176,6 +214,18 @@ GDPA_API int32_t gdpa_timing_read(gdpa_kernel_time_t* out, int32_t cap);
  */
 GDPA_API gdpa_status_t gdpa_selftest_wait_timeout(void* workspace, size_t workspace_bytes,
                                                   uint32_t timeout_us, void* stream);
+
+/*
+ * Self-test of the FMA-pipe exp2 that the softmax kernels use for part of
+ * their exponentials (Cody-Waite range reduction and a degree-3 minimax
+ * polynomial; relative error <= 7.5e-5 for -126 <= x < 127).  For n device
+ * floats x, writes that exp2 to y_fma and the hardware ex2.approx result to
+ * y_mufu (all device pointers, n >= 0), on `stream`.  Returns
+ * GDPA_ERR_INVALID_ARG for n < 0 or a null pointer with n > 0.  The Kunlun
+ * pages have no counterpart of this call.
+ */
+GDPA_API gdpa_status_t gdpa_selftest_exp2(const float* x, float* y_fma, float* y_mufu,
+                                          int64_t n, void* stream);
 
 /*
  * gdpa_fwd_no_alloc: gdpa_fwd for callers that cannot allocate device memory

@@ -8,10 +8,11 @@ libgdpa.so (CUDA C++ for sm_100a behind a C ABI, ``include/gdpa.h``);
 ``gdpa`` is its ctypes binding.
 """
 from . import gdpa  # noqa: F401
-from .gdpa import (GdpaError, Problem, bwd, bwd_workspace_bytes, fwd,  # noqa: F401
-                   fwd_workspace_bytes, load, problem, problem_for, workspace,
+from .gdpa import (GdpaError, Problem, bwd, bwd_bias, bwd_workspace_bytes, fwd,  # noqa: F401
+                   fwd_bias, fwd_workspace_bytes, load, problem, problem_for, workspace,
                    workspace_status)
 
-__all__ = ["gdpa", "GdpaError", "Problem", "fwd", "bwd", "fwd_workspace_bytes",
+__all__ = ["gdpa", "GdpaError", "Problem", "fwd", "bwd", "fwd_bias", "bwd_bias",
+           "fwd_workspace_bytes",
            "bwd_workspace_bytes", "load", "problem", "problem_for", "workspace",
            "workspace_status"]

@@ -43,12 +43,13 @@ static void clear_records() {
 
 // bf16 problems run on the tcgen05 kernels.
 cudaError_t launch_sm100_fwd(const gdpa_problem_t& p, const void* q, const void* k,
-                             const void* v, void* o, float* lse, WsHeader* ws,
+                             const void* v, const Bias& bs, void* o, float* lse, WsHeader* ws,
                              const Tile* tiles, cudaStream_t st);
 cudaError_t launch_sm100_bwd(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
-                             const void* k, const void* v, const void* o, const float* lse,
-                             const void* dout, void* dq, void* dk, void* dv, float* dq_acc,
-                             float* dsum, WsHeader* ws, Tile* tiles, cudaStream_t st);
+                             const void* k, const void* v, const Bias& bs, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                             float* dq_acc, float* dsum, WsHeader* ws, Tile* tiles,
+                             cudaStream_t st);
 int64_t sm100_bwd_items(const gdpa_problem_t& p);
 
 namespace {
@@ -142,9 +143,10 @@ gdpa_status_t gdpa_bwd_workspace_size(const gdpa_problem_t* p, size_t* bytes) {
   return GDPA_OK;
 }
 
-gdpa_status_t gdpa_fwd(const gdpa_problem_t* p, const void* q, const int32_t* offsets,
-                       const void* k, const void* v, void* o, float* lse, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+gdpa_status_t gdpa_fwd_bias(const gdpa_problem_t* p, const void* q, const int32_t* offsets,
+                            const void* k, const void* v, const float* b1, const float* b2,
+                            void* o, float* lse, void* workspace, size_t workspace_bytes,
+                            void* stream) {
   g_launches = 0;
   gdpa_status_t s = check_problem(p);
   if (s != GDPA_OK) return s;
@@ -152,28 +154,40 @@ gdpa_status_t gdpa_fwd(const gdpa_problem_t* p, const void* q, const int32_t* of
   const bool empty = p->total_tokens == 0;
   if (!offsets || !k || !v || (!empty && (!q || !o))) return GDPA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      ((uintptr_t)offsets & 3u) || ((uintptr_t)lse & 3u))
+      ((uintptr_t)offsets & 3u) || ((uintptr_t)lse & 3u) || ((uintptr_t)b1 & 3u) ||
+      ((uintptr_t)b2 & 3u))
     return GDPA_ERR_INVALID_ARG;
   const FwdLayout L = fwd_layout(*p);
   s = check_ws(workspace, workspace_bytes, L.total);
   if (s != GDPA_OK) return s;
   if (p->phi != GDPA_PHI_SOFTMAX) lse = nullptr;
+  Bias bs;
+  bs.b1 = b1;
+  bs.b2 = b2;
   cudaStream_t st = (cudaStream_t)stream;
   WsHeader* ws = (WsHeader*)workspace;
   Tile* tiles = (Tile*)((char*)workspace + L.tiles_off);
   cudaError_t e = launch_schedule(*p, offsets, L.bm, ws, tiles, st);
   if (e != cudaSuccess) return cuda_status(e);
   if (L.bm == kMmaBM)
-    e = launch_sm100_fwd(*p, q, k, v, o, lse, ws, tiles, st);
+    e = launch_sm100_fwd(*p, q, k, v, bs, o, lse, ws, tiles, st);
   else
-    e = launch_simt_fwd(*p, q, k, v, o, lse, ws, tiles, tile_capacity(*p, L.bm), st);
+    e = launch_simt_fwd(*p, q, k, v, bs, o, lse, ws, tiles, tile_capacity(*p, L.bm), st);
   return cuda_status(e);
 }
 
-gdpa_status_t gdpa_bwd(const gdpa_problem_t* p, const void* q, const int32_t* offsets,
-                       const void* k, const void* v, const void* o, const float* lse,
-                       const void* dout, void* dq, void* dk, void* dv, void* workspace,
+gdpa_status_t gdpa_fwd(const gdpa_problem_t* p, const void* q, const int32_t* offsets,
+                       const void* k, const void* v, void* o, float* lse, void* workspace,
                        size_t workspace_bytes, void* stream) {
+  return gdpa_fwd_bias(p, q, offsets, k, v, nullptr, nullptr, o, lse, workspace,
+                       workspace_bytes, stream);
+}
+
+gdpa_status_t gdpa_bwd_bias(const gdpa_problem_t* p, const void* q, const int32_t* offsets,
+                            const void* k, const void* v, const float* b1, const float* b2,
+                            const void* o, const float* lse, const void* dout, void* dq,
+                            void* dk, void* dv, float* db1, float* db2, void* workspace,
+                            size_t workspace_bytes, void* stream) {
   g_launches = 0;
   gdpa_status_t s = check_problem(p);
   if (s != GDPA_OK) return s;
@@ -184,30 +198,50 @@ gdpa_status_t gdpa_bwd(const gdpa_problem_t* p, const void* q, const int32_t* of
   if (!empty && p->phi == GDPA_PHI_SOFTMAX && (!o || !lse)) return GDPA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv) || (o && !aligned16(o)) || ((uintptr_t)offsets & 3u) ||
-      ((uintptr_t)lse & 3u))
+      ((uintptr_t)lse & 3u) || ((uintptr_t)b1 & 3u) || ((uintptr_t)b2 & 3u) ||
+      ((uintptr_t)db1 & 3u) || ((uintptr_t)db2 & 3u))
     return GDPA_ERR_INVALID_ARG;
   const BwdLayout L = bwd_layout(*p);
   s = check_ws(workspace, workspace_bytes, L.total);
   if (s != GDPA_OK) return s;
+  Bias bs;
+  bs.b1 = b1;
+  bs.b2 = b2;
+  bs.db1 = db1;
+  bs.db2 = db2;
   cudaStream_t st = (cudaStream_t)stream;
   WsHeader* ws = (WsHeader*)workspace;
   Tile* tiles = (Tile*)((char*)workspace + L.tiles_off);
   float* dsum = (float*)((char*)workspace + L.dsum_off);
   if (L.bm == kMmaBM) {
     float* dq_acc = (float*)((char*)workspace + L.dqacc_off);
-    return cuda_status(launch_sm100_bwd(*p, q, offsets, k, v, o, lse, dout, dq, dk, dv, dq_acc,
-                                        dsum, ws, tiles, st));
+    return cuda_status(launch_sm100_bwd(*p, q, offsets, k, v, bs, o, lse, dout, dq, dk, dv,
+                                        dq_acc, dsum, ws, tiles, st));
   }
   cudaError_t e = launch_schedule(*p, offsets, L.bm, ws, tiles, st);
   if (e != cudaSuccess) return cuda_status(e);
-  if (p->phi == GDPA_PHI_SOFTMAX) {
+  const bool softmax = p->phi == GDPA_PHI_SOFTMAX;
+  if (softmax && !b2) {
     e = launch_row_dot(*p, o, dout, dsum, st);
     if (e != cudaSuccess) return cuda_status(e);
   }
-  e = launch_simt_bwd_dq(*p, q, k, v, lse, dsum, dout, dq, ws, tiles, tile_capacity(*p, L.bm), st);
+  // db2, db1 = 0, and (with an output bias) the softmax row sums of O - b2
+  e = launch_bias_prep(*p, offsets, o, dout, b2, softmax && b2 ? dsum : nullptr, db1, db2, ws,
+                       st);
   if (e != cudaSuccess) return cuda_status(e);
-  e = launch_simt_bwd_dkdv(*p, q, offsets, k, v, lse, dsum, dout, dk, dv, ws, st);
+  e = launch_simt_bwd_dq(*p, q, k, v, bs, lse, dsum, dout, dq, ws, tiles,
+                         tile_capacity(*p, L.bm), st);
+  if (e != cudaSuccess) return cuda_status(e);
+  e = launch_simt_bwd_dkdv(*p, q, offsets, k, v, bs, lse, dsum, dout, dk, dv, ws, st);
   return cuda_status(e);
+}
+
+gdpa_status_t gdpa_bwd(const gdpa_problem_t* p, const void* q, const int32_t* offsets,
+                       const void* k, const void* v, const void* o, const float* lse,
+                       const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return gdpa_bwd_bias(p, q, offsets, k, v, nullptr, nullptr, o, lse, dout, dq, dk, dv, nullptr,
+                       nullptr, workspace, workspace_bytes, stream);
 }
 
 gdpa_status_t gdpa_workspace_status(const void* workspace, void* stream, int32_t* status) {

@@ -117,10 +117,24 @@ struct BwdArgs {
   float* dq_acc;         // [T, h, dh] fp32
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  const float* b1;       // [B, h, m] key bias (biased variant; may be NULL)
+  float* db1;            // [B, h, m] its gradient, zeroed beforehand (may be NULL)
   int64_t T;
   int h, m;
   float scale, scale_log2;
 };
+
+// This thread's key bias for the biased variant (zero past m or without b1).
+__device__ __forceinline__ float key_bias(const BwdArgs& a, const Tile& it, int key) {
+  return a.b1 != nullptr && key < a.m ? __ldg(a.b1 + ((int64_t)it.b * a.h + it.head) * a.m + key)
+                                      : 0.f;
+}
+// Adds this thread's partial sum of dS over its tokens into db1[b, head, key].
+__device__ __forceinline__ void add_key_bias_grad(const BwdArgs& a, const Tile& it, int key,
+                                                  float acc) {
+  if (a.db1 != nullptr && key < a.m)
+    atomicAdd(a.db1 + ((int64_t)it.b * a.h + it.head) * a.m + key, acc);
+}
 
 template <int DH>
 struct BwdCfg {
@@ -156,7 +170,7 @@ struct BwdCfg {
   static_assert(SMEM <= 232448u, "exceeds the 227 KB of shared memory a CTA can have");
 };
 
-template <int DH, int PHI>
+template <int DH, int PHI, bool BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
 gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmG,
@@ -378,6 +392,11 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
       const int nq = (n + 127) >> 7;
       const int t0 = a.offsets[it.b];
+      // biased variant: this key's bias (log2 units for softmax, halved for
+      // SiLU) and this thread's sum of dS over its tokens (for db1)
+      const float b1k = BIAS ? key_bias(a, it, key) : 0.f;
+      const float b1l = b1k * 1.4426950408889634f, hb = 0.5f * b1k;
+      float db1_acc = 0.f;
       // dQ_i drain: lane = query row of tile i; this group adds half of the columns
       auto drain_dq = [&](int ii, uint32_t step) -> bool {
         const uint32_t b = C::DQ2 ? (step & 1u) : 0u;
@@ -478,30 +497,32 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
               const float x = __uint_as_float(s[c + e]);
               const float g = __uint_as_float(dp[c + e]);
               float p, ds;
+              // u = s x + b1 (the biased logit; b1k = 0 without a key bias)
               if constexpr (SOFTMAX) {
-                p = ex2_approx(fmaf(x, c2, -wst[r]));
+                p = ex2_approx(fmaf(x, c2, BIAS ? b1l - wst[r] : -wst[r]));
                 ds = p * (g - wst[64 + r]);
               } else if constexpr (PHI == GDPA_PHI_SILU) {
-                const float hx = x * half_sc;
+                const float hx = fmaf(x, half_sc, hb);
                 const float th = tanh_approx(hx);
-                const float sg = fmaf(0.5f, th, 0.5f);          // logistic(x s)
-                p = fmaf(hx, th, hx);                             // x s * logistic(x s)
-                ds = g * sg * fmaf(x * sc, 1.f - sg, 1.f);
+                const float sg = fmaf(0.5f, th, 0.5f);          // logistic(u)
+                p = fmaf(hx, th, hx);                             // u * logistic(u)
+                ds = g * sg * fmaf(hx + hx, 1.f - sg, 1.f);
               } else if constexpr (PHI == GDPA_PHI_RELU) {
-                const float u = x * sc;
+                const float u = fmaf(x, sc, b1k);
                 p = relu_f(u);
                 ds = g * relu_grad(u);
               } else if constexpr (PHI == GDPA_PHI_GELU) {
-                const float u = x * sc;
+                const float u = fmaf(x, sc, b1k);
                 p = gelu_f(u);
                 ds = g * gelu_grad(u);
               } else {
-                p = x * sc;
+                p = fmaf(x, sc, b1k);
                 ds = g;
               }
               const bool valid = rbase + r < n;
               pv[e] = valid ? p : 0.f;
               dv2[e] = valid ? ds : 0.f;
+              if constexpr (BIAS) db1_acc += dv2[e];
             }
             pp[c / 2] = pack_bf16x2(pv[0], pv[1]);
             dd[c / 2] = pack_bf16x2(dv2[0], dv2[1]);
@@ -534,6 +555,7 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
       if (ok && C::DQ2 && !drain_dq(nq - 1, qs - 1)) ok = false;
       if (!ok) break;
+      if constexpr (BIAS) add_key_bias_grad(a, it, key, db1_acc);
       // ---------------------------------------------------------- dV / dK of this key block
       bool w = mbar_wait(bar(C::B_ACCFULL), ic & 1u, abort_flag, kTimeoutNs);
       if (!__all_sync(0xffffffffu, w)) {
@@ -689,7 +711,7 @@ __device__ __forceinline__ uint32_t stage_chunk(uint32_t box, int r, int j) {
   return box + (uint32_t)(r * 2 * DH) + ((uint32_t)(j ^ sw) << 4);
 }
 
-template <int DH, int PHI>
+template <int DH, int PHI, bool BIAS>
 __global__ void __launch_bounds__(kHalfThreads, 1)
 gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmG,
@@ -982,6 +1004,12 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
       const int n = it.rows;
       if (n == 0) continue;
       const int nq = (n + 127) >> 7;
+      // biased variant: this key's bias (log2 units for softmax, halved for
+      // SiLU) and this thread's sum of dS over its half of the tokens (for db1)
+      const int key = it.row0 + lrow;
+      const float b1k = BIAS ? key_bias(a, it, key) : 0.f;
+      const float b1l = b1k * 1.4426950408889634f, hb = 0.5f * b1k;
+      float db1_acc = 0.f;
       for (int i = 0; i < nq; ++i, ++qs) {
         const int rbase = 128 * i + 64 * grp;          // first sample row of this group's half
         const uint32_t dsb = sDS + (qs & 1u) * C::DSB + grp * 16384;
@@ -1012,30 +1040,32 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
               const float x = __uint_as_float(s[c + e]);
               const float g = __uint_as_float(dp[c + e]);
               float p, ds;
+              // u = s x + b1 (the biased logit; b1k = 0 without a key bias)
               if constexpr (SOFTMAX) {
-                p = ex2_approx(fmaf(x, c2, -st_l[r]));
+                p = ex2_approx(fmaf(x, c2, BIAS ? b1l - st_l[r] : -st_l[r]));
                 ds = p * (g - st_d[r]);
               } else if constexpr (PHI == GDPA_PHI_SILU) {
-                const float hx = x * half_sc;
+                const float hx = fmaf(x, half_sc, hb);
                 const float th = tanh_approx(hx);
-                const float sg = fmaf(0.5f, th, 0.5f);          // logistic(x s)
-                p = fmaf(hx, th, hx);                             // x s * logistic(x s)
-                ds = g * sg * fmaf(x * sc, 1.f - sg, 1.f);
+                const float sg = fmaf(0.5f, th, 0.5f);          // logistic(u)
+                p = fmaf(hx, th, hx);                             // u * logistic(u)
+                ds = g * sg * fmaf(hx + hx, 1.f - sg, 1.f);
               } else if constexpr (PHI == GDPA_PHI_RELU) {
-                const float u = x * sc;
+                const float u = fmaf(x, sc, b1k);
                 p = relu_f(u);
                 ds = g * relu_grad(u);
               } else if constexpr (PHI == GDPA_PHI_GELU) {
-                const float u = x * sc;
+                const float u = fmaf(x, sc, b1k);
                 p = gelu_f(u);
                 ds = g * gelu_grad(u);
               } else {
-                p = x * sc;
+                p = fmaf(x, sc, b1k);
                 ds = g;
               }
               const bool valid = rbase + r < n;
               pv[e] = valid ? p : 0.f;
               dv2[e] = valid ? ds : 0.f;
+              if constexpr (BIAS) db1_acc += dv2[e];
             }
             pp[c / 2] = pack_bf16x2(pv[0], pv[1]);
             dd[c / 2] = pack_bf16x2(dv2[0], dv2[1]);
@@ -1060,6 +1090,9 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(C::B_STATEMPTY + (int)(qs & 1u)));
         }
+      }
+      if constexpr (BIAS) {
+        if (ok) add_key_bias_grad(a, it, key, db1_acc);
       }
     }
   } else {
@@ -1271,11 +1304,11 @@ bool make_dq_map(const gdpa_problem_t& p, float* dq_acc, CUtensorMap* m) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DH, int PHI>
+template <int DH, int PHI, bool BIAS>
 cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
-                         const void* k, const void* v, const float* lse, const float* dsum,
-                         const void* g, void* dk, void* dv, float* dq_acc, WsHeader* ws,
-                         const Tile* tiles, cudaStream_t st) {
+                         const void* k, const void* v, const Bias& bs, const float* lse,
+                         const float* dsum, const void* g, void* dk, void* dv, float* dq_acc,
+                         WsHeader* ws, const Tile* tiles, cudaStream_t st) {
   CUtensorMap mq, mg, mk, mv;
   if (p.total_tokens == 0) q = g = k;   // no query rows: the maps are never read
   if (!make_bwd_maps<DH>(p, q, g, k, v, &mq, &mg, &mk, &mv)) return cudaErrorInvalidValue;
@@ -1289,6 +1322,8 @@ cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* 
   args.dq_acc = dq_acc;
   args.dk = reinterpret_cast<__nv_bfloat16*>(dk);
   args.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+  args.b1 = bs.b1;
+  args.db1 = bs.db1;
   args.T = p.total_tokens;
   args.h = p.h;
   args.m = p.m;
@@ -1296,7 +1331,7 @@ cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* 
   args.scale_log2 = p.scale * 1.4426950408889634f;
   if constexpr (DH <= 64) {
     using H = BwdHalfCfg<DH>;
-    auto hk = gdpa_bwd_half_kernel<DH, PHI>;
+    auto hk = gdpa_bwd_half_kernel<DH, PHI, BIAS>;
     CUtensorMap mdq, mdv, mdk, unused_q, unused_g;
     if (!make_dq_map<DH>(p, dq_acc, &mdq)) return cudaErrorInvalidValue;
     // the outputs dV, dK have the layout (and so the maps) of the inputs K, V
@@ -1309,7 +1344,7 @@ cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* 
     return cudaGetLastError();
   } else {
     using C = BwdCfg<DH>;
-    auto kern = gdpa_bwd_sm100_kernel<DH, PHI>;     // dh = 128 only
+    auto kern = gdpa_bwd_sm100_kernel<DH, PHI, BIAS>;     // dh = 128 only
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     if (e != cudaSuccess) return e;
     KernelScope ks_("gdpa_bwd_sm100", st);
@@ -1318,23 +1353,33 @@ cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* 
   }
 }
 
-template <int DH>
+template <int DH, bool BIAS>
 cudaError_t launch_bwd_dh(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
-                          const void* k, const void* v, const float* lse, const float* dsum,
-                          const void* g, void* dk, void* dv, float* dq_acc, WsHeader* ws,
-                          const Tile* tiles, cudaStream_t st) {
+                          const void* k, const void* v, const Bias& bs, const float* lse,
+                          const float* dsum, const void* g, void* dk, void* dv, float* dq_acc,
+                          WsHeader* ws, const Tile* tiles, cudaStream_t st) {
+#define GDPA_BWD_PHI(PHIV) \
+  launch_bwd_t<DH, PHIV, BIAS>(p, q, offsets, k, v, bs, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st)
   switch (p.phi) {
-    case GDPA_PHI_SOFTMAX:
-      return launch_bwd_t<DH, GDPA_PHI_SOFTMAX>(p, q, offsets, k, v, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st);
-    case GDPA_PHI_SILU:
-      return launch_bwd_t<DH, GDPA_PHI_SILU>(p, q, offsets, k, v, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st);
-    case GDPA_PHI_RELU:
-      return launch_bwd_t<DH, GDPA_PHI_RELU>(p, q, offsets, k, v, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st);
-    case GDPA_PHI_GELU:
-      return launch_bwd_t<DH, GDPA_PHI_GELU>(p, q, offsets, k, v, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st);
-    default:
-      return launch_bwd_t<DH, GDPA_PHI_IDENTITY>(p, q, offsets, k, v, lse, dsum, g, dk, dv, dq_acc, ws, tiles, st);
+    case GDPA_PHI_SOFTMAX: return GDPA_BWD_PHI(GDPA_PHI_SOFTMAX);
+    case GDPA_PHI_SILU: return GDPA_BWD_PHI(GDPA_PHI_SILU);
+    case GDPA_PHI_RELU: return GDPA_BWD_PHI(GDPA_PHI_RELU);
+    case GDPA_PHI_GELU: return GDPA_BWD_PHI(GDPA_PHI_GELU);
+    default: return GDPA_BWD_PHI(GDPA_PHI_IDENTITY);
   }
+#undef GDPA_BWD_PHI
+}
+
+template <int DH>
+cudaError_t launch_bwd_bias(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
+                            const void* k, const void* v, const Bias& bs, const float* lse,
+                            const float* dsum, const void* g, void* dk, void* dv, float* dq_acc,
+                            WsHeader* ws, const Tile* tiles, cudaStream_t st) {
+  if (bs.b1 || bs.db1)
+    return launch_bwd_dh<DH, true>(p, q, offsets, k, v, bs, lse, dsum, g, dk, dv, dq_acc, ws,
+                                   tiles, st);
+  return launch_bwd_dh<DH, false>(p, q, offsets, k, v, bs, lse, dsum, g, dk, dv, dq_acc, ws,
+                                  tiles, st);
 }
 
 }  // namespace
@@ -1343,31 +1388,37 @@ int64_t sm100_bwd_items(const gdpa_problem_t& p) {
   return (int64_t)p.B * p.h * ((p.m + 127) / 128);
 }
 
-// schedule (LPT list) -> prep (zero dQ accumulator, softmax D) -> fused
-// backward -> dQ conversion.
+// schedule (LPT list) -> prep (zero dQ accumulator, softmax D) -> [bias terms]
+// -> fused backward -> dQ conversion.
 cudaError_t launch_sm100_bwd(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
-                             const void* k, const void* v, const void* o, const float* lse,
-                             const void* dout, void* dq, void* dk, void* dv, float* dq_acc,
-                             float* dsum, WsHeader* ws, Tile* tiles, cudaStream_t st) {
+                             const void* k, const void* v, const Bias& bs, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                             float* dq_acc, float* dsum, WsHeader* ws, Tile* tiles,
+                             cudaStream_t st) {
   cudaError_t e = launch_schedule_kv(p, offsets, ws, tiles, st);
   if (e != cudaSuccess) return e;
   const int64_t rows = p.total_tokens * p.h;
   const int sms = device_sm_count();
+  const bool softmax = p.phi == GDPA_PHI_SOFTMAX;
   if (rows > 0) {
     KernelScope ks_("gdpa_bwd_prep", st);
     auto prep = p.dh == 32 ? bwd_prep_kernel<32> : p.dh == 64 ? bwd_prep_kernel<64>
                                                               : bwd_prep_kernel<128>;
+    // with an output bias the softmax row sums come from the bias kernel (O - b2)
     prep<<<sms * 8, 256, 0, st>>>(reinterpret_cast<const uint4*>(o),
                                   reinterpret_cast<const uint4*>(dout), dsum,
                                   reinterpret_cast<float4*>(dq_acc), rows, p.h, p.total_tokens,
-                                  p.phi == GDPA_PHI_SOFTMAX ? 1 : 0);
+                                  softmax && !bs.b2 ? 1 : 0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  e = launch_bias_prep(p, offsets, o, dout, bs.b2, softmax && bs.b2 ? dsum : nullptr, bs.db1,
+                       bs.db2, ws, st);
+  if (e != cudaSuccess) return e;
   switch (p.dh) {
-    case 32: e = launch_bwd_dh<32>(p, q, offsets, k, v, lse, dsum, dout, dk, dv, dq_acc, ws, tiles, st); break;
-    case 64: e = launch_bwd_dh<64>(p, q, offsets, k, v, lse, dsum, dout, dk, dv, dq_acc, ws, tiles, st); break;
-    case 128: e = launch_bwd_dh<128>(p, q, offsets, k, v, lse, dsum, dout, dk, dv, dq_acc, ws, tiles, st); break;
+    case 32: e = launch_bwd_bias<32>(p, q, offsets, k, v, bs, lse, dsum, dout, dk, dv, dq_acc, ws, tiles, st); break;
+    case 64: e = launch_bwd_bias<64>(p, q, offsets, k, v, bs, lse, dsum, dout, dk, dv, dq_acc, ws, tiles, st); break;
+    case 128: e = launch_bwd_bias<128>(p, q, offsets, k, v, bs, lse, dsum, dout, dk, dv, dq_acc, ws, tiles, st); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess || rows == 0) return e;

@@ -53,6 +53,16 @@ template <> struct Elem<__nv_bfloat16> {
 // ---------------------------------------------------------------------------
 // launchers (each returns cudaSuccess or the launch error)
 
+// Bias terms of the biased variant phi(s Q K^T + b1) V + b2 (each may be NULL):
+// b1 [B, h, m] and b2 [B, h, dh] inputs, db1 and db2 (same shapes) outputs; fp32.
+struct Bias {
+  const float* b1 = nullptr;
+  const float* b2 = nullptr;
+  float* db1 = nullptr;
+  float* db2 = nullptr;
+};
+
+
 // Builds the jagged tile list (tiles of `bm` rows) and clears the status word.
 cudaError_t launch_schedule(const gdpa_problem_t& p, const int32_t* offsets, int bm,
                             WsHeader* ws, Tile* tiles, cudaStream_t st);
@@ -63,18 +73,26 @@ cudaError_t launch_schedule_kv(const gdpa_problem_t& p, const int32_t* offsets, 
 
 // SIMT kernels (fp32 problems only; fp32 math).
 cudaError_t launch_simt_fwd(const gdpa_problem_t& p, const void* q, const void* k,
-                            const void* v, void* o, float* lse, WsHeader* ws,
+                            const void* v, const Bias& bs, void* o, float* lse, WsHeader* ws,
                             const Tile* tiles, int64_t tile_cap, cudaStream_t st);
 cudaError_t launch_row_dot(const gdpa_problem_t& p, const void* o, const void* dout,
                            float* dsum, cudaStream_t st);
 cudaError_t launch_simt_bwd_dq(const gdpa_problem_t& p, const void* q, const void* k,
-                               const void* v, const float* lse, const float* dsum,
+                               const void* v, const Bias& bs, const float* lse, const float* dsum,
                                const void* dout, void* dq, WsHeader* ws, const Tile* tiles,
                                int64_t tile_cap, cudaStream_t st);
 cudaError_t launch_simt_bwd_dkdv(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
-                                 const void* k, const void* v, const float* lse,
+                                 const void* k, const void* v, const Bias& bs, const float* lse,
                                  const float* dsum, const void* dout, void* dk, void* dv,
                                  WsHeader* ws, cudaStream_t st);
+
+// Backward bias terms: db2 = per-sample token sums of dO, softmax row sums
+// D = rowsum(dO * (O - b2)) into `dsum` (when not NULL), db1 zeroed (the
+// fused kernels add into it).  Skips its work when the scheduler rejected the
+// offsets.
+cudaError_t launch_bias_prep(const gdpa_problem_t& p, const int32_t* offsets, const void* o,
+                             const void* g, const float* b2, float* dsum, float* db1,
+                             float* db2, const WsHeader* ws, cudaStream_t st);
 
 // Brackets one kernel launch: counts it for gdpa_last_launch_count() and, while
 // gdpa_timing_enable(1) is in force, records CUDA events around it on `st`.
@@ -112,6 +130,31 @@ __device__ __forceinline__ float gelu_grad(float x) {
   float cdf, gauss;
   normal_cdf_gauss(x, cdf, gauss);
   return fmaf(x * 0.3989422804014327f, gauss, cdf);
+}
+
+// 2^x for two values at once on the FMA pipe, without the MUFU unit: Cody-Waite
+// range reduction x = n + f with n = floor(x) and f in [0, 1), 2^f from a
+// degree-3 polynomial, and 2^n added into the exponent field.  The polynomial
+// minimises the largest relative error |p(f) / 2^f - 1| over [0, 1] (Remez
+// exchange, exp2_fit.py in the package, which reproduces these coefficients):
+// the error is at most 7.5e-5, well below half an ulp of bf16 (2^-9), the
+// precision of the P operand it feeds.  x is clamped at -126 so that the
+// biased exponent of the result stays >= 0 (every x <= -126 gives about
+// 2^-126, negligible next to a row sum >= 1); x must be < 127.
+constexpr float kExp2C0 = 0.99992520f, kExp2C1 = 0.69583356f, kExp2C2 = 0.22606716f,
+                kExp2C3 = 0.07802452f;
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rd(x, make_float2(12582912.f, 12582912.f));   // 1.5 * 2^23 + floor(x)
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));  // floor(x), exact
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);             // x - floor(x), exact
+  float2 q = __ffma2_rn(f, make_float2(kExp2C3, kExp2C3), make_float2(kExp2C2, kExp2C2));
+  q = __ffma2_rn(q, f, make_float2(kExp2C1, kExp2C1));
+  q = __ffma2_rn(q, f, make_float2(kExp2C0, kExp2C0));
+  // the low bits of t hold n (1.5 * 2^23 has an ulp of 1): n << 23 scales q by 2^n
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
 }  // namespace gdpa

@@ -39,3 +39,35 @@ extern "C" gdpa_status_t gdpa_selftest_wait_timeout(void* workspace, size_t work
   }
   return cudaGetLastError() == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
 }
+
+namespace gdpa {
+namespace {
+
+// y_fma[i] = exp2_fma2(x[i]) (the FMA-pipe exp2 of the softmax kernels) and
+// y_mufu[i] = ex2.approx.ftz (the MUFU unit), for checking the former against
+// a reference exp2 and against the latter.
+__global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y_fma,
+                                     float* __restrict__ y_mufu, int64_t n) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const float v = x[i];
+    y_fma[i] = exp2_fma2(make_float2(v, v)).x;
+    y_mufu[i] = sm100::ex2_approx(v);
+  }
+}
+
+}  // namespace
+}  // namespace gdpa
+
+extern "C" gdpa_status_t gdpa_selftest_exp2(const float* x, float* y_fma, float* y_mufu,
+                                            int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y_fma || !y_mufu))) return GDPA_ERR_INVALID_ARG;
+  if (n == 0) return GDPA_OK;
+  const int64_t blocks = (n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184;
+  {
+    gdpa::KernelScope ks_("gdpa_selftest_exp2", (cudaStream_t)stream);
+    gdpa::exp2_selftest_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(x, y_fma,
+                                                                                   y_mufu, n);
+  }
+  return cudaGetLastError() == cudaSuccess ? GDPA_OK : GDPA_ERR_CUDA;
+}

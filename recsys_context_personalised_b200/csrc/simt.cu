@@ -32,6 +32,7 @@ __device__ __forceinline__ float silu_grad(float x) {
 template <typename T, int DH>
 __global__ void __launch_bounds__(kThreads)
 simt_fwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                const float* __restrict__ b1, const float* __restrict__ b2,
                 T* __restrict__ o, float* __restrict__ lse, int64_t Ttot, int h, int m, int phi,
                 float scale, const WsHeader* __restrict__ ws, const Tile* __restrict__ tiles) {
   if ((int)blockIdx.x >= ws->tile_count) return;
@@ -51,6 +52,7 @@ simt_fwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
   }
   const T* kb = k + ((int64_t)tl.b * h + tl.head) * (int64_t)m * DH;
   const T* vb = v + ((int64_t)tl.b * h + tl.head) * (int64_t)m * DH;
+  const float* b1r = b1 ? b1 + ((int64_t)tl.b * h + tl.head) * m : nullptr;
   float acc[CW];
 #pragma unroll
   for (int j = 0; j < CW; ++j) acc[j] = 0.f;
@@ -76,7 +78,8 @@ simt_fwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
       float dot = 0.f;
 #pragma unroll 8
       for (int d = 0; d < DH; ++d) dot = fmaf(qr[d], kr[d], dot);
-      s[i] = scale * dot;
+      const int key = k0 + c * 8 + i;
+      s[i] = b1r && key < m ? fmaf(scale, dot, b1r[key]) : scale * dot;
     }
     if (phi == GDPA_PHI_SOFTMAX) {
       float cm = -INFINITY;
@@ -125,8 +128,9 @@ simt_fwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     float inv = 1.f;
     if (phi == GDPA_PHI_SOFTMAX) inv = 1.f / lrun;
     T* orow = o + ((int64_t)(tl.row0 + r) * h + tl.head) * DH + c * CW;
+    const float* b2r = b2 ? b2 + ((int64_t)tl.b * h + tl.head) * DH + c * CW : nullptr;
 #pragma unroll
-    for (int j = 0; j < CW; ++j) orow[j] = Elem<T>::from_f(acc[j] * inv);
+    for (int j = 0; j < CW; ++j) orow[j] = Elem<T>::from_f(fmaf(acc[j], inv, b2r ? b2r[j] : 0.f));
     if (phi == GDPA_PHI_SOFTMAX && c == 0 && lse != nullptr)
       lse[(int64_t)tl.head * Ttot + tl.row0 + r] = mrun + logf(lrun);
   }
@@ -181,7 +185,8 @@ __device__ __forceinline__ float dlogit(int phi, float s, float dp, float lse_r,
 template <typename T, int DH>
 __global__ void __launch_bounds__(kThreads)
 simt_bwd_dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                   const float* __restrict__ lse, const float* __restrict__ dsum,
+                   const float* __restrict__ b1, const float* __restrict__ lse,
+                   const float* __restrict__ dsum,
                    const T* __restrict__ g, T* __restrict__ dq, int64_t Ttot, int h, int m,
                    int phi, float scale, const WsHeader* __restrict__ ws,
                    const Tile* __restrict__ tiles) {
@@ -213,6 +218,7 @@ simt_bwd_dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
   }
   const T* kb = k + ((int64_t)tl.b * h + tl.head) * (int64_t)m * DH;
   const T* vb = v + ((int64_t)tl.b * h + tl.head) * (int64_t)m * DH;
+  const float* b1r = b1 ? b1 + ((int64_t)tl.b * h + tl.head) * m : nullptr;
   float acc[CW];
 #pragma unroll
   for (int j = 0; j < CW; ++j) acc[j] = 0.f;
@@ -243,7 +249,8 @@ simt_bwd_dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
         pdot = fmaf(gr[d], vr[d], pdot);
       }
       float p;
-      float ds = dlogit(phi, scale * sdot, pdot, lse_r, d_r, &p);
+      const float x = b1r && k0 + kk < m ? fmaf(scale, sdot, b1r[k0 + kk]) : scale * sdot;
+      float ds = dlogit(phi, x, pdot, lse_r, d_r, &p);
       if (k0 + kk >= m || r >= tl.rows) ds = 0.f;
       Ds[r * PL + kk] = ds;
     }
@@ -267,6 +274,7 @@ template <typename T, int DH>
 __global__ void __launch_bounds__(kThreads)
 simt_bwd_dkdv_kernel(const T* __restrict__ q, const int32_t* __restrict__ offsets,
                      const T* __restrict__ k, const T* __restrict__ v,
+                     const float* __restrict__ b1, float* __restrict__ db1,
                      const float* __restrict__ lse, const float* __restrict__ dsum,
                      const T* __restrict__ g, T* __restrict__ dk, T* __restrict__ dv,
                      int64_t Ttot, int h, int m, int phi, float scale,
@@ -301,6 +309,9 @@ simt_bwd_dkdv_kernel(const T* __restrict__ q, const int32_t* __restrict__ offset
   }
   const int t0 = offsets[b];
   const int n = offsets[b + 1] - t0;
+  // this thread's key bias (row r of the key tile) and its share of db1
+  const float b1k = b1 && key0 + r < m ? b1[((int64_t)b * h + head) * m + key0 + r] : 0.f;
+  float db1_acc = 0.f;
   float ak[CW], av[CW];
 #pragma unroll
   for (int j = 0; j < CW; ++j) ak[j] = av[j] = 0.f;
@@ -341,11 +352,12 @@ simt_bwd_dkdv_kernel(const T* __restrict__ q, const int32_t* __restrict__ offset
         pdot = fmaf(vr[d], gr[d], pdot);
       }
       float p;
-      float ds = dlogit(phi, scale * sdot, pdot, Ls[tt], Dr[tt], &p);
+      float ds = dlogit(phi, fmaf(scale, sdot, b1k), pdot, Ls[tt], Dr[tt], &p);
       if (i0 + tt >= n || key0 + r >= m) {
         ds = 0.f;
         p = 0.f;
       }
+      db1_acc += ds;
       Ps[r * PL + tt] = p;
       Dss[r * PL + tt] = ds;
     }
@@ -361,6 +373,10 @@ simt_bwd_dkdv_kernel(const T* __restrict__ q, const int32_t* __restrict__ offset
       }
     }
   }
+  // the 4 lanes of key r each summed dS over 8 of every 32 tokens
+  db1_acc += __shfl_xor_sync(0xffffffffu, db1_acc, 1);
+  db1_acc += __shfl_xor_sync(0xffffffffu, db1_acc, 2);
+  if (db1 && c == 0 && key0 + r < m) db1[((int64_t)b * h + head) * m + key0 + r] = db1_acc;
   if (key0 + r < m) {
     const int64_t at = kvbase + (int64_t)(key0 + r) * DH + c * CW;
 #pragma unroll
@@ -379,28 +395,31 @@ template <typename T, int DH>
 size_t dkdv_smem() { return sizeof(float) * (2 * kRows * (DH + 1) + 2 * kChunk * (DH + 1) + 2 * kRows * (kChunk + 1) + 2 * kChunk); }
 
 template <typename T, int DH>
-cudaError_t fwd_t(const gdpa_problem_t& p, const void* q, const void* k, const void* v, void* o,
-                  float* lse, WsHeader* ws, const Tile* tiles, int64_t cap, cudaStream_t st) {
+cudaError_t fwd_t(const gdpa_problem_t& p, const void* q, const void* k, const void* v,
+                  const Bias& bs, void* o, float* lse, WsHeader* ws, const Tile* tiles,
+                  int64_t cap, cudaStream_t st) {
   auto kern = simt_fwd_kernel<T, DH>;
   const size_t sm = fwd_smem<T, DH>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   KernelScope ks_("gdpa_simt_fwd", st);
-  kern<<<(unsigned)cap, kThreads, sm, st>>>((const T*)q, (const T*)k, (const T*)v, (T*)o, lse,
-                                             p.total_tokens, p.h, p.m, p.phi, p.scale, ws, tiles);
+  kern<<<(unsigned)cap, kThreads, sm, st>>>((const T*)q, (const T*)k, (const T*)v, bs.b1, bs.b2,
+                                             (T*)o, lse, p.total_tokens, p.h, p.m, p.phi, p.scale,
+                                             ws, tiles);
   return cudaGetLastError();
 }
 
 template <typename T, int DH>
 cudaError_t dq_t(const gdpa_problem_t& p, const void* q, const void* k, const void* v,
-                 const float* lse, const float* dsum, const void* g, void* dq, WsHeader* ws,
-                 const Tile* tiles, int64_t cap, cudaStream_t st) {
+                 const Bias& bs, const float* lse, const float* dsum, const void* g, void* dq,
+                 WsHeader* ws, const Tile* tiles, int64_t cap, cudaStream_t st) {
   auto kern = simt_bwd_dq_kernel<T, DH>;
   const size_t sm = dq_smem<T, DH>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   KernelScope ks_("gdpa_simt_bwd_dq", st);
-  kern<<<(unsigned)cap, kThreads, sm, st>>>((const T*)q, (const T*)k, (const T*)v, lse, dsum,
+  kern<<<(unsigned)cap, kThreads, sm, st>>>((const T*)q, (const T*)k, (const T*)v, bs.b1, lse,
+                                             dsum,
                                              (const T*)g, (T*)dq, p.total_tokens, p.h, p.m, p.phi,
                                              p.scale, ws, tiles);
   return cudaGetLastError();
@@ -408,16 +427,16 @@ cudaError_t dq_t(const gdpa_problem_t& p, const void* q, const void* k, const vo
 
 template <typename T, int DH>
 cudaError_t dkdv_t(const gdpa_problem_t& p, const void* q, const int32_t* offsets, const void* k,
-                   const void* v, const float* lse, const float* dsum, const void* g, void* dk,
-                   void* dv, WsHeader* ws, cudaStream_t st) {
+                   const void* v, const Bias& bs, const float* lse, const float* dsum,
+                   const void* g, void* dk, void* dv, WsHeader* ws, cudaStream_t st) {
   auto kern = simt_bwd_dkdv_kernel<T, DH>;
   const size_t sm = dkdv_smem<T, DH>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const int64_t blocks = (int64_t)p.B * p.h * ((p.m + kRows - 1) / kRows);
   KernelScope ks_("gdpa_simt_bwd_dkdv", st);
-  kern<<<(unsigned)blocks, kThreads, sm, st>>>((const T*)q, offsets, (const T*)k, (const T*)v, lse,
-                                                dsum, (const T*)g, (T*)dk, (T*)dv, p.total_tokens,
+  kern<<<(unsigned)blocks, kThreads, sm, st>>>((const T*)q, offsets, (const T*)k, (const T*)v,
+                                                bs.b1, bs.db1, lse, dsum, (const T*)g, (T*)dk, (T*)dv, p.total_tokens,
                                                 p.h, p.m, p.phi, p.scale, ws);
   return cudaGetLastError();
 }
@@ -430,18 +449,18 @@ cudaError_t dkdv_t(const gdpa_problem_t& p, const void* q, const int32_t* offset
     default: return cudaErrorInvalidValue;                                         \
   }
 
-template <int DH> cudaError_t fwd_f32(const gdpa_problem_t& p, const void* q, const void* k, const void* v, void* o, float* lse, WsHeader* ws, const Tile* t, int64_t cap, cudaStream_t st) { return fwd_t<float, DH>(p, q, k, v, o, lse, ws, t, cap, st); }
-template <int DH> cudaError_t dq_f32(const gdpa_problem_t& p, const void* q, const void* k, const void* v, const float* l, const float* ds, const void* g, void* dq, WsHeader* ws, const Tile* t, int64_t cap, cudaStream_t st) { return dq_t<float, DH>(p, q, k, v, l, ds, g, dq, ws, t, cap, st); }
-template <int DH> cudaError_t dkdv_f32(const gdpa_problem_t& p, const void* q, const int32_t* off, const void* k, const void* v, const float* l, const float* ds, const void* g, void* dk, void* dv, WsHeader* ws, cudaStream_t st) { return dkdv_t<float, DH>(p, q, off, k, v, l, ds, g, dk, dv, ws, st); }
+template <int DH> cudaError_t fwd_f32(const gdpa_problem_t& p, const void* q, const void* k, const void* v, const Bias& bs, void* o, float* lse, WsHeader* ws, const Tile* t, int64_t cap, cudaStream_t st) { return fwd_t<float, DH>(p, q, k, v, bs, o, lse, ws, t, cap, st); }
+template <int DH> cudaError_t dq_f32(const gdpa_problem_t& p, const void* q, const void* k, const void* v, const Bias& bs, const float* l, const float* ds, const void* g, void* dq, WsHeader* ws, const Tile* t, int64_t cap, cudaStream_t st) { return dq_t<float, DH>(p, q, k, v, bs, l, ds, g, dq, ws, t, cap, st); }
+template <int DH> cudaError_t dkdv_f32(const gdpa_problem_t& p, const void* q, const int32_t* off, const void* k, const void* v, const Bias& bs, const float* l, const float* ds, const void* g, void* dk, void* dv, WsHeader* ws, cudaStream_t st) { return dkdv_t<float, DH>(p, q, off, k, v, bs, l, ds, g, dk, dv, ws, st); }
 
 }  // namespace
 
 cudaError_t launch_simt_fwd(const gdpa_problem_t& p, const void* q, const void* k, const void* v,
-                            void* o, float* lse, WsHeader* ws, const Tile* tiles, int64_t cap,
-                            cudaStream_t st) {
+                            const Bias& bs, void* o, float* lse, WsHeader* ws, const Tile* tiles,
+                            int64_t cap, cudaStream_t st) {
   if (cap <= 0) return cudaSuccess;
   if (p.dtype != GDPA_DTYPE_F32) return cudaErrorInvalidValue;
-  GDPA_DISPATCH_DH(p.dh, fwd_f32, p, q, k, v, o, lse, ws, tiles, cap, st);
+  GDPA_DISPATCH_DH(p.dh, fwd_f32, p, q, k, v, bs, o, lse, ws, tiles, cap, st);
 }
 
 cudaError_t launch_row_dot(const gdpa_problem_t& p, const void* o, const void* g, float* dsum,
@@ -459,20 +478,20 @@ cudaError_t launch_row_dot(const gdpa_problem_t& p, const void* o, const void* g
 }
 
 cudaError_t launch_simt_bwd_dq(const gdpa_problem_t& p, const void* q, const void* k,
-                               const void* v, const float* lse, const float* dsum,
+                               const void* v, const Bias& bs, const float* lse, const float* dsum,
                                const void* g, void* dq, WsHeader* ws, const Tile* tiles,
                                int64_t cap, cudaStream_t st) {
   if (cap <= 0) return cudaSuccess;
   if (p.dtype != GDPA_DTYPE_F32) return cudaErrorInvalidValue;
-  GDPA_DISPATCH_DH(p.dh, dq_f32, p, q, k, v, lse, dsum, g, dq, ws, tiles, cap, st);
+  GDPA_DISPATCH_DH(p.dh, dq_f32, p, q, k, v, bs, lse, dsum, g, dq, ws, tiles, cap, st);
 }
 
 cudaError_t launch_simt_bwd_dkdv(const gdpa_problem_t& p, const void* q, const int32_t* offsets,
-                                 const void* k, const void* v, const float* lse,
+                                 const void* k, const void* v, const Bias& bs, const float* lse,
                                  const float* dsum, const void* g, void* dk, void* dv,
                                  WsHeader* ws, cudaStream_t st) {
   if (p.dtype != GDPA_DTYPE_F32) return cudaErrorInvalidValue;
-  GDPA_DISPATCH_DH(p.dh, dkdv_f32, p, q, offsets, k, v, lse, dsum, g, dk, dv, ws, st);
+  GDPA_DISPATCH_DH(p.dh, dkdv_f32, p, q, offsets, k, v, bs, lse, dsum, g, dk, dv, ws, st);
 }
 
 }  // namespace gdpa

@@ -24,8 +24,8 @@ STATUS = {0: "GDPA_OK", 1: "GDPA_ERR_INVALID_ARG", 2: "GDPA_ERR_UNSUPPORTED",
           3: "GDPA_ERR_CUDA", 4: "GDPA_ERR_TIMEOUT", 5: "GDPA_ERR_WORKSPACE"}
 
 EXPORTED = ("gdpa_fwd_workspace_size", "gdpa_bwd_workspace_size", "gdpa_fwd", "gdpa_bwd",
-            "gdpa_workspace_status", "gdpa_status_string", "gdpa_last_launch_count",
-            "gdpa_timing_enable", "gdpa_timing_read")
+            "gdpa_workspace_status", "gdpa_fwd_bias", "gdpa_bwd_bias", "gdpa_status_string",
+            "gdpa_last_launch_count", "gdpa_timing_enable", "gdpa_timing_read")
 
 
 class Problem(ctypes.Structure):
@@ -65,6 +65,9 @@ def load(path: str = LIB_PATH):
     lib.gdpa_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.gdpa_bwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.gdpa_workspace_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
+    lib.gdpa_fwd_bias.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.gdpa_bwd_bias.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                  sz, vp]
     lib.gdpa_status_string.argtypes = [ctypes.c_int]
     lib.gdpa_status_string.restype = ctypes.c_char_p
     lib.gdpa_last_launch_count.restype = ctypes.c_int32
@@ -72,7 +75,7 @@ def load(path: str = LIB_PATH):
     lib.gdpa_timing_enable.restype = ctypes.c_int
     lib.gdpa_timing_read.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int32]
     lib.gdpa_timing_read.restype = ctypes.c_int32
-    for name in EXPORTED[:5]:
+    for name in EXPORTED[:7]:
         getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -160,6 +163,46 @@ def bwd(p: Problem, q, offsets, k, v, o, lse, dout, dq=None, dk=None, dv=None, w
     if rc:
         raise GdpaError(rc, "gdpa_bwd")
     return dq, dk, dv
+
+
+def fwd_bias(p: Problem, q, offsets, k, v, b1=None, b2=None, o=None, lse=None, ws=None,
+             stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Run gdpa_fwd_bias: o = phi(s q k^T + b1) v + b2 (fp32 biases b1 [B,h,m],
+    b2 [B,h,dh], either may be None)."""
+    lib = load()
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and p.phi == PHI_SOFTMAX:
+        lse = torch.empty((p.h, p.total_tokens), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(fwd_workspace_bytes(p), q.device)
+    rc = lib.gdpa_fwd_bias(ctypes.byref(p), _ptr(q), _ptr(offsets), _ptr(k), _ptr(v), _ptr(b1),
+                           _ptr(b2), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise GdpaError(rc, "gdpa_fwd_bias")
+    return o, lse
+
+
+def bwd_bias(p: Problem, q, offsets, k, v, b1, b2, o, lse, dout, dq=None, dk=None, dv=None,
+             db1=None, db2=None, want_bias_grads=True, ws=None, stream=None):
+    """Run gdpa_bwd_bias; returns (dq, dk, dv, db1, db2) (the last two None
+    when ``want_bias_grads`` is False and none were given)."""
+    lib = load()
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if want_bias_grads:
+        B, h, m, dh = k.shape
+        db1 = torch.empty((B, h, m), dtype=torch.float32, device=k.device) if db1 is None else db1
+        db2 = torch.empty((B, h, dh), dtype=torch.float32, device=k.device) if db2 is None else db2
+    if ws is None:
+        ws = workspace(bwd_workspace_bytes(p), q.device)
+    rc = lib.gdpa_bwd_bias(ctypes.byref(p), _ptr(q), _ptr(offsets), _ptr(k), _ptr(v), _ptr(b1),
+                           _ptr(b2), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                           _ptr(db1), _ptr(db2), _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise GdpaError(rc, "gdpa_bwd_bias")
+    return dq, dk, dv, db1, db2
 
 
 def workspace_status(ws: torch.Tensor, stream=None) -> int:

@@ -81,4 +81,7 @@ def test_device_exp2_against_numpy():
     assert rel_fma.max() <= 1.2 * BOUND, rel_fma.max()
     # the polynomial is well below bf16's half-ulp (2^-9), like the hardware unit
     assert rel_mufu.max() <= 2.0 ** -20
-    assert (y_fma.cpu().numpy() == _emulate(x.cpu().numpy())).mean() > 0.99
+    # the device fuses the Horner steps (one rounding per step instead of two),
+    # so it matches the float32 emulation to a few ulps, not bit for bit
+    emu = _emulate(x.cpu().numpy()).astype(np.float64)
+    assert np.max(np.abs(y_fma.cpu().double().numpy() / emu - 1)) <= 2.0 ** -21
