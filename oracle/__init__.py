@@ -143,3 +143,60 @@ def bwd(q, k, v, dout, offsets, phi, scale, nthreads: int = 0, lib=None, b1=None
     if bias_grads:
         return dq, dk, dv, db1, db2
     return dq, dk, dv
+
+
+# --------------------------------------------------------------------------
+# Weight Generation (context vector -> per-sample K or V), weight_gen_oracle.c
+
+_WG_SRC = os.path.join(_HERE, "weight_gen_oracle.c")
+_WG_LIB = os.path.join(_HERE, "libwg_oracle.so")
+_wg_lib = None
+
+
+def wg_load(path: str = None):
+    """Load (building if needed) the Weight Generation oracle library."""
+    global _wg_lib
+    if path is None and _wg_lib is not None:
+        return _wg_lib
+    lib = ctypes.CDLL(build(src=_WG_SRC, out=_WG_LIB) if path is None else path)
+    i32, i64, fp, dp = ctypes.c_int, ctypes.c_int64, ctypes.POINTER(ctypes.c_float), \
+        ctypes.POINTER(ctypes.c_double)
+    lib.wg_oracle_fwd.argtypes = [i32, i64, i32, fp, fp, dp, i32]
+    lib.wg_oracle_fwd.restype = i32
+    lib.wg_oracle_bwd.argtypes = [i32, i64, i32, fp, fp, fp, dp, dp, i32]
+    lib.wg_oracle_bwd.restype = i32
+    if path is None:
+        _wg_lib = lib
+    return lib
+
+
+def weight_gen(w, ctx, nthreads: int = 0, lib=None):
+    """Y [B, F] float64 = ctx [B, C] applied to W [F, C]: Y[b, f] = sum_c W[f, c] ctx[b, c]."""
+    lib = lib or wg_load()
+    w, ctx = _f32(w), _f32(ctx)
+    F, C = w.shape
+    B = ctx.shape[0]
+    assert ctx.shape == (B, C)
+    y = np.zeros((B, F), dtype=np.float64)
+    rc = lib.wg_oracle_fwd(B, F, C, _ptr(w, ctypes.c_float), _ptr(ctx, ctypes.c_float),
+                           _ptr(y, ctypes.c_double), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"wg_oracle_fwd failed with code {rc}")
+    return y
+
+
+def weight_gen_bwd(w, ctx, dy, nthreads: int = 0, lib=None):
+    """(dW [F, C], dctx [B, C]) float64 for an upstream dY [B, F]."""
+    lib = lib or wg_load()
+    w, ctx, dy = _f32(w), _f32(ctx), _f32(dy)
+    F, C = w.shape
+    B = ctx.shape[0]
+    assert dy.shape == (B, F)
+    dw = np.zeros((F, C), dtype=np.float64)
+    dctx = np.zeros((B, C), dtype=np.float64)
+    rc = lib.wg_oracle_bwd(B, F, C, _ptr(w, ctypes.c_float), _ptr(ctx, ctypes.c_float),
+                           _ptr(dy, ctypes.c_float), _ptr(dw, ctypes.c_double),
+                           _ptr(dctx, ctypes.c_double), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"wg_oracle_bwd failed with code {rc}")
+    return dw, dctx

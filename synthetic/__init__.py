@@ -234,16 +234,42 @@ def _gen_rows(key, row_ranges, row_len, std, dtype, device, chunk: int = 1 << 24
     return out
 
 
-def _linear_map_kv(wl: Workload, key_w: int, ctx_key: int, samples, dtype, device):
-    """K_b = reshape(W c_b): fp32 weight [h*m*dh, 64], 64-dim N(0,1) context."""
+CTX_DIM = 64   # context vector length of the linear-map workload
+
+
+def _wg_weight(wl: Workload, key_w: int, device) -> torch.Tensor:
+    """fp32 weight [h*m*dh, 64] of the linear-map recipe, N(0, 1/(64 dh))."""
     rows = wl.h * wl.m * wl.dh
-    wstd = 1.0 / math.sqrt(64.0 * wl.dh)
-    w = _normal_block(key_w, 0, rows * 64, device).mul_(wstd)
-    w = w.to(torch.float32).to(torch.float64).view(rows, 64)        # fp32 weight
-    out = []
-    for b in samples:
-        c = _normal_block(ctx_key, b * 64, 64, device)
-        out.append(round_to(w @ c, dtype))
+    wstd = 1.0 / math.sqrt(CTX_DIM * wl.dh)
+    w = _normal_block(key_w, 0, rows * CTX_DIM, device).mul_(wstd)
+    return w.to(torch.float32).view(rows, CTX_DIM)
+
+
+def _wg_contexts(ctx_key: int, samples, device) -> torch.Tensor:
+    """fp32 N(0, 1) context vectors [len(samples), 64], one per sample."""
+    if not samples:
+        return torch.empty(0, CTX_DIM, dtype=torch.float32, device=device)
+    return torch.stack([_normal_block(ctx_key, b * CTX_DIM, CTX_DIM, device)
+                        for b in samples]).to(torch.float32)
+
+
+def weight_gen_factors(wid: int, which: str = "k", seed: int = 0, samples=None, device="cpu"):
+    """The random numbers of the linear-map recipe: the fp32 weight [h*m*dh, 64]
+    of K (``which="k"``) or V, and the fp32 contexts [len(samples), 64]."""
+    wl = WORKLOADS[wid]
+    sel = list(range(wl.B)) if samples is None else [int(b) for b in samples]
+    key_w = stream_key(seed, wid, T_WK if which == "k" else T_WV)
+    w = _wg_weight(wl, key_w, device)
+    ctx = _wg_contexts(stream_key(seed, wid, T_CTX), sel, device)
+    return w, ctx
+
+
+def _linear_map_kv(wl: Workload, key_w: int, ctx_key: int, samples, dtype, device):
+    """K_b = reshape(W c_b): fp32 weight [h*m*dh, 64], fp32 64-dim N(0,1) context
+    (the workload's input recipe, evaluated in float64 and rounded once)."""
+    w = _wg_weight(wl, key_w, device).to(torch.float64)
+    out = [round_to(w @ c.to(torch.float64), dtype)
+           for c in _wg_contexts(ctx_key, list(samples), device)]
     return torch.cat(out) if out else torch.empty(0, dtype=dtype, device=device)
 
 
