@@ -200,3 +200,68 @@ def weight_gen_bwd(w, ctx, dy, nthreads: int = 0, lib=None):
     if rc != 0:
         raise RuntimeError(f"wg_oracle_bwd failed with code {rc}")
     return dw, dctx
+
+
+# --------------------------------------------------------------------------
+# seed-query attention pooling (first level of HSP), pooling_oracle.c
+
+_POOL_SRC = os.path.join(_HERE, "pooling_oracle.c")
+_POOL_LIB = os.path.join(_HERE, "libpool_oracle.so")
+_pool_lib = None
+
+
+def pool_load(path: str = None):
+    """Load (building if needed) the pooling oracle library."""
+    global _pool_lib
+    if path is None and _pool_lib is not None:
+        return _pool_lib
+    lib = ctypes.CDLL(build(src=_POOL_SRC, out=_POOL_LIB) if path is None else path)
+    i32, i64p, fp, dp, f64 = (ctypes.c_int, ctypes.POINTER(ctypes.c_int64),
+                              ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_double),
+                              ctypes.c_double)
+    lib.pool_oracle_fwd.argtypes = [i32, i32, i32, i32, i64p, fp, fp, fp, f64, dp, dp, i32]
+    lib.pool_oracle_fwd.restype = i32
+    lib.pool_oracle_bwd.argtypes = [i32, i32, i32, i32, i64p, fp, fp, fp, fp, f64, dp, dp, dp,
+                                    i32]
+    lib.pool_oracle_bwd.restype = i32
+    if path is None:
+        _pool_lib = lib
+    return lib
+
+
+def pool_fwd(seeds, k, v, offsets, scale, nthreads: int = 0, lib=None):
+    """(O [B, h, S, dh], LSE [B, h, S]) float64 of seed-query attention pooling."""
+    lib = lib or pool_load()
+    seeds, k, v = _f32(seeds), _f32(k), _f32(v)
+    off = np.ascontiguousarray(offsets, dtype=np.int64)
+    h, S, dh = seeds.shape
+    B = off.shape[0] - 1
+    assert k.shape == (int(off[-1]), h, dh) and v.shape == k.shape
+    o = np.zeros((B, h, S, dh), dtype=np.float64)
+    lse = np.zeros((B, h, S), dtype=np.float64)
+    rc = lib.pool_oracle_fwd(B, h, dh, S, _ptr(off, ctypes.c_int64), _ptr(seeds, ctypes.c_float),
+                             _ptr(k, ctypes.c_float), _ptr(v, ctypes.c_float), float(scale),
+                             _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"pool_oracle_fwd failed with code {rc}")
+    return o, lse
+
+
+def pool_bwd(seeds, k, v, dout, offsets, scale, nthreads: int = 0, lib=None):
+    """(dseeds [h, S, dh], dK [T, h, dh], dV [T, h, dh]) float64."""
+    lib = lib or pool_load()
+    seeds, k, v, g = _f32(seeds), _f32(k), _f32(v), _f32(dout)
+    off = np.ascontiguousarray(offsets, dtype=np.int64)
+    h, S, dh = seeds.shape
+    B = off.shape[0] - 1
+    assert g.shape == (B, h, S, dh)
+    ds = np.zeros((h, S, dh), dtype=np.float64)
+    dk = np.zeros(k.shape, dtype=np.float64)
+    dv = np.zeros(v.shape, dtype=np.float64)
+    rc = lib.pool_oracle_bwd(B, h, dh, S, _ptr(off, ctypes.c_int64), _ptr(seeds, ctypes.c_float),
+                             _ptr(k, ctypes.c_float), _ptr(v, ctypes.c_float),
+                             _ptr(g, ctypes.c_float), float(scale), _ptr(ds, ctypes.c_double),
+                             _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"pool_oracle_bwd failed with code {rc}")
+    return ds, dk, dv
