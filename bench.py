@@ -48,6 +48,7 @@ L2_FLUSH_BYTES = 256 << 20              # > the 126 MB L2
 # algorithmic FLOPs credited to each kernel, in units of T*h*m*dh
 KERNEL_FLOPS = {"gdpa_fwd_sm100": 4, "gdpa_bwd_sm100": 8, "gdpa_simt_fwd": 4,
                 "gdpa_simt_bwd_dq": 4, "gdpa_simt_bwd_dkdv": 4}
+WG_KERNEL = "gdpa_weight_gen"
 TENSOR_KERNELS = {"gdpa_fwd_sm100", "gdpa_bwd_sm100"}
 FWD_KERNELS = {"gdpa_fwd_sm100", "gdpa_simt_fwd"}
 # Source files whose contents decide each fused kernel's DRAM traffic.
@@ -80,6 +81,9 @@ def parse(argv=None):
                     help="passes of the oracle over its fixed sample for cpu_baseline")
     ap.add_argument("--samples", type=int, default=0,
                     help="run only the first N samples of the workload (small profiling case)")
+    ap.add_argument("--weight-gen", action="store_true",
+                    help="linear-map workload only: generate K and V from the context vectors "
+                         "(Weight Generation) inside every step, before the GDPA forward")
     ap.add_argument("--phi", default=None,
                     choices=["identity", "silu", "softmax", "relu", "gelu"],
                     help="the same workload with another activation (the PFFN variants' phi)")
@@ -122,9 +126,10 @@ def fwd_bytes(wl, T):
     return b + (4 * T * wl.h if wl.phi_name == "softmax" else 0)
 
 
-def config_dict(wl, T, n_gpus, subset=None):
+def config_dict(wl, T, n_gpus, subset=None, weight_gen=False):
     """The `config` object of the JSON line (identical in both arms)."""
-    return {"workload": wl.name if subset is None else
+    return {"weight_gen": weight_gen,
+            "workload": wl.name if subset is None else
             f"{wl.name} (first {len(subset)} samples only: profiling case)",
             "B": wl.B if subset is None else len(subset), "h": wl.h, "dh": wl.dh, "m": wl.m,
             "phi": wl.phi_name, "scale": wl.scale, "lengths": wl.lengths,
@@ -364,7 +369,8 @@ def run_reference(args, rank):
           "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
           "ms_per_step": 1e3 * secs / max(args.steps, 1), "higher_is_better": True,
           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-          "config": config_dict(wl, int(lengths.sum()), args.gpus),
+          "config": config_dict(wl, int(lengths.sum()), args.gpus,
+                                weight_gen=bool(getattr(args, "weight_gen", False))),
           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                            "sample": oracle_desc(wl, samples, tokens // max(args.steps, 1))},
           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -418,7 +424,18 @@ def main(argv=None):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     launches = [0]
 
+    wg = None
+    if args.weight_gen:
+        if wl.kv_recipe != "linear_map" or subset is not None:
+            raise SystemExit("bench.py: --weight-gen needs the linear-map workload (2), all samples")
+        wg = {x: syn.weight_gen_factors(wl.wid, x, seed=rank, device=dev) for x in ("k", "v")}
+
     def step():
+        if wg is not None:       # K, V = reshape(W c_b) for every sample, then the GDPA forward
+            G.weight_gen(wg["k"][0], wg["k"][1], y=k.view(wl.B, -1), stream=stream)
+            launches[0] += 1
+            G.weight_gen(wg["v"][0], wg["v"][1], y=v.view(wl.B, -1), stream=stream)
+            launches[0] += 1
         G.fwd(p, q, off, k, v, o=o, lse=lse, ws=ws_f, stream=stream)
         launches[0] += G.last_launch_count()
         if wl.backward:
@@ -499,6 +516,18 @@ def main(argv=None):
     roof = roofline(top)
     fwd_name = next((k_ for k_ in per_kernel if k_ in FWD_KERNELS), None)
     roof_fwd = roofline(fwd_name) if fwd_name else None
+    roof_wg = None
+    if wg is not None and WG_KERNEL in per_kernel:
+        # HBM-bound map: w (fp32) and ctx read, y (bf16) written, per launch
+        nl, tot_ms = per_kernel[WG_KERNEL]
+        avg = tot_ms / max(nl, 1)
+        F = wl.h * wl.m * wl.dh
+        nbytes = F * syn.CTX_DIM * 4 + wl.B * syn.CTX_DIM * 4 + wl.B * F * 2
+        gbs = nbytes / (avg / 1e3) / 1e9
+        roof_wg = {"bound": "hbm", "kernel": WG_KERNEL, "achieved": gbs, "peak": pk["hbm"],
+                   "unit": "GB/s", "frac": gbs / pk["hbm"], "algorithmic_bytes": nbytes,
+                   "launches": nl, "avg_ms": avg, "peak_source": f"{pk['source']} HBM copy",
+                   "tflops": 2.0 * wl.B * F * syn.CTX_DIM / (avg / 1e3) / 1e12}
     kernels = {k_: {"launches": v_[0], "ms": v_[1], "share": v_[1] / max(ms, 1e-9)}
                for k_, v_ in per_kernel.items()}
 
@@ -626,7 +655,7 @@ def main(argv=None):
               "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
               "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
               "vs_baseline": None, "dtype": "f32" if fp32 else "bf16", "data": "synthetic",
-              "config": config_dict(wl, T, world, subset),
+              "config": config_dict(wl, T, world, subset, bool(args.weight_gen)),
               "pct_of_bf16_peak": None if fp32 else 100.0 * value / (world * bf16_peak),
               "bf16_peak": None if fp32 else {"value": bf16_peak, "source": peak_why,
                                               "nominal_at_median_clock": nominal},
@@ -634,7 +663,8 @@ def main(argv=None):
               "fwd_flops_per_step": FLOPS_FWD * unit_flops,
               "bwd_flops_per_step": FLOPS_BWD * unit_flops if wl.backward else 0.0,
               "gpu_launches": n_launch, "kernels": kernels, "roofline": roof,
-              "roofline_fwd": roof_fwd, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk})
+              "roofline_fwd": roof_fwd, "roofline_weight_gen": roof_wg, "cpu_baseline": cpu,
+              "e2e": e2e, "clocks": clk})
     if world > 1:
         dist.destroy_process_group()
 

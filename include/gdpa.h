@@ -169,6 +169,89 @@ GDPA_API gdpa_status_t gdpa_bwd_bias(const gdpa_problem_t* p, const void* q,
                                      size_t workspace_bytes, void* stream);
 
 /*
+ * Weight Generation: each sample's GDPA keys (or values) from its context
+ * vector.  The Kunlun summary (gist.science/es/paper/2602.10016, section 2.1)
+ * lists Weight Generation in the Interaction Block, and the RecSysChannel
+ * review ("Kunlun ... [2/2]", item 1) says that K and V are obtained from the
+ * context features; neither page gives the map.  This library computes its
+ * plainest reading, a learned linear map per output tensor:
+ *
+ *     y[b, f] = sum_c w[f, c] * ctx[b, c],   b < B, f < F,
+ *
+ * rounded to bf16, with y[b] viewed as [h, m, dh] (F = h * m * dh): K or V of
+ * gdpa_fwd for sample b.
+ *   w   fp32 [F, C] (device, 16-byte aligned), C = 32 or 64 (the backward: 64),
+ *       F a multiple of 8.
+ *   ctx fp32 [B, C] (device, 16-byte aligned).
+ *   y   bf16 [B, F] (device, 16-byte aligned): output, every element written.
+ *   status_ws: NULL, or a device buffer of >= 256 bytes, 256-byte aligned,
+ *     whose status word is cleared and receives GDPA_ERR_TIMEOUT if a bounded
+ *     wait inside the kernel expires (read with gdpa_workspace_status).
+ * The products run on the tensor cores in tf32 (10 mantissa bits) with fp32
+ * accumulation.  Returns GDPA_ERR_UNSUPPORTED for another C or F % 8 != 0,
+ * GDPA_ERR_INVALID_ARG for a null or misaligned pointer; asynchronous on
+ * `stream`; allocates nothing.
+ */
+GDPA_API gdpa_status_t gdpa_weight_gen(int32_t B, int64_t F, int32_t C, const float* w,
+                                       const float* ctx, void* y, void* status_ws,
+                                       void* stream);
+
+/* Workspace bytes gdpa_weight_gen_bwd needs (written to *bytes).  Host only. */
+GDPA_API gdpa_status_t gdpa_weight_gen_bwd_workspace_size(int32_t B, int64_t F, int32_t C,
+                                                          size_t* bytes);
+
+/*
+ * Backward of gdpa_weight_gen for an upstream gradient dy of y:
+ *     dw[f, c] = sum_b dy[b, f] * ctx[b, c],   dctx[b, c] = sum_f dy[b, f] * w[f, c].
+ *   w, ctx: the forward's inputs (fp32, device, 16-byte aligned).
+ *   dy bf16 [B, F]: input (e.g. the dk or dv of gdpa_bwd viewed as [B, h*m*dh]).
+ *   dw fp32 [F, C], dctx fp32 [B, C]: outputs (device, 16-byte aligned), every
+ *     element written.
+ *   workspace: device, >= gdpa_weight_gen_bwd_workspace_size bytes, 256-byte
+ *     aligned (bf16 copies of w and ctx, and the status word that a bounded-wait
+ *     expiry sets to GDPA_ERR_TIMEOUT; read with gdpa_workspace_status).
+ * Supported: C = 64, F a multiple of 8, B <= 896 (GDPA_ERR_UNSUPPORTED
+ * otherwise).  The products run on the tensor cores with bf16 operands and
+ * fp32 accumulation; dctx is reduced across CTAs in fp32 in a non-deterministic
+ * order.  Asynchronous on `stream`; allocates nothing.
+ */
+GDPA_API gdpa_status_t gdpa_weight_gen_bwd(int32_t B, int64_t F, int32_t C, const float* w,
+                                           const float* ctx, const void* dy, float* dw,
+                                           float* dctx, void* workspace, size_t workspace_bytes,
+                                           void* stream);
+
+/*
+ * Seed-query attention pooling, the first level of Hierarchical Seed Pooling
+ * (HSP).  The Kunlun summary (section 2.2, HSP bullet) says HSP replaces the
+ * random learnable queries of pooling by multi-head attention with learned
+ * seed-level representations for long sequences (then compressed by
+ * SumKronLinear, which is not part of this call); the RecSysChannel review
+ * (item 3) places it after GDPA.  Read as attention with learned seeds: for
+ * every sample b and head j,
+ *
+ *     O[b, j] = softmax_rows(scale * seeds[j] K_bj^T) V_bj,
+ *     LSE[b, j, i] = ln sum_t exp(scale * seeds[j, i] . k_t)   (natural log),
+ *
+ * with K_bj, V_bj the rows t in [offsets[b], offsets[b+1]) of head j.  A
+ * sample without tokens gets O = 0 and LSE = -inf.
+ *   seeds bf16 [h, S, dh], k and v bf16 [T, h, dh], offsets int32 [B+1]
+ *   (device, as in gdpa_fwd), o bf16 [B, h, S, dh] (output, every element
+ *   written), lse fp32 [B, h, S] (output; may be NULL).  Base pointers 16-byte
+ *   aligned (lse and offsets 4-byte).
+ *   Supported: dh = 32 or 64, 1 <= S <= 128, B <= 4096 (GDPA_ERR_UNSUPPORTED
+ *   otherwise); max_n, total_tokens and the error behaviour as in gdpa_fwd.
+ *   workspace: device, >= gdpa_pool_workspace_size bytes, 256-byte aligned;
+ *   device-detected errors go to its status word (gdpa_workspace_status).
+ */
+GDPA_API gdpa_status_t gdpa_pool_workspace_size(int32_t B, int32_t h, int32_t dh, int32_t S,
+                                                size_t* bytes);
+GDPA_API gdpa_status_t gdpa_pool_fwd(int32_t B, int32_t h, int32_t dh, int32_t S,
+                                     int64_t total_tokens, int32_t max_n, float scale,
+                                     const void* seeds, const int32_t* offsets, const void* k,
+                                     const void* v, void* o, float* lse, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/*
  * Device-detected status of the last gdpa_fwd/gdpa_bwd that used `workspace`
  * (GDPA_OK, GDPA_ERR_INVALID_ARG for inconsistent offsets, GDPA_ERR_TIMEOUT).
  * Synchronises `stream`; writes the code to *status (host).

@@ -51,6 +51,9 @@ cudaError_t launch_sm100_bwd(const gdpa_problem_t& p, const void* q, const int32
                              float* dq_acc, float* dsum, WsHeader* ws, Tile* tiles,
                              cudaStream_t st);
 int64_t sm100_bwd_items(const gdpa_problem_t& p);
+cudaError_t launch_sm100_pool(int B, int h, int dh, int S, int64_t T, float scale,
+                              const void* seeds, const void* k, const void* v, void* o,
+                              float* lse, WsHeader* ws, const Tile* tiles, cudaStream_t st);
 
 namespace {
 
@@ -242,6 +245,55 @@ gdpa_status_t gdpa_bwd(const gdpa_problem_t* p, const void* q, const int32_t* of
                        size_t workspace_bytes, void* stream) {
   return gdpa_bwd_bias(p, q, offsets, k, v, nullptr, nullptr, o, lse, dout, dq, dk, dv, nullptr,
                        nullptr, workspace, workspace_bytes, stream);
+}
+
+namespace {
+// B <= 4096 (the pooling scheduler sorts the samples in one CTA's shared memory)
+gdpa_status_t check_pool(int32_t B, int32_t h, int32_t dh, int32_t S, int64_t T, int32_t max_n,
+                         float scale) {
+  if (B < 1 || h < 1 || S < 1 || max_n < 0 || T < 0 || T >= (int64_t)1 << 31 ||
+      (int64_t)max_n * B < T || !(scale == scale))
+    return GDPA_ERR_INVALID_ARG;
+  if ((dh != 32 && dh != 64) || S > 128 || B > 4096 || (int64_t)B * h >= (int64_t)1 << 24)
+    return GDPA_ERR_UNSUPPORTED;
+  return GDPA_OK;
+}
+size_t pool_ws_bytes(int32_t B, int32_t h) {
+  return align_up(sizeof(WsHeader) + sizeof(Tile) * (size_t)B * ((h + 1) / 2), 256);
+}
+}  // namespace
+
+gdpa_status_t gdpa_pool_workspace_size(int32_t B, int32_t h, int32_t dh, int32_t S,
+                                       size_t* bytes) {
+  const gdpa_status_t s = check_pool(B, h, dh, S, 0, 0, 1.f);
+  if (s != GDPA_OK) return s;
+  if (!bytes) return GDPA_ERR_INVALID_ARG;
+  *bytes = pool_ws_bytes(B, h);
+  return GDPA_OK;
+}
+
+gdpa_status_t gdpa_pool_fwd(int32_t B, int32_t h, int32_t dh, int32_t S, int64_t total_tokens,
+                            int32_t max_n, float scale, const void* seeds,
+                            const int32_t* offsets, const void* k, const void* v, void* o,
+                            float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  g_launches = 0;
+  gdpa_status_t s = check_pool(B, h, dh, S, total_tokens, max_n, scale);
+  if (s != GDPA_OK) return s;
+  const bool empty = total_tokens == 0;
+  if (!offsets || !seeds || !o || (!empty && (!k || !v))) return GDPA_ERR_INVALID_ARG;
+  if (!aligned16(seeds) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      ((uintptr_t)offsets & 3u) || ((uintptr_t)lse & 3u))
+    return GDPA_ERR_INVALID_ARG;
+  s = check_ws(workspace, workspace_bytes, pool_ws_bytes(B, h));
+  if (s != GDPA_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  WsHeader* ws = (WsHeader*)workspace;
+  Tile* tiles = (Tile*)((char*)workspace + sizeof(WsHeader));
+  cudaError_t e = launch_schedule_pool(offsets, B, h, total_tokens, max_n, ws, tiles, st);
+  if (e == cudaSuccess) e = launch_pool_empty(offsets, B, h, S, dh, o, lse, ws, st);
+  if (e == cudaSuccess)
+    e = launch_sm100_pool(B, h, dh, S, total_tokens, scale, seeds, k, v, o, lse, ws, tiles, st);
+  return cuda_status(e);
 }
 
 gdpa_status_t gdpa_workspace_status(const void* workspace, void* stream, int32_t* status) {

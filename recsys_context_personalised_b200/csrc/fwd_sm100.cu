@@ -72,6 +72,7 @@ struct FwdArgs {
   const float* b2;   // [B, h, dh] output bias (may be NULL)
   int64_t T;
   int h, m, nkv;
+  int S;             // seed-query pooling: seeds per head (the output rows of an item)
   float scale;       // s
   float scale_log2;  // s * log2(e)
 };
@@ -135,17 +136,17 @@ __device__ __forceinline__ Pair load_pair(const Tile* tiles, int count, int p) {
 }
 
 // Epilogue of one activation warp (TMEM lane quadrant `quad`, lane = tile
-// row): its 32 O rows, times `inv`, rounded to bf16 and stored to o [T, h, DH]
-// for the rows the tile owns.  The rows pass through the warp's own 4 KB of
+// row): its 32 O rows, times `inv`, rounded to bf16 and stored to row r <
+// nrows of the tile at obase + r * row_stride.  The rows pass through the warp's own 4 KB of
 // shared memory (`ostg`; 64 columns at a time, 16-byte chunks swizzled by
 // row) so that every global store instruction writes whole rows: CPR lanes
 // per row, 32 / CPR rows per instruction.  Arrives on `oempty` (the O
 // accumulator is free) right after the last TMEM read, before the stores.
 // `b2row` (DH values, or NULL) is the output bias added to every row.
 template <int DH>
-__device__ __forceinline__ void store_o_rows(uint32_t my_o, uint32_t ostg, float inv,
-                                             const Tile& tl, int quad, int lane,
-                                             __nv_bfloat16* o, int h, uint32_t oempty,
+__device__ __forceinline__ void store_o_rows(uint32_t my_o, uint32_t ostg, float inv, int nrows,
+                                             int quad, int lane, __nv_bfloat16* obase,
+                                             int64_t row_stride, uint32_t oempty,
                                              const float* b2row = nullptr) {
   constexpr int PC = DH < 64 ? DH : 64;           // columns per pass
   constexpr int CPR = PC / 8;                     // 16-byte chunks per row
@@ -193,9 +194,7 @@ __device__ __forceinline__ void store_o_rows(uint32_t my_o, uint32_t ostg, float
                    : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
                    : "r"(chunk_addr(r, jl)));
       const int tr = quad * 32 + r;                 // tile row
-      if (tr < tl.rows)
-        *reinterpret_cast<uint4*>(o + ((int64_t)(tl.row0 + tr) * h + tl.head) * DH + c0 +
-                                  jl * 8) = val;
+      if (tr < nrows) *reinterpret_cast<uint4*>(obase + (int64_t)tr * row_stride + c0 + jl * 8) = val;
     }
     __syncwarp();
   }
@@ -629,8 +628,9 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       tc_fence_after();
       const float inv = SOFTMAX ? 1.f / l_run : 1.f;
       const bool store = row < tl.rows;
-      store_o_rows<DH>(my_o, base + C::OFF_OSTG + (uint32_t)(warp - 4) * C::OSTG_WARP, inv, tl,
-                       quad, lane, a.o, a.h, bar(C::B_OEMPTY + grp),
+      store_o_rows<DH>(my_o, base + C::OFF_OSTG + (uint32_t)(warp - 4) * C::OSTG_WARP, inv,
+                       tl.rows, quad, lane, a.o + ((int64_t)tl.row0 * a.h + tl.head) * DH,
+                       (int64_t)a.h * DH, bar(C::B_OEMPTY + grp),
                        BIAS && a.b2 ? a.b2 + ((int64_t)tl.b * a.h + tl.head) * DH : nullptr);
       if (SOFTMAX && store && a.lse != nullptr)
         a.lse[(int64_t)tl.head * a.T + tl.row0 + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
@@ -712,13 +712,14 @@ __device__ __forceinline__ float row_extreme(const uint32_t (&s)[128]) {
   return NEG ? fmin3(fminf(e[0], e[1]), e[2], e[3]) : fmax3(fmaxf(e[0], e[1]), e[2], e[3]);
 }
 
-template <int DH, int PHI, bool BIAS>
+template <int DH, int PHI, bool BIAS, bool POOL>
 __global__ void __launch_bounds__(kThreads, 1)
 gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
   using C = FwdCfg<DH>;
   static_assert(C::P_SEP, "needs P in TMEM columns of its own");
+  static_assert(!POOL || (PHI == GDPA_PHI_SOFTMAX && !BIAS), "pooling is softmax attention");
   constexpr bool SOFTMAX = PHI == GDPA_PHI_SOFTMAX;
   constexpr uint32_t IDESC_S = idesc_bf16(128, 128, 0, 0);
   constexpr uint32_t IDESC_O = idesc_bf16(128, DH, 0, 1);
@@ -769,9 +770,26 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int count = a.ws->tile_count;
-  const int npairs = (count + 1) >> 1;
-  const int nkv = a.nkv;
   const int stride = gridDim.x;
+  // GDPA: work item p = query tiles 2p, 2p+1 of the jagged tile list, all with
+  // a.nkv key blocks of a.m keys.  Seed-query pooling (POOL): item p = heads
+  // (2k, 2k+1) of one sample, the seeds of each head as the 128-row query
+  // tile, the sample's n_b tokens as ceil(n_b / 128) key blocks.
+  const int npairs = POOL ? count : (count + 1) >> 1;
+  auto get_pair = [&](int p) -> Pair {
+    if constexpr (POOL) {
+      Pair r;
+      r.a = a.tiles[p];
+      r.has_b = r.a.head + 1 < a.h;
+      r.b = r.a;
+      r.b.head = r.a.head + 1;
+      r.share = false;
+      return r;
+    } else {
+      return load_pair(a.tiles, count, p);
+    }
+  };
+  auto pair_nkv = [&](const Pair& pr) -> int { return POOL ? (pr.a.rows + 127) >> 7 : a.nkv; };
 
   if (warp < 4) {
     setmaxnreg_dec<80>();
@@ -786,9 +804,14 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
         if (!mbar_wait(bar(C::B_KVEMPTY + slot), sphase ^ 1u, abort_flag, kTimeoutNs)) return false;
         mbar_expect_tx(bar(C::B_KVFULL + slot), C::TILEB);
 #pragma unroll
-        for (int c = 0; c < C::NCH; ++c)
-          tma_load_4d(sKV + slot * C::TILEB + c * C::CHUNKB, map, bar(C::B_KVFULL + slot),
-                      c * C::CH, j * C::BN, tl.head, tl.b);
+        for (int c = 0; c < C::NCH; ++c) {
+          if constexpr (POOL)   // tokens [T, h, dh]: rows past the sample are masked later
+            tma_load_3d(sKV + slot * C::TILEB + c * C::CHUNKB, map, bar(C::B_KVFULL + slot),
+                        c * C::CH, tl.head, tl.row0 + j * C::BN);
+          else
+            tma_load_4d(sKV + slot * C::TILEB + c * C::CHUNKB, map, bar(C::B_KVFULL + slot),
+                        c * C::CH, j * C::BN, tl.head, tl.b);
+        }
         if (++slot == (uint32_t)C::NS) {
           slot = 0;
           sphase ^= 1u;
@@ -806,28 +829,37 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
         mbar_expect_tx(bar(C::B_QFULL + qs), (pr.has_b ? 2u : 1u) * C::TILEB);
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
-          tma_load_3d(qaddr + c * C::CHUNKB, &tmQ, bar(C::B_QFULL + qs), c * C::CH, pr.a.head,
-                      pr.a.row0);
-          if (pr.has_b)
-            tma_load_3d(qaddr + C::TILEB + c * C::CHUNKB, &tmQ, bar(C::B_QFULL + qs), c * C::CH,
-                        pr.b.head, pr.b.row0);
+          if constexpr (POOL) {   // seeds [h, S, dh] of heads a, b; rows >= S read as zero
+            tma_load_3d(qaddr + c * C::CHUNKB, &tmQ, bar(C::B_QFULL + qs), c * C::CH, 0,
+                        pr.a.head);
+            if (pr.has_b)
+              tma_load_3d(qaddr + C::TILEB + c * C::CHUNKB, &tmQ, bar(C::B_QFULL + qs),
+                          c * C::CH, 0, pr.b.head);
+          } else {
+            tma_load_3d(qaddr + c * C::CHUNKB, &tmQ, bar(C::B_QFULL + qs), c * C::CH, pr.a.head,
+                        pr.a.row0);
+            if (pr.has_b)
+              tma_load_3d(qaddr + C::TILEB + c * C::CHUNKB, &tmQ, bar(C::B_QFULL + qs),
+                          c * C::CH, pr.b.head, pr.b.row0);
+          }
         }
         return true;
       };
       int p = blockIdx.x;
       bool ok = p < npairs;
       if (ok) {
-        const Pair pr = load_pair(a.tiles, count, p);
+        const Pair pr = get_pair(p);
         ok = load_q(pr, 0) && load_both(&tmK, pr, 0);
       }
       for (uint32_t ic = 0; ok && p < npairs; p += stride, ++ic) {
-        const Pair pr = load_pair(a.tiles, count, p);
+        const Pair pr = get_pair(p);
+        const int nkv = pair_nkv(pr);
         const bool has_next = p + stride < npairs;
         for (int j = 0; ok && j < nkv; ++j) {
           if (j + 1 < nkv) {
             ok = load_both(&tmK, pr, j + 1);
           } else if (has_next) {
-            const Pair pn = load_pair(a.tiles, count, p + stride);
+            const Pair pn = get_pair(p + stride);
             ok = load_q(pn, ic + 1) && load_both(&tmK, pn, 0);
           }
           if (ok) ok = load_both(&tmV, pr, j);
@@ -873,7 +905,7 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
       };
       auto issue_s_pair = [&](const Pair& pr, uint32_t qs, int j) -> bool {
         const bool sep = !pr.share;
-        const bool last = j == nkv - 1;
+        const bool last = j == pair_nkv(pr) - 1;
         const int ka = take();
         if (ka < 0 || !issue_s(0, qs, ka, last && !pr.has_b)) return false;
         if (!pr.has_b || sep) release(ka);
@@ -886,7 +918,7 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
       };
       // O_x += P_x V once the group has written P_x; PFREE_x reports that P_x
       // has been read, OFULL_x (last key block) that O_x is complete.
-      auto issue_pv = [&](int x, int vs, int j) -> bool {
+      auto issue_pv = [&](int x, int vs, int j, int nkv) -> bool {
         if (!mbar_wait(bar(C::B_PFULL + x), pv_cnt[x] & 1u, abort_flag, kTimeoutNs)) return false;
         ++pv_cnt[x];
         if (j == 0 &&
@@ -909,30 +941,32 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
       };
       auto issue_pv_pair = [&](const Pair& pr, int j) -> bool {
         const bool sep = !pr.share;
+        const int nkv = pair_nkv(pr);
         const int va = take();
-        if (va < 0 || !issue_pv(0, va, j)) return false;
+        if (va < 0 || !issue_pv(0, va, j, nkv)) return false;
         if (!pr.has_b || sep) release(va);
         if (pr.has_b) {
           const int vb = sep ? take() : va;
-          if (vb < 0 || !issue_pv(1, vb, j)) return false;
+          if (vb < 0 || !issue_pv(1, vb, j, nkv)) return false;
           release(vb);
         }
         return true;
       };
       int p = blockIdx.x;
       if (p < npairs) {
-        const Pair pr = load_pair(a.tiles, count, p);
+        const Pair pr = get_pair(p);
         ok = mbar_wait(bar(C::B_QFULL + 0), 0u, abort_flag, kTimeoutNs) && issue_s_pair(pr, 0, 0);
       }
       for (uint32_t ic = 0; ok && p < npairs; p += stride, ++ic) {
-        const Pair pr = load_pair(a.tiles, count, p);
+        const Pair pr = get_pair(p);
+        const int nkv = pair_nkv(pr);
         const uint32_t qs = ic % C::QST;
         const bool has_next = p + stride < npairs;
         for (int j = 0; ok && j < nkv; ++j) {
           if (j + 1 < nkv) {
             ok = issue_s_pair(pr, qs, j + 1);
           } else if (has_next) {
-            const Pair pn = load_pair(a.tiles, count, p + stride);
+            const Pair pn = get_pair(p + stride);
             const uint32_t qn = (ic + 1) % C::QST, qph = ((ic + 1) / C::QST) & 1u;
             ok = mbar_wait(bar(C::B_QFULL + qn), qph, abort_flag, kTimeoutNs) &&
                  issue_s_pair(pn, qn, 0);
@@ -957,10 +991,13 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
     uint32_t sc = 0, oc = 0;
     bool ok = true;
     for (int p = blockIdx.x; ok && p < npairs; p += stride) {
-      const Pair pr = load_pair(a.tiles, count, p);
+      const Pair pr = get_pair(p);
       if (grp == 1 && !pr.has_b) continue;
       const Tile tl = grp ? pr.b : pr.a;
-      if (quad * 32 >= tl.rows) {
+      const int nkv = pair_nkv(pr);
+      const int kv_len = POOL ? tl.rows : a.m;          // keys of the item
+      const int out_rows = POOL ? a.S : tl.rows;        // output rows of the item
+      if (quad * 32 >= out_rows) {
         // every row of this warp lies past the tile's rows: those rows of O are
         // never stored, so the warp computes nothing and only keeps its part
         // in every barrier of the item
@@ -1019,7 +1056,7 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar(C::B_SFREE + grp));      // S_x may be overwritten now
-        const int valid = min(C::BN, a.m - j * C::BN);
+        const int valid = min(C::BN, kv_len - j * C::BN);
         if constexpr (BIAS) {
           // s := s * mul + b1 (mul: s log2 e for softmax, s / 2 for SiLU, s
           // otherwise); the activation below then takes mul = 1
@@ -1162,11 +1199,18 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
       tc_fence_after();
       ++oc;
       const float inv = SOFTMAX ? 1.f / l_run : 1.f;
-      store_o_rows<DH>(my_o, base + C::OFF_OSTG + (uint32_t)(warp - 4) * C::OSTG_WARP, inv, tl,
-                       quad, lane, a.o, a.h, bar(C::B_OEMPTY + grp),
+      // GDPA: rows of the tile in o [T, h, DH]; pooling: the seeds of (b, head) in o [B, h, S, DH]
+      __nv_bfloat16* obase = POOL ? a.o + ((int64_t)tl.b * a.h + tl.head) * a.S * DH
+                                  : a.o + ((int64_t)tl.row0 * a.h + tl.head) * DH;
+      store_o_rows<DH>(my_o, base + C::OFF_OSTG + (uint32_t)(warp - 4) * C::OSTG_WARP, inv,
+                       out_rows, quad, lane, obase, POOL ? (int64_t)DH : (int64_t)a.h * DH,
+                       bar(C::B_OEMPTY + grp),
                        BIAS && a.b2 ? a.b2 + ((int64_t)tl.b * a.h + tl.head) * DH : nullptr);
-      if (SOFTMAX && row < tl.rows && a.lse != nullptr)
-        a.lse[(int64_t)tl.head * a.T + tl.row0 + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      if (SOFTMAX && row < out_rows && a.lse != nullptr) {
+        const int64_t at = POOL ? ((int64_t)tl.b * a.h + tl.head) * a.S + row
+                                : (int64_t)tl.head * a.T + tl.row0 + row;
+        a.lse[at] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      }
     }
   }
 
@@ -1228,7 +1272,7 @@ bool make_maps(const gdpa_problem_t& p, const void* q, const void* k, const void
 template <int DH, int PHI, bool BIAS>
 constexpr auto fwd_kernel() {
   if constexpr (DH <= 64)
-    return gdpa_fwd_early_kernel<DH, PHI, BIAS>;
+    return gdpa_fwd_early_kernel<DH, PHI, BIAS, false>;
   else
     return gdpa_fwd_sm100_kernel<DH, PHI, BIAS>;
 }
@@ -1243,7 +1287,7 @@ cudaError_t launch_fwd_t(const gdpa_problem_t& p, const void* q, const void* k, 
   auto kern = fwd_kernel<DH, PHI, BIAS>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
-  FwdArgs args;
+  FwdArgs args = {};
   args.tiles = tiles;
   args.ws = ws;
   args.o = reinterpret_cast<__nv_bfloat16*>(o);
@@ -1284,6 +1328,56 @@ cudaError_t launch_fwd_bias(const gdpa_problem_t& p, const void* q, const void* 
   return launch_fwd_dh<DH, false>(p, q, k, v, bs, o, lse, ws, tiles, st);
 }
 
+// Seed-query pooling on the dh <= 64 forward kernel: seeds [h, S, DH] as the
+// query tiles (rows >= S read as zero), the jagged tokens [T, h, DH] as keys
+// and values, softmax over each sample's tokens.
+template <int DH>
+cudaError_t launch_pool_t(int B, int h, int S, int64_t T, float scale, const void* seeds,
+                          const void* k, const void* v, void* o, float* lse, WsHeader* ws,
+                          const Tile* tiles, cudaStream_t st) {
+  using C = FwdCfg<DH>;
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorInvalidValue;
+  const CUtensorMapSwizzle sw = DH < 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUtensorMap mq, mk, mv;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)DH, (cuuint64_t)S, (cuuint64_t)h};
+    const cuuint64_t strides[2] = {(cuuint64_t)DH * 2, (cuuint64_t)S * DH * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)C::CH, 128, 1};
+    if (enc(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(seeds), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  const cuuint64_t dims[3] = {(cuuint64_t)DH, (cuuint64_t)h, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)DH * 2, (cuuint64_t)h * DH * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)C::CH, 1, 128};
+  for (int i = 0; i < 2; ++i)
+    if (enc(i ? &mv : &mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(i ? v : k), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  auto kern = gdpa_fwd_early_kernel<DH, GDPA_PHI_SOFTMAX, false, true>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return e;
+  FwdArgs args = {};
+  args.tiles = tiles;
+  args.ws = ws;
+  args.o = reinterpret_cast<__nv_bfloat16*>(o);
+  args.lse = lse;
+  args.T = T;
+  args.h = h;
+  args.m = 0;
+  args.nkv = 0;
+  args.S = S;
+  args.scale = scale;
+  args.scale_log2 = scale * 1.4426950408889634f;
+  KernelScope ks_("gdpa_pool_fwd_sm100", st);
+  kern<<<device_sm_count(), kThreads, C::SMEM, st>>>(mq, mk, mv, args);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_sm100_fwd(const gdpa_problem_t& p, const void* q, const void* k,
@@ -1296,6 +1390,15 @@ cudaError_t launch_sm100_fwd(const gdpa_problem_t& p, const void* q, const void*
     case 128: return launch_fwd_bias<128>(p, q, k, v, bs, o, lse, ws, tiles, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_sm100_pool(int B, int h, int dh, int S, int64_t T, float scale,
+                              const void* seeds, const void* k, const void* v, void* o,
+                              float* lse, WsHeader* ws, const Tile* tiles, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  if (dh == 32) return launch_pool_t<32>(B, h, S, T, scale, seeds, k, v, o, lse, ws, tiles, st);
+  if (dh == 64) return launch_pool_t<64>(B, h, S, T, scale, seeds, k, v, o, lse, ws, tiles, st);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace gdpa

@@ -71,6 +71,13 @@ cudaError_t launch_schedule(const gdpa_problem_t& p, const int32_t* offsets, int
 cudaError_t launch_schedule_kv(const gdpa_problem_t& p, const int32_t* offsets, WsHeader* ws,
                                Tile* tiles, cudaStream_t st);
 
+// Seed-pooling work list (one item per (sample with tokens, pair of heads),
+// longest first; B <= 4096) and the outputs of samples without tokens.
+cudaError_t launch_schedule_pool(const int32_t* offsets, int B, int h, int64_t T, int max_n,
+                                 WsHeader* ws, Tile* tiles, cudaStream_t st);
+cudaError_t launch_pool_empty(const int32_t* offsets, int B, int h, int S, int dh, void* o,
+                              float* lse, const WsHeader* ws, cudaStream_t st);
+
 // SIMT kernels (fp32 problems only; fp32 math).
 cudaError_t launch_simt_fwd(const gdpa_problem_t& p, const void* q, const void* k,
                             const void* v, const Bias& bs, void* o, float* lse, WsHeader* ws,

@@ -149,6 +149,92 @@ schedule_kv_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T,
   if (tid == 0) ws->tile_count = (int)((long long)B * per_sample);
 }
 
+
+// Seed-pooling work list: one item per (sample, pair of heads 2k, 2k+1) of the
+// samples that have tokens, longest samples first (B <= 4096): item fields
+// b, head = 2k, row0 = offsets[b], rows = n_b.  Samples without tokens get no
+// item (pool_empty_kernel writes their outputs).
+__global__ void __launch_bounds__(kSchedThreads)
+schedule_pool_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T, int max_n,
+                     WsHeader* ws, Tile* __restrict__ tiles) {
+  __shared__ int s_bad;
+  __shared__ int s_nz;
+  __shared__ int2 s_key[kSortMax];   // (n_b, b)
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    s_bad = 0;
+    s_nz = 0;
+    ws->status = GDPA_OK;
+    if (offsets[0] != 0 || (int64_t)offsets[B] != T) s_bad = 1;
+  }
+  __syncthreads();
+  for (int b = tid; b < B; b += kSchedThreads) {
+    const int n = offsets[b + 1] - offsets[b];
+    if (n < 0 || n > max_n) s_bad = 1;
+    if (n > 0) atomicAdd(&s_nz, 1);
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (tid == 0) {
+      ws->status = GDPA_ERR_INVALID_ARG;
+      ws->tile_count = 0;
+    }
+    return;
+  }
+  int P2 = 1;
+  while (P2 < B) P2 <<= 1;
+  for (int i = tid; i < P2; i += kSchedThreads)
+    s_key[i] = i < B ? make_int2(offsets[i + 1] - offsets[i], i) : make_int2(-1, 0x7fffffff);
+  __syncthreads();
+  // bitonic sort: descending n, ascending b (samples without tokens sort last)
+  for (int k = 2; k <= P2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < P2; i += kSchedThreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const int2 x = s_key[i], y = s_key[ixj];
+          const bool x_first = x.x > y.x || (x.x == y.x && x.y < y.y);
+          const bool up = (i & k) == 0;
+          if (up ? !x_first : x_first) {
+            s_key[i] = y;
+            s_key[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const int hp = (h + 1) / 2;
+  const long long items = (long long)s_nz * hp;
+  for (long long idx = tid; idx < items; idx += kSchedThreads) {
+    const int b = s_key[(int)(idx / hp)].y;
+    Tile w;
+    w.b = b;
+    w.head = 2 * (int)(idx % hp);
+    w.row0 = offsets[b];
+    w.rows = offsets[b + 1] - offsets[b];
+    tiles[idx] = w;
+  }
+  if (tid == 0) ws->tile_count = (int)items;
+}
+
+// Outputs of the samples without tokens: O = 0 and LSE = -inf (every seed
+// pools over an empty set).  One thread per 8 columns of an output row.
+__global__ void pool_empty_kernel(const int32_t* __restrict__ offsets, int B, int h, int S,
+                                  int dh, uint4* __restrict__ o, float* __restrict__ lse,
+                                  const WsHeader* __restrict__ ws) {
+  if (ws->status == GDPA_ERR_INVALID_ARG) return;
+  const int per_row = dh / 8;
+  const int64_t n = (int64_t)B * h * S * per_row;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const int64_t row = i / per_row;                  // (b, head, seed)
+    const int b = (int)(row / ((int64_t)h * S));
+    if (offsets[b + 1] != offsets[b]) continue;
+    o[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (lse != nullptr && i % per_row == 0) lse[row] = -INFINITY;
+  }
+}
 }  // namespace
 
 cudaError_t launch_schedule_kv(const gdpa_problem_t& p, const int32_t* offsets, WsHeader* ws,
@@ -164,6 +250,28 @@ cudaError_t launch_schedule(const gdpa_problem_t& p, const int32_t* offsets, int
   KernelScope ks_("gdpa_schedule", st);
   schedule_kernel<<<1, kSchedThreads, 0, st>>>(offsets, p.B, p.h, p.total_tokens, p.max_n,
                                                 bm, ws, tiles, tile_capacity(p, bm));
+  return cudaGetLastError();
+}
+
+}  // namespace gdpa
+
+namespace gdpa {
+
+cudaError_t launch_schedule_pool(const int32_t* offsets, int B, int h, int64_t T, int max_n,
+                                 WsHeader* ws, Tile* tiles, cudaStream_t st) {
+  KernelScope ks_("gdpa_schedule_pool", st);
+  schedule_pool_kernel<<<1, kSchedThreads, 0, st>>>(offsets, B, h, T, max_n, ws, tiles);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pool_empty(const int32_t* offsets, int B, int h, int S, int dh, void* o,
+                              float* lse, const WsHeader* ws, cudaStream_t st) {
+  const int64_t n = (int64_t)B * h * S * (dh / 8);
+  if (n == 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  KernelScope ks_("gdpa_pool_empty", st);
+  pool_empty_kernel<<<(unsigned)blocks, 256, 0, st>>>(offsets, B, h, S, dh, (uint4*)o, lse, ws);
   return cudaGetLastError();
 }
 

@@ -24,7 +24,8 @@ STATUS = {0: "GDPA_OK", 1: "GDPA_ERR_INVALID_ARG", 2: "GDPA_ERR_UNSUPPORTED",
           3: "GDPA_ERR_CUDA", 4: "GDPA_ERR_TIMEOUT", 5: "GDPA_ERR_WORKSPACE"}
 
 EXPORTED = ("gdpa_fwd_workspace_size", "gdpa_bwd_workspace_size", "gdpa_fwd", "gdpa_bwd",
-            "gdpa_workspace_status", "gdpa_fwd_bias", "gdpa_bwd_bias", "gdpa_status_string",
+            "gdpa_workspace_status", "gdpa_fwd_bias", "gdpa_bwd_bias", "gdpa_weight_gen",
+            "gdpa_status_string",
             "gdpa_last_launch_count", "gdpa_timing_enable", "gdpa_timing_read")
 
 
@@ -75,7 +76,21 @@ def load(path: str = LIB_PATH):
     lib.gdpa_timing_enable.restype = ctypes.c_int
     lib.gdpa_timing_read.argtypes = [ctypes.POINTER(KernelTime), ctypes.c_int32]
     lib.gdpa_timing_read.restype = ctypes.c_int32
-    for name in EXPORTED[:7]:
+    lib.gdpa_weight_gen.argtypes = [ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, vp, vp, vp,
+                                    vp, vp]
+    lib.gdpa_weight_gen_bwd_workspace_size.argtypes = [ctypes.c_int32, ctypes.c_int64,
+                                                       ctypes.c_int32, ctypes.POINTER(sz)]
+    lib.gdpa_weight_gen_bwd_workspace_size.restype = ctypes.c_int
+    lib.gdpa_weight_gen_bwd.argtypes = [ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, vp, vp,
+                                        vp, vp, vp, vp, sz, vp]
+    lib.gdpa_weight_gen_bwd.restype = ctypes.c_int
+    i32 = ctypes.c_int32
+    lib.gdpa_pool_workspace_size.argtypes = [i32, i32, i32, i32, ctypes.POINTER(sz)]
+    lib.gdpa_pool_workspace_size.restype = ctypes.c_int
+    lib.gdpa_pool_fwd.argtypes = [i32, i32, i32, i32, ctypes.c_int64, i32, ctypes.c_float, vp, vp,
+                                  vp, vp, vp, vp, vp, sz, vp]
+    lib.gdpa_pool_fwd.restype = ctypes.c_int
+    for name in EXPORTED[:8]:
         getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -203,6 +218,67 @@ def bwd_bias(p: Problem, q, offsets, k, v, b1, b2, o, lse, dout, dq=None, dk=Non
     if rc:
         raise GdpaError(rc, "gdpa_bwd_bias")
     return dq, dk, dv, db1, db2
+
+
+def weight_gen(w: torch.Tensor, ctx: torch.Tensor, y: Optional[torch.Tensor] = None,
+               status_ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Run gdpa_weight_gen: y [B, F] bf16 = ctx [B, C] applied to w [F, C] (fp32)."""
+    F, C = w.shape
+    B = ctx.shape[0]
+    if y is None:
+        y = torch.empty((B, F), dtype=torch.bfloat16, device=w.device)
+    rc = load().gdpa_weight_gen(B, F, C, _ptr(w), _ptr(ctx), _ptr(y), _ptr(status_ws),
+                                _stream(stream))
+    if rc:
+        raise GdpaError(rc, "gdpa_weight_gen")
+    return y
+
+
+def weight_gen_bwd(w: torch.Tensor, ctx: torch.Tensor, dy: torch.Tensor, ws=None, stream=None):
+    """Run gdpa_weight_gen_bwd; returns (dw [F, C], dctx [B, C]) in fp32."""
+    lib = load()
+    F, C = w.shape
+    B = ctx.shape[0]
+    n = ctypes.c_size_t()
+    rc = lib.gdpa_weight_gen_bwd_workspace_size(B, F, C, ctypes.byref(n))
+    if rc:
+        raise GdpaError(rc, "gdpa_weight_gen_bwd_workspace_size")
+    if ws is None:
+        ws = workspace(n.value, w.device)
+    dw = torch.empty((F, C), dtype=torch.float32, device=w.device)
+    dctx = torch.empty((B, C), dtype=torch.float32, device=w.device)
+    rc = lib.gdpa_weight_gen_bwd(B, F, C, _ptr(w), _ptr(ctx), _ptr(dy), _ptr(dw), _ptr(dctx),
+                                 _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise GdpaError(rc, "gdpa_weight_gen_bwd")
+    return dw, dctx
+
+
+def pool_fwd(seeds: torch.Tensor, offsets, k: torch.Tensor, v: torch.Tensor, scale: float,
+             offsets_host, o=None, lse=None, ws=None, stream=None, want_lse=True):
+    """Run gdpa_pool_fwd (seed-query attention pooling): seeds [h, S, dh],
+    jagged k, v [T, h, dh] with device ``offsets`` (host copy ``offsets_host``
+    for T and max_n); returns (o [B, h, S, dh], lse [B, h, S] or None)."""
+    lib = load()
+    h, S, dh = seeds.shape
+    off = [int(x) for x in offsets_host]
+    B, T = len(off) - 1, off[-1]
+    max_n = max((off[i + 1] - off[i] for i in range(B)), default=0)
+    if o is None:
+        o = torch.empty((B, h, S, dh), dtype=seeds.dtype, device=seeds.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, h, S), dtype=torch.float32, device=seeds.device)
+    if ws is None:
+        n = ctypes.c_size_t()
+        rc = lib.gdpa_pool_workspace_size(B, h, dh, S, ctypes.byref(n))
+        if rc:
+            raise GdpaError(rc, "gdpa_pool_workspace_size")
+        ws = workspace(n.value, seeds.device)
+    rc = lib.gdpa_pool_fwd(B, h, dh, S, T, max_n, scale, _ptr(seeds), _ptr(offsets), _ptr(k),
+                           _ptr(v), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise GdpaError(rc, "gdpa_pool_fwd")
+    return o, lse
 
 
 def workspace_status(ws: torch.Tensor, stream=None) -> int:

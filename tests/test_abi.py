@@ -97,3 +97,19 @@ def test_selftest_rejects_bad_arguments():
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(ImportError):
         G.load(str(tmp_path / "libgdpa.so"))
+
+
+def test_weight_gen_rejects_unsupported_shapes_on_host():
+    import ctypes
+    lib = pkg.load()
+    n = ctypes.c_size_t()
+    assert lib.gdpa_weight_gen_bwd_workspace_size(100, 1024, 32, ctypes.byref(n)) == 2
+    assert lib.gdpa_weight_gen_bwd_workspace_size(897, 1024, 64, ctypes.byref(n)) == 2
+    assert lib.gdpa_weight_gen_bwd_workspace_size(100, 1020, 64, ctypes.byref(n)) == 2
+    assert lib.gdpa_weight_gen_bwd_workspace_size(100, 1024, 64, ctypes.byref(n)) == 0
+    assert n.value >= 256 + 1024 * 64 * 2 + 100 * 64 * 2
+    # argument checks come before any CUDA call
+    assert lib.gdpa_weight_gen(4, 64, 48, 4096, 4096, 4096, None, None) == 2
+    assert lib.gdpa_weight_gen(4, 60, 64, 4096, 4096, 4096, None, None) == 2
+    assert lib.gdpa_weight_gen(4, 64, 64, None, 4096, 4096, None, None) == 1
+    assert lib.gdpa_weight_gen(4, 64, 64, 4100, 4096, 4096, None, None) == 1
