@@ -265,3 +265,66 @@ def pool_bwd(seeds, k, v, dout, offsets, scale, nthreads: int = 0, lib=None):
     if rc != 0:
         raise RuntimeError(f"pool_oracle_bwd failed with code {rc}")
     return ds, dk, dv
+
+
+# --------------------------------------------------------------------------
+# sliding-window self-attention on the jagged sequence, window_oracle.c
+
+_WIN_SRC = os.path.join(_HERE, "window_oracle.c")
+_WIN_LIB = os.path.join(_HERE, "libwin_oracle.so")
+_win_lib = None
+
+
+def win_load(path: str = None):
+    """Load (building if needed) the sliding-window oracle library."""
+    global _win_lib
+    if path is None and _win_lib is not None:
+        return _win_lib
+    lib = ctypes.CDLL(build(src=_WIN_SRC, out=_WIN_LIB) if path is None else path)
+    i32, i64p, fp, dp, f64 = (ctypes.c_int, ctypes.POINTER(ctypes.c_int64),
+                              ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_double),
+                              ctypes.c_double)
+    lib.win_oracle_fwd.argtypes = [i32, i32, i32, i32, i64p, fp, fp, fp, f64, dp, dp, i32]
+    lib.win_oracle_fwd.restype = i32
+    lib.win_oracle_bwd.argtypes = [i32, i32, i32, i32, i64p, fp, fp, fp, fp, f64, dp, dp, dp, i32]
+    lib.win_oracle_bwd.restype = i32
+    if path is None:
+        _win_lib = lib
+    return lib
+
+
+def win_fwd(q, k, v, offsets, window, scale, nthreads: int = 0, lib=None):
+    """(O [T, h, dh], LSE [h, T]) float64 of causal sliding-window attention."""
+    lib = lib or win_load()
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    off = np.ascontiguousarray(offsets, dtype=np.int64)
+    T, h, dh = q.shape
+    B = off.shape[0] - 1
+    assert k.shape == q.shape and v.shape == q.shape and int(off[-1]) == T
+    o = np.zeros((T, h, dh), dtype=np.float64)
+    lse = np.zeros((h, T), dtype=np.float64)
+    rc = lib.win_oracle_fwd(B, h, dh, int(window), _ptr(off, ctypes.c_int64),
+                            _ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                            _ptr(v, ctypes.c_float), float(scale), _ptr(o, ctypes.c_double),
+                            _ptr(lse, ctypes.c_double), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"win_oracle_fwd failed with code {rc}")
+    return o, lse
+
+
+def win_bwd(q, k, v, dout, offsets, window, scale, nthreads: int = 0, lib=None):
+    """(dQ, dK, dV) [T, h, dh] float64."""
+    lib = lib or win_load()
+    q, k, v, g = _f32(q), _f32(k), _f32(v), _f32(dout)
+    off = np.ascontiguousarray(offsets, dtype=np.int64)
+    T, h, dh = q.shape
+    B = off.shape[0] - 1
+    dq, dk, dv = (np.zeros((T, h, dh), dtype=np.float64) for _ in range(3))
+    rc = lib.win_oracle_bwd(B, h, dh, int(window), _ptr(off, ctypes.c_int64),
+                            _ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                            _ptr(v, ctypes.c_float), _ptr(g, ctypes.c_float), float(scale),
+                            _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double),
+                            _ptr(dv, ctypes.c_double), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"win_oracle_bwd failed with code {rc}")
+    return dq, dk, dv

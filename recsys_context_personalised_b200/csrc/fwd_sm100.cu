@@ -682,7 +682,7 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 // Registers: the launch gives 168 per thread (384 x 168 = 64,512); warps 0-3
 // drop to 80 and the two activation warpgroups rise to 208 (a thread holds a
 // whole 128-column S row): 128 x 80 + 256 x 208 = 63,488 <= 64,512.
-constexpr int kPolyPairs = 3;
+constexpr int kPolyPairs = 0;
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;

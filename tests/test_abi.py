@@ -113,3 +113,15 @@ def test_weight_gen_rejects_unsupported_shapes_on_host():
     assert lib.gdpa_weight_gen(4, 60, 64, 4096, 4096, 4096, None, None) == 2
     assert lib.gdpa_weight_gen(4, 64, 64, None, 4096, 4096, None, None) == 1
     assert lib.gdpa_weight_gen(4, 64, 64, 4100, 4096, 4096, None, None) == 1
+
+
+def test_pool_rejects_unsupported_shapes_on_host():
+    import ctypes
+    lib = pkg.load()
+    n = ctypes.c_size_t()
+    assert lib.gdpa_pool_workspace_size(4, 2, 128, 16, ctypes.byref(n)) == 2     # dh 128
+    assert lib.gdpa_pool_workspace_size(4, 2, 64, 129, ctypes.byref(n)) == 2     # S > 128
+    assert lib.gdpa_pool_workspace_size(4097, 2, 64, 16, ctypes.byref(n)) == 2   # B > 4096
+    assert lib.gdpa_pool_workspace_size(0, 2, 64, 16, ctypes.byref(n)) == 1
+    assert lib.gdpa_pool_workspace_size(4, 3, 64, 16, ctypes.byref(n)) == 0
+    assert n.value >= 256 + 16 * 4 * 2
