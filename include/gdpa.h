@@ -252,6 +252,30 @@ GDPA_API gdpa_status_t gdpa_pool_fwd(int32_t B, int32_t h, int32_t dh, int32_t S
                                      size_t workspace_bytes, void* stream);
 
 /*
+ * Sliding-window self-attention on the jagged token sequence.  The Kunlun
+ * summary (section 2.2, sliding-window bullet) restricts self-attention on the
+ * sequence to local windows, from O(T^2) to O(T w), without giving the
+ * window's alignment; this library takes the causal window of width `window`:
+ * token t of a sample attends to the tokens t' of the same sample with
+ * t - window < t' <= t.  Per head j:
+ *
+ *     O_t = sum_t' softmax_t'(scale * q_t . k_t') v_t',   LSE[j, t] = ln sum_t' exp(...)
+ *
+ *   q, k, v, o bf16 [T, h, dh] (device; o every row written), offsets int32
+ *   [B+1] (device), lse fp32 [h, T] (output; may be NULL).  Base pointers
+ *   16-byte aligned (lse, offsets 4-byte).  dh = 32 or 64; window >= 1.
+ *   workspace: device, >= gdpa_window_workspace_size bytes, 256-byte aligned.
+ *   max_n, total_tokens and the error behaviour as in gdpa_fwd.
+ */
+GDPA_API gdpa_status_t gdpa_window_workspace_size(int32_t B, int32_t h, int32_t dh,
+                                                  int64_t total_tokens, size_t* bytes);
+GDPA_API gdpa_status_t gdpa_window_fwd(int32_t B, int32_t h, int32_t dh, int64_t total_tokens,
+                                       int32_t max_n, int32_t window, float scale,
+                                       const void* q, const int32_t* offsets, const void* k,
+                                       const void* v, void* o, float* lse, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/*
  * Device-detected status of the last gdpa_fwd/gdpa_bwd that used `workspace`
  * (GDPA_OK, GDPA_ERR_INVALID_ARG for inconsistent offsets, GDPA_ERR_TIMEOUT).
  * Synchronises `stream`; writes the code to *status (host).

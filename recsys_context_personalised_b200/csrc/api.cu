@@ -51,6 +51,10 @@ cudaError_t launch_sm100_bwd(const gdpa_problem_t& p, const void* q, const int32
                              float* dq_acc, float* dsum, WsHeader* ws, Tile* tiles,
                              cudaStream_t st);
 int64_t sm100_bwd_items(const gdpa_problem_t& p);
+cudaError_t launch_sm100_window(int h, int dh, int64_t T, int window, float scale,
+                                const int32_t* offsets, const void* q, const void* k,
+                                const void* v, void* o, float* lse, WsHeader* ws,
+                                const Tile* tiles, cudaStream_t st);
 cudaError_t launch_sm100_pool(int B, int h, int dh, int S, int64_t T, float scale,
                               const void* seeds, const void* k, const void* v, void* o,
                               float* lse, WsHeader* ws, const Tile* tiles, cudaStream_t st);
@@ -293,6 +297,69 @@ gdpa_status_t gdpa_pool_fwd(int32_t B, int32_t h, int32_t dh, int32_t S, int64_t
   if (e == cudaSuccess) e = launch_pool_empty(offsets, B, h, S, dh, o, lse, ws, st);
   if (e == cudaSuccess)
     e = launch_sm100_pool(B, h, dh, S, total_tokens, scale, seeds, k, v, o, lse, ws, tiles, st);
+  return cuda_status(e);
+}
+
+namespace {
+gdpa_status_t check_window(int32_t B, int32_t h, int32_t dh, int64_t T, int32_t max_n,
+                           int32_t window, float scale) {
+  if (B < 1 || h < 1 || window < 1 || max_n < 0 || T < 0 || T >= (int64_t)1 << 31 ||
+      (int64_t)max_n * B < T || !(scale == scale))
+    return GDPA_ERR_INVALID_ARG;
+  if ((dh != 32 && dh != 64) || (int64_t)B * h >= (int64_t)1 << 24) return GDPA_ERR_UNSUPPORTED;
+  return GDPA_OK;
+}
+// the query-tile list of (h + 1) / 2 head pairs
+gdpa_problem_t window_list_problem(int32_t B, int32_t h, int64_t T, int32_t max_n) {
+  gdpa_problem_t p = {};
+  p.B = B;
+  p.h = (h + 1) / 2;
+  p.dh = 64;
+  p.m = 1;
+  p.max_n = max_n;
+  p.dtype = GDPA_DTYPE_BF16;
+  p.total_tokens = T;
+  p.phi = GDPA_PHI_SOFTMAX;
+  p.scale = 1.f;
+  return p;
+}
+}  // namespace
+
+gdpa_status_t gdpa_window_workspace_size(int32_t B, int32_t h, int32_t dh, int64_t total_tokens,
+                                         size_t* bytes) {
+  const int32_t max_n = total_tokens >= 0 && total_tokens < 0x7fffffff ? (int32_t)total_tokens : 0;
+  const gdpa_status_t s = check_window(B, h, dh, total_tokens, max_n, 1, 1.f);
+  if (s != GDPA_OK) return s;
+  if (!bytes) return GDPA_ERR_INVALID_ARG;
+  const gdpa_problem_t lp = window_list_problem(B, h, total_tokens, 0);
+  *bytes = align_up(sizeof(WsHeader) + sizeof(Tile) * (size_t)tile_capacity(lp, kMmaBM), 256);
+  return GDPA_OK;
+}
+
+gdpa_status_t gdpa_window_fwd(int32_t B, int32_t h, int32_t dh, int64_t total_tokens,
+                              int32_t max_n, int32_t window, float scale, const void* q,
+                              const int32_t* offsets, const void* k, const void* v, void* o,
+                              float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  g_launches = 0;
+  gdpa_status_t s = check_window(B, h, dh, total_tokens, max_n, window, scale);
+  if (s != GDPA_OK) return s;
+  const bool empty = total_tokens == 0;
+  if (!offsets || (!empty && (!q || !k || !v || !o))) return GDPA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      ((uintptr_t)offsets & 3u) || ((uintptr_t)lse & 3u))
+    return GDPA_ERR_INVALID_ARG;
+  const gdpa_problem_t lp = window_list_problem(B, h, total_tokens, max_n);
+  const size_t need =
+      align_up(sizeof(WsHeader) + sizeof(Tile) * (size_t)tile_capacity(lp, kMmaBM), 256);
+  s = check_ws(workspace, workspace_bytes, need);
+  if (s != GDPA_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  WsHeader* ws = (WsHeader*)workspace;
+  Tile* tiles = (Tile*)((char*)workspace + sizeof(WsHeader));
+  cudaError_t e = launch_schedule(lp, offsets, kMmaBM, ws, tiles, st);
+  if (e == cudaSuccess)
+    e = launch_sm100_window(h, dh, total_tokens, window, scale, offsets, q, k, v, o, lse, ws,
+                            tiles, st);
   return cuda_status(e);
 }
 

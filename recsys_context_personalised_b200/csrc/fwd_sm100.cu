@@ -73,6 +73,8 @@ struct FwdArgs {
   int64_t T;
   int h, m, nkv;
   int S;             // seed-query pooling: seeds per head (the output rows of an item)
+  int window;        // sliding window: keys t - window < t' <= t
+  const int32_t* offsets;   // sliding window: device offsets (sample starts)
   float scale;       // s
   float scale_log2;  // s * log2(e)
 };
@@ -684,6 +686,10 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 // whole 128-column S row): 128 x 80 + 256 x 208 = 63,488 <= 64,512.
 constexpr int kPolyPairs = 0;
 
+// Modes of the dh <= 64 forward kernel: the GDPA operator, seed-query pooling
+// (first level of HSP) and sliding-window self-attention on the jagged tokens.
+constexpr int kModeGdpa = 0, kModePool = 1, kModeWindow = 2;
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -712,14 +718,16 @@ __device__ __forceinline__ float row_extreme(const uint32_t (&s)[128]) {
   return NEG ? fmin3(fminf(e[0], e[1]), e[2], e[3]) : fmax3(fmaxf(e[0], e[1]), e[2], e[3]);
 }
 
-template <int DH, int PHI, bool BIAS, bool POOL>
+template <int DH, int PHI, bool BIAS, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
   using C = FwdCfg<DH>;
   static_assert(C::P_SEP, "needs P in TMEM columns of its own");
-  static_assert(!POOL || (PHI == GDPA_PHI_SOFTMAX && !BIAS), "pooling is softmax attention");
+  constexpr bool POOL = MODE == kModePool, WIN = MODE == kModeWindow;
+  static_assert(MODE == kModeGdpa || (PHI == GDPA_PHI_SOFTMAX && !BIAS),
+                "pooling and sliding-window attention are softmax attention");
   constexpr bool SOFTMAX = PHI == GDPA_PHI_SOFTMAX;
   constexpr uint32_t IDESC_S = idesc_bf16(128, 128, 0, 0);
   constexpr uint32_t IDESC_O = idesc_bf16(128, DH, 0, 1);
@@ -774,22 +782,35 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
   // GDPA: work item p = query tiles 2p, 2p+1 of the jagged tile list, all with
   // a.nkv key blocks of a.m keys.  Seed-query pooling (POOL): item p = heads
   // (2k, 2k+1) of one sample, the seeds of each head as the 128-row query
-  // tile, the sample's n_b tokens as ceil(n_b / 128) key blocks.
-  const int npairs = POOL ? count : (count + 1) >> 1;
+  // tile, the sample's n_b tokens as ceil(n_b / 128) key blocks.  Sliding
+  // window (WIN): item p = heads (2k, 2k+1) of one 128-row query tile; its
+  // keys are the sample's tokens from kstart = max(sample start, row0 - w + 1)
+  // to the tile's last row, masked per element to the causal window.
+  const int npairs = MODE == kModeGdpa ? (count + 1) >> 1 : count;
   auto get_pair = [&](int p) -> Pair {
-    if constexpr (POOL) {
+    if constexpr (MODE != kModeGdpa) {
       Pair r;
       r.a = a.tiles[p];
+      if (WIN) r.a.head *= 2;                        // the list holds head pairs
       r.has_b = r.a.head + 1 < a.h;
       r.b = r.a;
       r.b.head = r.a.head + 1;
-      r.share = false;
+      r.share = !r.has_b;     // a lone head streams its K/V once, like a shared pair
       return r;
     } else {
       return load_pair(a.tiles, count, p);
     }
   };
-  auto pair_nkv = [&](const Pair& pr) -> int { return POOL ? (pr.a.rows + 127) >> 7 : a.nkv; };
+  // first key row of a window item (WIN only)
+  auto win_kstart = [&](const Tile& t) -> int {
+    const int lo = t.row0 - a.window + 1, s0 = __ldg(a.offsets + t.b);
+    return lo > s0 ? lo : s0;
+  };
+  auto pair_nkv = [&](const Pair& pr) -> int {
+    if constexpr (POOL) return (pr.a.rows + 127) >> 7;
+    if constexpr (WIN) return (pr.a.row0 + pr.a.rows - win_kstart(pr.a) + 127) >> 7;
+    return a.nkv;
+  };
 
   if (warp < 4) {
     setmaxnreg_dec<80>();
@@ -805,9 +826,9 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
         mbar_expect_tx(bar(C::B_KVFULL + slot), C::TILEB);
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
-          if constexpr (POOL)   // tokens [T, h, dh]: rows past the sample are masked later
+          if constexpr (MODE != kModeGdpa)   // tokens [T, h, dh], masked later
             tma_load_3d(sKV + slot * C::TILEB + c * C::CHUNKB, map, bar(C::B_KVFULL + slot),
-                        c * C::CH, tl.head, tl.row0 + j * C::BN);
+                        c * C::CH, tl.head, (WIN ? win_kstart(tl) : tl.row0) + j * C::BN);
           else
             tma_load_4d(sKV + slot * C::TILEB + c * C::CHUNKB, map, bar(C::B_KVFULL + slot),
                         c * C::CH, j * C::BN, tl.head, tl.b);
@@ -995,8 +1016,9 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
       if (grp == 1 && !pr.has_b) continue;
       const Tile tl = grp ? pr.b : pr.a;
       const int nkv = pair_nkv(pr);
-      const int kv_len = POOL ? tl.rows : a.m;          // keys of the item
+      const int kv_len = POOL ? tl.rows : a.m;          // keys of the item (not WIN)
       const int out_rows = POOL ? a.S : tl.rows;        // output rows of the item
+      const int kstart = WIN ? win_kstart(tl) : 0;
       if (quad * 32 >= out_rows) {
         // every row of this warp lies past the tile's rows: those rows of O are
         // never stored, so the warp computes nothing and only keeps its part
@@ -1091,10 +1113,19 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
         {
           if constexpr (SOFTMAX) {
             const bool neg = !BIAS && c2 < 0.f;
-            if (valid < C::BN) {
+            // keys of this block that this row may see: columns [clo, chi]
+            int clo = 0, chi = valid - 1;
+            if constexpr (WIN) {
+              const int kb0 = kstart + j * C::BN, qpos = tl.row0 + row;
+              clo = max(0, qpos - a.window + 1 - kb0);
+              chi = min(C::BN - 1, qpos - kb0);
+            }
+            const bool partial = WIN ? __any_sync(0xffffffffu, clo > 0 || chi < C::BN - 1)
+                                     : valid < C::BN;
+            if (partial) {
               const uint32_t fill = __float_as_uint(neg ? INFINITY : -INFINITY);
 #pragma unroll
-              for (int i = 0; i < 128; ++i) s[i] = i < valid ? s[i] : fill;
+              for (int i = 0; i < 128; ++i) s[i] = i >= clo && i <= chi ? s[i] : fill;
             }
             const float m_blk =
                 (neg ? row_extreme<true>(s) : row_extreme<false>(s)) * (BIAS ? 1.f : c2);
@@ -1121,9 +1152,9 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
                 e.x = ex2_approx(x.x);
                 e.y = ex2_approx(x.y);
               }
-              if (valid < C::BN) {
-                e.x = 2 * i < valid ? e.x : 0.f;
-                e.y = 2 * i + 1 < valid ? e.y : 0.f;
+              if (partial) {
+                e.x = 2 * i >= clo && 2 * i <= chi ? e.x : 0.f;
+                e.y = 2 * i + 1 >= clo && 2 * i + 1 <= chi ? e.y : 0.f;
               }
               acc[i & 3] = __fadd2_rn(acc[i & 3], e);
               pk[i] = pack_bf16x2(e.x, e.y);
@@ -1272,7 +1303,7 @@ bool make_maps(const gdpa_problem_t& p, const void* q, const void* k, const void
 template <int DH, int PHI, bool BIAS>
 constexpr auto fwd_kernel() {
   if constexpr (DH <= 64)
-    return gdpa_fwd_early_kernel<DH, PHI, BIAS, false>;
+    return gdpa_fwd_early_kernel<DH, PHI, BIAS, kModeGdpa>;
   else
     return gdpa_fwd_sm100_kernel<DH, PHI, BIAS>;
 }
@@ -1328,6 +1359,46 @@ cudaError_t launch_fwd_bias(const gdpa_problem_t& p, const void* q, const void* 
   return launch_fwd_dh<DH, false>(p, q, k, v, bs, o, lse, ws, tiles, st);
 }
 
+// Sliding-window self-attention on the dh <= 64 forward kernel: q, k, v all
+// jagged [T, h, DH] (one 3-D map each), work items = query tiles x head pairs.
+template <int DH>
+cudaError_t launch_window_t(int h, int64_t T, int window, float scale, const int32_t* offsets,
+                            const void* q, const void* k, const void* v, void* o, float* lse,
+                            WsHeader* ws, const Tile* tiles, cudaStream_t st) {
+  using C = FwdCfg<DH>;
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorInvalidValue;
+  const CUtensorMapSwizzle sw = DH < 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const cuuint64_t dims[3] = {(cuuint64_t)DH, (cuuint64_t)h, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)DH * 2, (cuuint64_t)h * DH * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)C::CH, 1, 128};
+  CUtensorMap maps[3];
+  const void* ptrs[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i)
+    if (enc(&maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptrs[i]), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  auto kern = gdpa_fwd_early_kernel<DH, GDPA_PHI_SOFTMAX, false, kModeWindow>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return e;
+  FwdArgs args = {};
+  args.tiles = tiles;
+  args.ws = ws;
+  args.o = reinterpret_cast<__nv_bfloat16*>(o);
+  args.lse = lse;
+  args.T = T;
+  args.h = h;
+  args.window = window;
+  args.offsets = offsets;
+  args.scale = scale;
+  args.scale_log2 = scale * 1.4426950408889634f;
+  KernelScope ks_("gdpa_window_fwd_sm100", st);
+  kern<<<device_sm_count(), kThreads, C::SMEM, st>>>(maps[0], maps[1], maps[2], args);
+  return cudaGetLastError();
+}
+
 // Seed-query pooling on the dh <= 64 forward kernel: seeds [h, S, DH] as the
 // query tiles (rows >= S read as zero), the jagged tokens [T, h, DH] as keys
 // and values, softmax over each sample's tokens.
@@ -1358,7 +1429,7 @@ cudaError_t launch_pool_t(int B, int h, int S, int64_t T, float scale, const voi
             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
-  auto kern = gdpa_fwd_early_kernel<DH, GDPA_PHI_SOFTMAX, false, true>;
+  auto kern = gdpa_fwd_early_kernel<DH, GDPA_PHI_SOFTMAX, false, kModePool>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   FwdArgs args = {};
@@ -1398,6 +1469,18 @@ cudaError_t launch_sm100_pool(int B, int h, int dh, int S, int64_t T, float scal
   if (T == 0) return cudaSuccess;
   if (dh == 32) return launch_pool_t<32>(B, h, S, T, scale, seeds, k, v, o, lse, ws, tiles, st);
   if (dh == 64) return launch_pool_t<64>(B, h, S, T, scale, seeds, k, v, o, lse, ws, tiles, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_sm100_window(int h, int dh, int64_t T, int window, float scale,
+                                const int32_t* offsets, const void* q, const void* k,
+                                const void* v, void* o, float* lse, WsHeader* ws,
+                                const Tile* tiles, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  if (dh == 32)
+    return launch_window_t<32>(h, T, window, scale, offsets, q, k, v, o, lse, ws, tiles, st);
+  if (dh == 64)
+    return launch_window_t<64>(h, T, window, scale, offsets, q, k, v, o, lse, ws, tiles, st);
   return cudaErrorInvalidValue;
 }
 

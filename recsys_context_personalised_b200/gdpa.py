@@ -90,6 +90,11 @@ def load(path: str = LIB_PATH):
     lib.gdpa_pool_fwd.argtypes = [i32, i32, i32, i32, ctypes.c_int64, i32, ctypes.c_float, vp, vp,
                                   vp, vp, vp, vp, vp, sz, vp]
     lib.gdpa_pool_fwd.restype = ctypes.c_int
+    lib.gdpa_window_workspace_size.argtypes = [i32, i32, i32, ctypes.c_int64, ctypes.POINTER(sz)]
+    lib.gdpa_window_workspace_size.restype = ctypes.c_int
+    lib.gdpa_window_fwd.argtypes = [i32, i32, i32, ctypes.c_int64, i32, i32, ctypes.c_float, vp,
+                                    vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.gdpa_window_fwd.restype = ctypes.c_int
     for name in EXPORTED[:8]:
         getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
@@ -278,6 +283,33 @@ def pool_fwd(seeds: torch.Tensor, offsets, k: torch.Tensor, v: torch.Tensor, sca
                            _ptr(v), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
     if rc:
         raise GdpaError(rc, "gdpa_pool_fwd")
+    return o, lse
+
+
+def window_fwd(q: torch.Tensor, offsets, k: torch.Tensor, v: torch.Tensor, window: int,
+               scale: float, offsets_host, o=None, lse=None, ws=None, stream=None,
+               want_lse=True):
+    """Run gdpa_window_fwd (causal sliding-window attention on jagged q, k, v
+    [T, h, dh]); returns (o [T, h, dh], lse [h, T] or None)."""
+    lib = load()
+    T, h, dh = q.shape
+    off = [int(x) for x in offsets_host]
+    B = len(off) - 1
+    max_n = max((off[i + 1] - off[i] for i in range(B)), default=0)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((h, T), dtype=torch.float32, device=q.device)
+    if ws is None:
+        n = ctypes.c_size_t()
+        rc = lib.gdpa_window_workspace_size(B, h, dh, T, ctypes.byref(n))
+        if rc:
+            raise GdpaError(rc, "gdpa_window_workspace_size")
+        ws = workspace(n.value, q.device)
+    rc = lib.gdpa_window_fwd(B, h, dh, T, max_n, window, scale, _ptr(q), _ptr(offsets), _ptr(k),
+                             _ptr(v), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise GdpaError(rc, "gdpa_window_fwd")
     return o, lse
 
 
