@@ -58,7 +58,12 @@ KERNEL_SOURCES = {"gdpa_fwd_sm100": ("fwd_sm100.cu", "sm100.cuh", "gdpa_internal
 # a fused kernel, from one ncu capture: {kernel: {workload id: (bytes per unit,
 # sha16 of the kernel's sources at capture time)}}.  An entry whose hash no
 # longer matches the sources is not used (the traffic is then reported null).
-TRAFFIC_PER_UNIT = {}
+TRAFFIC_PER_UNIT = {
+    # 64-sample case of workload 5: 581.8 MB read + 35.5 MB written in one launch
+    "gdpa_fwd_sm100": {5: (0.0141204, "f8734db370efc1eb")},
+    # same case: 744.7 MB read + 589.3 MB written in one launch
+    "gdpa_bwd_sm100": {5: (0.0305141, "0fb05f418498559f")},
+}
 # fp32 FFMA peak for the SIMT kernels: 148 SMs * 128 FMA/clk * 2 flop * 1.965 GHz
 SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # dense bf16 tcgen05 rate of one SM (flop per clock), for the clock-scaled nominal peak
@@ -84,6 +89,15 @@ def parse(argv=None):
     ap.add_argument("--weight-gen", action="store_true",
                     help="linear-map workload only: generate K and V from the context vectors "
                          "(Weight Generation) inside every step, before the GDPA forward")
+    ap.add_argument("--bias", action="store_true",
+                    help="the biased PFFN variant: key bias b1 [B,h,m] and output bias b2 "
+                         "[B,h,dh] (fp32, N(0,1)/2) in every forward and backward")
+    ap.add_argument("--pool", type=int, default=0, metavar="S",
+                    help="seed-query attention pooling instead of GDPA: S seeds per head attend "
+                         "over the workload's jagged tokens (keys and values [T,h,dh])")
+    ap.add_argument("--window", type=int, default=0, metavar="W",
+                    help="causal sliding-window self-attention of width W on the workload's "
+                         "jagged tokens instead of GDPA")
     ap.add_argument("--phi", default=None,
                     choices=["identity", "silu", "softmax", "relu", "gelu"],
                     help="the same workload with another activation (the PFFN variants' phi)")
@@ -126,9 +140,9 @@ def fwd_bytes(wl, T):
     return b + (4 * T * wl.h if wl.phi_name == "softmax" else 0)
 
 
-def config_dict(wl, T, n_gpus, subset=None, weight_gen=False):
+def config_dict(wl, T, n_gpus, subset=None, weight_gen=False, bias=False):
     """The `config` object of the JSON line (identical in both arms)."""
-    return {"weight_gen": weight_gen,
+    return {"weight_gen": weight_gen, "bias": bias,
             "workload": wl.name if subset is None else
             f"{wl.name} (first {len(subset)} samples only: profiling case)",
             "B": wl.B if subset is None else len(subset), "h": wl.h, "dh": wl.dh, "m": wl.m,
@@ -378,15 +392,247 @@ def run_reference(args, rank):
           "tokens_per_s": tokens / secs})
 
 
+def variant_flops(kind, lengths, h, dh, S=0, window=0):
+    """Algorithmic FLOPs of one forward of an attention variant over a jagged
+    batch: pooling 4*S*T*h*dh (S seeds x n_b keys per sample); the causal
+    window 4*h*dh * sum over tokens of the keys in their window, where a
+    sample of n tokens holds n(n+1)/2 (n <= W) or W*n - W(W-1)/2 of them."""
+    n = [int(x) for x in lengths]
+    if kind == "pool":
+        return 4.0 * S * sum(n) * h * dh
+    W = int(window)
+    keys = sum(x * (x + 1) // 2 if x <= W else W * x - W * (W - 1) // 2 for x in n)
+    return 4.0 * h * dh * keys
+
+
+VARIANT_KERNELS = {"pool": "gdpa_pool_fwd_sm100", "window": "gdpa_window_fwd_sm100"}
+
+
+def variant_oracle_sample(lengths, flops_of, budget=ORACLE_STEP_FLOPS):
+    """A fixed seeded choice of samples whose oracle FLOPs fill `budget`."""
+    import numpy as np
+    order = np.random.default_rng(1234).permutation(len(lengths))
+    pick, acc = [], 0.0
+    for b in order:
+        f = flops_of([lengths[b]])
+        if pick and acc + f > budget:
+            break
+        pick.append(int(b))
+        acc += f
+    return sorted(pick)
+
+
+def run_variant(args, rank, world, local_rank):
+    """Seed-query pooling (--pool S) or the causal sliding window (--window W)
+    over the jagged tokens of a workload: per-step device events with the L2
+    flushed between steps, max over ranks, the kernel's roofline, the oracle
+    on a bounded sample, and an end-to-end pass from pinned host memory."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from recsys_context_personalised_b200 import gdpa as G
+    import synthetic as syn
+
+    kind = "pool" if args.pool else "window"
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    wl = syn.WORKLOADS[args.workload]
+    lens = syn.lengths(wl, seed=rank)
+    offs = syn.offsets_from_lengths(lens)
+    B, T, h, dh = wl.B, int(offs[-1]), wl.h, wl.dh
+    S, W = int(args.pool), int(args.window)
+    scale = 1.0 / dh ** 0.5
+    gen = torch.Generator(device=dev)
+
+    def draw(tid, *shape):
+        gen.manual_seed(1_000_003 * (rank + 1) + tid)
+        return torch.randn(*shape, generator=gen, device=dev).to(torch.bfloat16)
+
+    k, v = draw(1, T, h, dh), draw(2, T, h, dh)
+    q = draw(0, h, S, dh) if kind == "pool" else draw(0, T, h, dh)
+    off = torch.tensor(offs, dtype=torch.int32, device=dev)
+    shape = (B, T, int(lens.max()))
+    if kind == "pool":
+        o = torch.empty((B, h, S, dh), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, h, S), dtype=torch.float32, device=dev)
+        n_ws = ctypes_size(G.load().gdpa_pool_workspace_size, B, h, dh, S)
+    else:
+        o = torch.empty_like(q)
+        lse = torch.empty((h, T), dtype=torch.float32, device=dev)
+        n_ws = ctypes_size(G.load().gdpa_window_workspace_size, B, h, dh, T)
+    ws = torch.empty(max(n_ws, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    launches = [0]
+
+    def step(q_=q, k_=k, v_=v, o_=o):
+        if kind == "pool":
+            G.pool_fwd(q_, off, k_, v_, scale, None, o=o_, lse=lse, ws=ws, stream=stream,
+                       shape=shape)
+        else:
+            G.window_fwd(q_, off, k_, v_, W, scale, None, o=o_, lse=lse, ws=ws, stream=stream,
+                         shape=shape)
+        launches[0] += G.last_launch_count()
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    if G.workspace_status(ws):
+        raise RuntimeError("device-side status error during warm-up")
+
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    G.timing_enable(True)
+    launches[0] = 0
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    per_kernel = G.timing_read()
+    G.timing_enable(False)
+    clk = clocks.stop()
+    if G.workspace_status(ws):
+        raise RuntimeError("device-side status error in the timed steps")
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in evs)
+    flops = variant_flops(kind, lens, h, dh, S, W)
+    agg = aggregate(ms, flops * args.steps, float(T) * args.steps, float(launches[0]), world,
+                    dist, dev)
+    pk = peaks()
+    bf16_peak, peak_why = choose_bf16_peak(pk, clk)
+    name = VARIANT_KERNELS[kind]
+    nl, tot_ms = per_kernel.get(name, (0, 0.0))
+    avg_ms = tot_ms / max(nl, 1)
+    ach = flops / (avg_ms / 1e3) / 1e12 if avg_ms > 0 else 0.0
+    roof = {"bound": "tensor", "achieved": ach, "peak": bf16_peak, "unit": "TFLOP/s",
+            "frac": ach / bf16_peak, "peak_source": peak_why, "kernel": name, "traffic": None,
+            "traffic_source": "null: no capture of this kernel", "launches": nl,
+            "avg_ms": avg_ms}
+    kernels = {k_: {"launches": v_[0], "ms": v_[1], "share": v_[1] / max(ms, 1e-9)}
+               for k_, v_ in per_kernel.items()}
+
+    # end to end: pinned host inputs in, the call, O out, every step (one stream)
+    e2e = None
+    if not args.no_e2e and args.e2e_steps > 0:
+        ins = ([k, v] if kind == "pool" else [q, k, v])
+        h_in = [x.cpu().pin_memory() for x in ins]
+        h_off = torch.tensor(offs, dtype=torch.int32).pin_memory()
+        h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in h_in) + h_off.numel() * 4
+        d2h = h_o.numel() * h_o.element_size()
+
+        def e2e_step():
+            off.copy_(h_off, non_blocking=True)
+            for dst, src in zip(ins, h_in):
+                dst.copy_(src, non_blocking=True)
+            step()
+            h_o.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ea = aggregate(e0.elapsed_time(e1), flops * args.e2e_steps, 0.0, 0.0, world, dist, dev)
+        e2e = {"value": ea["tflops"], "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps,
+               "ms_per_step": ea["ms_max"] / args.e2e_steps,
+               "api": f"recsys_context_personalised_b200.gdpa.{kind}_fwd with inputs copied "
+                      "from and O copied to pinned host memory every step (one stream)"}
+        del h_in, h_o
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        pick = variant_oracle_sample(lens, lambda n_: variant_flops(kind, n_, h, dh, S, W))
+        rows = np.concatenate([np.arange(offs[b], offs[b + 1]) for b in pick]).astype(np.int64)
+        sub_off = syn.offsets_from_lengths([lens[b] for b in pick])
+        ridx = torch.tensor(rows, device=dev)
+        kh, vh = (x.index_select(0, ridx).float().cpu().numpy() for x in (k, v))
+        f = dt = 0.0
+        for _ in range(max(args.cpu_passes, 1)):
+            t0 = time.perf_counter()
+            if kind == "pool":
+                oracle.pool_fwd(q.float().cpu().numpy(), kh, vh, sub_off, scale)
+            else:
+                qh = q.index_select(0, ridx).float().cpu().numpy()
+                oracle.win_fwd(qh, kh, vh, sub_off, W, scale)
+            dt += time.perf_counter() - t0
+            f += variant_flops(kind, [lens[b] for b in pick], h, dh, S, W)
+        cpu = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+               "kind": "oracle",
+               "sample": f"{len(pick)} of {B} samples ({len(rows)} tokens, all {h} heads), fwd, "
+                         f"fixed seeded choice, {args.cpu_passes} passes, {dt:.1f} s"}
+
+    if rank == 0:
+        what = (f"hsp_seed_pool_S{S}" if kind == "pool" else f"sliding_window_W{W}")
+        emit({"metric": ("HSP seed-query pooling fwd TFLOP/s" if kind == "pool" else
+                         "sliding-window self-attention fwd TFLOP/s"),
+              "value": agg["tflops"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+              "warmup": args.warmup, "ms_per_step": agg["ms_max"] / args.steps,
+              "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+              "data": "synthetic",
+              "config": {"workload": f"{what}_tokens_of_{wl.name}", "B": B, "h": h, "dh": dh,
+                         "seeds": S or None, "window": W or None, "lengths": wl.lengths,
+                         "tokens_per_rank": T, "scale": scale,
+                         "inputs": "N(0,1) bf16 from a seeded torch generator per tensor",
+                         "parallelism": f"replicas x{world} (samples independent)",
+                         "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write "
+                               "outside the per-step events)"},
+              "pct_of_bf16_peak": 100.0 * agg["tflops"] / (world * bf16_peak),
+              "flops_per_step": flops, "tokens_per_s": agg["tokens_per_s"],
+              "gpu_launches": agg["launches"], "kernels": kernels, "roofline": roof,
+              "cpu_baseline": cpu, "e2e": e2e, "clocks": clk})
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def ctypes_size(fn, *args_):
+    """Call a `*_workspace_size` entry point; the size in bytes."""
+    import ctypes
+    n = ctypes.c_size_t()
+    rc = fn(*args_, ctypes.byref(n))
+    if rc:
+        raise RuntimeError(f"workspace size query failed with code {rc}")
+    return int(n.value)
+
+
 def main(argv=None):
     args = parse(argv)
+    if args.pool and args.window:
+        raise SystemExit("bench.py: --pool and --window are separate workloads")
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         argv = sys.argv[1:] if argv is None else list(argv)
         cmd = torchrun_command(argv, args.gpus, _free_port())
         raise SystemExit(subprocess.call(cmd))
     rank, world, local_rank = world_from_env(args)
     if args.impl == "reference":
+        if args.pool or args.window:
+            raise SystemExit("bench.py: the reference arm times the GDPA workloads; the "
+                             "attention variants report the oracle as cpu_baseline")
         run_reference(args, rank)
+        return
+    if args.pool or args.window:
+        run_variant(args, rank, world, local_rank)
         return
 
     import torch
@@ -430,16 +676,31 @@ def main(argv=None):
             raise SystemExit("bench.py: --weight-gen needs the linear-map workload (2), all samples")
         wg = {x: syn.weight_gen_factors(wl.wid, x, seed=rank, device=dev) for x in ("k", "v")}
 
+    b1 = b2 = db1 = db2 = None
+    if args.bias:            # the biased PFFN variant: phi(s Q K^T + b1) V + b2
+        bgen = torch.Generator(device=dev)
+        bgen.manual_seed(7919 + rank)
+        b1 = 0.5 * torch.randn((k.shape[0], wl.h, wl.m), generator=bgen, device=dev)
+        b2 = 0.5 * torch.randn((k.shape[0], wl.h, wl.dh), generator=bgen, device=dev)
+        db1, db2 = torch.empty_like(b1), torch.empty_like(b2)
+
     def step():
         if wg is not None:       # K, V = reshape(W c_b) for every sample, then the GDPA forward
             G.weight_gen(wg["k"][0], wg["k"][1], y=k.view(wl.B, -1), stream=stream)
             launches[0] += 1
             G.weight_gen(wg["v"][0], wg["v"][1], y=v.view(wl.B, -1), stream=stream)
             launches[0] += 1
-        G.fwd(p, q, off, k, v, o=o, lse=lse, ws=ws_f, stream=stream)
+        if args.bias:
+            G.fwd_bias(p, q, off, k, v, b1, b2, o=o, lse=lse, ws=ws_f, stream=stream)
+        else:
+            G.fwd(p, q, off, k, v, o=o, lse=lse, ws=ws_f, stream=stream)
         launches[0] += G.last_launch_count()
         if wl.backward:
-            G.bwd(p, q, off, k, v, o, lse, g, dq=dq, dk=dk, dv=dv, ws=ws_b, stream=stream)
+            if args.bias:
+                G.bwd_bias(p, q, off, k, v, b1, b2, o, lse, g, dq=dq, dk=dk, dv=dv, db1=db1,
+                           db2=db2, ws=ws_b, stream=stream)
+            else:
+                G.bwd(p, q, off, k, v, o, lse, g, dq=dq, dk=dk, dv=dv, ws=ws_b, stream=stream)
             launches[0] += G.last_launch_count()
 
     for _ in range(max(args.warmup, 0)):
@@ -539,7 +800,7 @@ def main(argv=None):
     # directions and the compute overlap; per-chunk events order every reuse
     # of a buffer (also from one step to the next).
     e2e = None
-    if not args.no_e2e and args.e2e_steps > 0:
+    if not args.no_e2e and args.e2e_steps > 0 and not args.bias:
         o_full = o.clone()          # O of the full-batch call (the forward is deterministic)
         ins = [q, k, v] + ([g] if wl.backward else [])
         outs = [o] + ([dq, dk, dv] if wl.backward else [])
@@ -655,7 +916,8 @@ def main(argv=None):
               "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
               "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
               "vs_baseline": None, "dtype": "f32" if fp32 else "bf16", "data": "synthetic",
-              "config": config_dict(wl, T, world, subset, bool(args.weight_gen)),
+              "config": config_dict(wl, T, world, subset, bool(args.weight_gen),
+                                    bool(args.bias)),
               "pct_of_bf16_peak": None if fp32 else 100.0 * value / (world * bf16_peak),
               "bf16_peak": None if fp32 else {"value": bf16_peak, "source": peak_why,
                                               "nominal_at_median_clock": nominal},

@@ -259,16 +259,25 @@ def weight_gen_bwd(w: torch.Tensor, ctx: torch.Tensor, dy: torch.Tensor, ws=None
     return dw, dctx
 
 
+def _batch_shape(offsets_host, shape):
+    """(B, T, max_n) of a jagged batch: from ``shape`` when given, else from
+    the host copy of the offsets."""
+    if shape is not None:
+        return tuple(int(x) for x in shape)
+    off = [int(x) for x in offsets_host]
+    B = len(off) - 1
+    return B, off[-1], max((off[i + 1] - off[i] for i in range(B)), default=0)
+
+
 def pool_fwd(seeds: torch.Tensor, offsets, k: torch.Tensor, v: torch.Tensor, scale: float,
-             offsets_host, o=None, lse=None, ws=None, stream=None, want_lse=True):
+             offsets_host, o=None, lse=None, ws=None, stream=None, want_lse=True, shape=None):
     """Run gdpa_pool_fwd (seed-query attention pooling): seeds [h, S, dh],
     jagged k, v [T, h, dh] with device ``offsets`` (host copy ``offsets_host``
-    for T and max_n); returns (o [B, h, S, dh], lse [B, h, S] or None)."""
+    for B, T and max_n, or ``shape`` = (B, T, max_n)); returns
+    (o [B, h, S, dh], lse [B, h, S] or None)."""
     lib = load()
     h, S, dh = seeds.shape
-    off = [int(x) for x in offsets_host]
-    B, T = len(off) - 1, off[-1]
-    max_n = max((off[i + 1] - off[i] for i in range(B)), default=0)
+    B, T, max_n = _batch_shape(offsets_host, shape)
     if o is None:
         o = torch.empty((B, h, S, dh), dtype=seeds.dtype, device=seeds.device)
     if lse is None and want_lse:
@@ -288,14 +297,13 @@ def pool_fwd(seeds: torch.Tensor, offsets, k: torch.Tensor, v: torch.Tensor, sca
 
 def window_fwd(q: torch.Tensor, offsets, k: torch.Tensor, v: torch.Tensor, window: int,
                scale: float, offsets_host, o=None, lse=None, ws=None, stream=None,
-               want_lse=True):
+               want_lse=True, shape=None):
     """Run gdpa_window_fwd (causal sliding-window attention on jagged q, k, v
-    [T, h, dh]); returns (o [T, h, dh], lse [h, T] or None)."""
+    [T, h, dh]; B and max_n from ``offsets_host`` or ``shape`` = (B, T, max_n));
+    returns (o [T, h, dh], lse [h, T] or None)."""
     lib = load()
     T, h, dh = q.shape
-    off = [int(x) for x in offsets_host]
-    B = len(off) - 1
-    max_n = max((off[i + 1] - off[i] for i in range(B)), default=0)
+    B, _, max_n = _batch_shape(offsets_host, shape)
     if o is None:
         o = torch.empty_like(q)
     if lse is None and want_lse:

@@ -2,6 +2,8 @@
 override, the end-to-end chunking, the oracle sample, the peak choice, the
 traffic record's source hash and the multi-rank launch."""
 import argparse
+
+import numpy as np
 import os
 
 import pytest
@@ -129,3 +131,31 @@ def test_world_size_must_match_gpus(monkeypatch):
     assert bench.world_from_env(bench.parse(["--gpus", "2"])) == (1, 2, 1)
     with pytest.raises(SystemExit):
         bench.world_from_env(bench.parse(["--gpus", "4"]))
+
+
+def test_variant_flops_window_counts_the_keys_of_every_window():
+    """4*h*dh per (query, key) pair of the causal window t - W < t' <= t,
+    counted one token at a time."""
+    rng = np.random.default_rng(3)
+    lengths = rng.integers(0, 700, size=40)
+    for W in (1, 2, 17, 128, 1000):
+        pairs = sum(min(W, t + 1) for n in lengths for t in range(int(n)))
+        assert bench.variant_flops("window", lengths, 16, 64, window=W) == 4.0 * 16 * 64 * pairs
+
+
+def test_variant_flops_pool_is_seeds_times_tokens():
+    lengths = [0, 5, 130]
+    assert bench.variant_flops("pool", lengths, 16, 64, S=64) == 4.0 * 64 * 135 * 16 * 64
+
+
+def test_variant_oracle_sample_fills_its_budget_and_is_fixed():
+    lengths = np.arange(1, 200)
+    f = lambda n: float(sum(n))
+    a = bench.variant_oracle_sample(lengths, f, budget=500.0)
+    assert a == bench.variant_oracle_sample(lengths, f, budget=500.0)
+    assert a == sorted(set(a)) and sum(lengths[b] for b in a) <= 500 + max(lengths)
+
+
+def test_pool_and_window_are_exclusive():
+    with pytest.raises(SystemExit):
+        bench.main(["--pool", "64", "--window", "128"])
