@@ -98,6 +98,8 @@ def parse(argv=None):
     ap.add_argument("--window", type=int, default=0, metavar="W",
                     help="causal sliding-window self-attention of width W on the workload's "
                          "jagged tokens instead of GDPA")
+    ap.add_argument("--variant-backward", action="store_true",
+                    help="with --pool or --window: every step runs the forward and the backward")
     ap.add_argument("--phi", default=None,
                     choices=["identity", "silu", "softmax", "relu", "gelu"],
                     help="the same workload with another activation (the PFFN variants' phi)")
@@ -405,7 +407,8 @@ def variant_flops(kind, lengths, h, dh, S=0, window=0):
     return 4.0 * h * dh * keys
 
 
-VARIANT_KERNELS = {"pool": "gdpa_pool_fwd_sm100", "window": "gdpa_window_fwd_sm100"}
+VARIANT_KERNELS = {"pool": ("gdpa_pool_fwd_sm100", "gdpa_pool_bwd_sm100"),
+                   "window": ("gdpa_window_fwd_sm100", "gdpa_window_bwd_sm100")}
 
 
 def variant_oracle_sample(lengths, flops_of, budget=ORACLE_STEP_FLOPS):
@@ -458,6 +461,7 @@ def run_variant(args, rank, world, local_rank):
 
     k, v = draw(1, T, h, dh), draw(2, T, h, dh)
     q = draw(0, h, S, dh) if kind == "pool" else draw(0, T, h, dh)
+    bwd = bool(args.variant_backward)
     off = torch.tensor(offs, dtype=torch.int32, device=dev)
     shape = (B, T, int(lens.max()))
     if kind == "pool":
@@ -469,6 +473,15 @@ def run_variant(args, rank, world, local_rank):
         lse = torch.empty((h, T), dtype=torch.float32, device=dev)
         n_ws = ctypes_size(G.load().gdpa_window_workspace_size, B, h, dh, T)
     ws = torch.empty(max(n_ws, 1), dtype=torch.uint8, device=dev)
+    if bwd:
+        dout = draw(3, *o.shape)
+        dk, dv = torch.empty_like(k), torch.empty_like(v)
+        dq = (torch.empty((h, S, dh), dtype=torch.float32, device=dev) if kind == "pool"
+              else torch.empty_like(q))
+        n_wb = (ctypes_size(G.load().gdpa_pool_bwd_workspace_size, B, h, dh, S, T)
+                if kind == "pool" else
+                ctypes_size(G.load().gdpa_window_bwd_workspace_size, B, h, dh, T))
+        ws_b = torch.empty(max(n_wb, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     launches = [0]
@@ -481,6 +494,14 @@ def run_variant(args, rank, world, local_rank):
             G.window_fwd(q_, off, k_, v_, W, scale, None, o=o_, lse=lse, ws=ws, stream=stream,
                          shape=shape)
         launches[0] += G.last_launch_count()
+        if bwd and kind == "pool":
+            G.pool_bwd(q_, off, k_, v_, o_, lse, dout, scale, None, dk=dk, dv=dv, dseeds=dq,
+                       ws=ws_b, stream=stream, shape=shape)
+            launches[0] += G.last_launch_count()
+        elif bwd:
+            G.window_bwd(q_, off, k_, v_, o_, lse, dout, W, scale, None, dq=dq, dk=dk, dv=dv,
+                         ws=ws_b, stream=stream, shape=shape)
+            launches[0] += G.last_launch_count()
 
     for _ in range(max(args.warmup, 0)):
         step()
@@ -507,18 +528,21 @@ def run_variant(args, rank, world, local_rank):
     per_kernel = G.timing_read()
     G.timing_enable(False)
     clk = clocks.stop()
-    if G.workspace_status(ws):
+    if G.workspace_status(ws) or (bwd and G.workspace_status(ws_b)):
         raise RuntimeError("device-side status error in the timed steps")
     ms = sum(e0.elapsed_time(e1) for e0, e1 in evs)
-    flops = variant_flops(kind, lens, h, dh, S, W)
+    fwd_flops = variant_flops(kind, lens, h, dh, S, W)
+    flops = fwd_flops * (3.0 if bwd else 1.0)      # the backward credits 8 per 4 of the forward
     agg = aggregate(ms, flops * args.steps, float(T) * args.steps, float(launches[0]), world,
                     dist, dev)
     pk = peaks()
     bf16_peak, peak_why = choose_bf16_peak(pk, clk)
-    name = VARIANT_KERNELS[kind]
+    names = VARIANT_KERNELS[kind] if bwd else VARIANT_KERNELS[kind][:1]
+    name = max(names, key=lambda k_: per_kernel.get(k_, (0, 0.0))[1])
     nl, tot_ms = per_kernel.get(name, (0, 0.0))
     avg_ms = tot_ms / max(nl, 1)
-    ach = flops / (avg_ms / 1e3) / 1e12 if avg_ms > 0 else 0.0
+    kflops = fwd_flops * (2.0 if name.endswith("bwd_sm100") else 1.0)
+    ach = kflops / (avg_ms / 1e3) / 1e12 if avg_ms > 0 else 0.0
     roof = {"bound": "tensor", "achieved": ach, "peak": bf16_peak, "unit": "TFLOP/s",
             "frac": ach / bf16_peak, "peak_source": peak_why, "kernel": name, "traffic": None,
             "traffic_source": "null: no capture of this kernel", "launches": nl,
@@ -529,19 +553,21 @@ def run_variant(args, rank, world, local_rank):
     # end to end: pinned host inputs in, the call, O out, every step (one stream)
     e2e = None
     if not args.no_e2e and args.e2e_steps > 0:
-        ins = ([k, v] if kind == "pool" else [q, k, v])
+        ins = ([k, v] if kind == "pool" else [q, k, v]) + ([dout] if bwd else [])
+        outs = [o] + ([dq, dk, dv] if bwd else [])
         h_in = [x.cpu().pin_memory() for x in ins]
         h_off = torch.tensor(offs, dtype=torch.int32).pin_memory()
-        h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h_out = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in outs]
         h2d = sum(x.numel() * x.element_size() for x in h_in) + h_off.numel() * 4
-        d2h = h_o.numel() * h_o.element_size()
+        d2h = sum(x.numel() * x.element_size() for x in h_out)
 
         def e2e_step():
             off.copy_(h_off, non_blocking=True)
             for dst, src in zip(ins, h_in):
                 dst.copy_(src, non_blocking=True)
             step()
-            h_o.copy_(o, non_blocking=True)
+            for dst, src in zip(h_out, outs):
+                dst.copy_(src, non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -556,37 +582,50 @@ def run_variant(args, rank, world, local_rank):
         e2e = {"value": ea["tflops"], "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps,
                "ms_per_step": ea["ms_max"] / args.e2e_steps,
-               "api": f"recsys_context_personalised_b200.gdpa.{kind}_fwd with inputs copied "
-                      "from and O copied to pinned host memory every step (one stream)"}
-        del h_in, h_o
+               "api": f"recsys_context_personalised_b200.gdpa.{kind}_fwd"
+                      f"{f' + {kind}_bwd' if bwd else ''} with inputs copied from and outputs "
+                      "copied to pinned host memory every step (one stream)"}
+        del h_in, h_out
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
-        pick = variant_oracle_sample(lens, lambda n_: variant_flops(kind, n_, h, dh, S, W))
+        mult = 3.0 if bwd else 1.0
+        pick = variant_oracle_sample(lens, lambda n_: mult * variant_flops(kind, n_, h, dh, S, W))
         rows = np.concatenate([np.arange(offs[b], offs[b + 1]) for b in pick]).astype(np.int64)
         sub_off = syn.offsets_from_lengths([lens[b] for b in pick])
         ridx = torch.tensor(rows, device=dev)
         kh, vh = (x.index_select(0, ridx).float().cpu().numpy() for x in (k, v))
+        qh = (q.float().cpu().numpy() if kind == "pool" else
+              q.index_select(0, ridx).float().cpu().numpy())
+        gh = None
+        if bwd:
+            gh = (dout.index_select(0, torch.tensor(pick, device=dev)) if kind == "pool" else
+                  dout.index_select(0, ridx)).float().cpu().numpy()
         f = dt = 0.0
         for _ in range(max(args.cpu_passes, 1)):
             t0 = time.perf_counter()
             if kind == "pool":
-                oracle.pool_fwd(q.float().cpu().numpy(), kh, vh, sub_off, scale)
+                oracle.pool_fwd(qh, kh, vh, sub_off, scale)
+                if bwd:
+                    oracle.pool_bwd(qh, kh, vh, gh, sub_off, scale)
             else:
-                qh = q.index_select(0, ridx).float().cpu().numpy()
                 oracle.win_fwd(qh, kh, vh, sub_off, W, scale)
+                if bwd:
+                    oracle.win_bwd(qh, kh, vh, gh, sub_off, W, scale)
             dt += time.perf_counter() - t0
-            f += variant_flops(kind, [lens[b] for b in pick], h, dh, S, W)
+            f += mult * variant_flops(kind, [lens[b] for b in pick], h, dh, S, W)
         cpu = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
                "kind": "oracle",
-               "sample": f"{len(pick)} of {B} samples ({len(rows)} tokens, all {h} heads), fwd, "
-                         f"fixed seeded choice, {args.cpu_passes} passes, {dt:.1f} s"}
+               "sample": f"{len(pick)} of {B} samples ({len(rows)} tokens, all {h} heads), "
+                         f"{'fwd+bwd' if bwd else 'fwd'}, fixed seeded choice, "
+                         f"{args.cpu_passes} passes, {dt:.1f} s"}
 
     if rank == 0:
         what = (f"hsp_seed_pool_S{S}" if kind == "pool" else f"sliding_window_W{W}")
-        emit({"metric": ("HSP seed-query pooling fwd TFLOP/s" if kind == "pool" else
-                         "sliding-window self-attention fwd TFLOP/s"),
+        emit({"metric": ("HSP seed-query pooling " if kind == "pool" else
+                         "sliding-window self-attention ") + ("fwd+bwd" if bwd else "fwd") +
+                        " TFLOP/s",
               "value": agg["tflops"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
               "warmup": args.warmup, "ms_per_step": agg["ms_max"] / args.steps,
               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -599,7 +638,7 @@ def run_variant(args, rank, world, local_rank):
                          "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write "
                                "outside the per-step events)"},
               "pct_of_bf16_peak": 100.0 * agg["tflops"] / (world * bf16_peak),
-              "flops_per_step": flops, "tokens_per_s": agg["tokens_per_s"],
+              "flops_per_step": flops, "backward": bwd, "tokens_per_s": agg["tokens_per_s"],
               "gpu_launches": agg["launches"], "kernels": kernels, "roofline": roof,
               "cpu_baseline": cpu, "e2e": e2e, "clocks": clk})
     if world > 1:

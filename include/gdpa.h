@@ -252,6 +252,30 @@ GDPA_API gdpa_status_t gdpa_pool_fwd(int32_t B, int32_t h, int32_t dh, int32_t S
                                      size_t workspace_bytes, void* stream);
 
 /*
+ * Gradient of gdpa_pool_fwd for an upstream dO (same passage; the softmax
+ * attention gradient with the seeds as queries):
+ *
+ *     dV_t = sum_i P[i, t] dO_i,   dS = P * (dP - D),   dP = dO V^T,   D_i = dO_i . O_i,
+ *     dK_t = scale * sum_i dS[i, t] seeds_i,   dseeds_i = scale * sum_b sum_t dS[i, t] k_t,
+ *
+ * per sample b and head j; the seeds' gradient sums over every sample.
+ *   seeds, k, v, o (from gdpa_pool_fwd), lse (its fp32 [B, h, S] output,
+ *   natural log, required), dout bf16 [B, h, S, dh]; outputs dseeds fp32
+ *   [h, S, dh] (overwritten), dk, dv bf16 [T, h, dh] (every row written).
+ *   Same shapes, limits, alignment and error behaviour as gdpa_pool_fwd.
+ *   workspace: device, >= gdpa_pool_bwd_workspace_size bytes, 256-byte
+ *   aligned; device-detected errors go to its status word.
+ */
+GDPA_API gdpa_status_t gdpa_pool_bwd_workspace_size(int32_t B, int32_t h, int32_t dh, int32_t S,
+                                                    int64_t total_tokens, size_t* bytes);
+GDPA_API gdpa_status_t gdpa_pool_bwd(int32_t B, int32_t h, int32_t dh, int32_t S,
+                                     int64_t total_tokens, int32_t max_n, float scale,
+                                     const void* seeds, const int32_t* offsets, const void* k,
+                                     const void* v, const void* o, const float* lse,
+                                     const void* dout, float* dseeds, void* dk, void* dv,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Sliding-window self-attention on the jagged token sequence.  The Kunlun
  * summary (section 2.2, sliding-window bullet) restricts self-attention on the
  * sequence to local windows, from O(T^2) to O(T w), without giving the
@@ -274,6 +298,25 @@ GDPA_API gdpa_status_t gdpa_window_fwd(int32_t B, int32_t h, int32_t dh, int64_t
                                        const void* q, const int32_t* offsets, const void* k,
                                        const void* v, void* o, float* lse, void* workspace,
                                        size_t workspace_bytes, void* stream);
+
+/*
+ * Gradient of gdpa_window_fwd for an upstream dO: dQ, dK, dV of the causal
+ * window's softmax attention (same passage), with D_t = dO_t . O_t.
+ *   q, k, v, o (from gdpa_window_fwd), lse (its fp32 [h, T] output, natural
+ *   log, required), dout bf16 [T, h, dh]; outputs dq, dk, dv bf16 [T, h, dh]
+ *   (every row written).  Same limits, alignment and error behaviour as
+ *   gdpa_window_fwd, and B <= 4096 (GDPA_ERR_UNSUPPORTED otherwise).
+ *   workspace: device, >= gdpa_window_bwd_workspace_size bytes, 256-byte
+ *   aligned; device-detected errors go to its status word.
+ */
+GDPA_API gdpa_status_t gdpa_window_bwd_workspace_size(int32_t B, int32_t h, int32_t dh,
+                                                      int64_t total_tokens, size_t* bytes);
+GDPA_API gdpa_status_t gdpa_window_bwd(int32_t B, int32_t h, int32_t dh, int64_t total_tokens,
+                                       int32_t max_n, int32_t window, float scale,
+                                       const void* q, const int32_t* offsets, const void* k,
+                                       const void* v, const void* o, const float* lse,
+                                       const void* dout, void* dq, void* dk, void* dv,
+                                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Device-detected status of the last gdpa_fwd/gdpa_bwd that used `workspace`

@@ -58,6 +58,18 @@ cudaError_t launch_sm100_window(int h, int dh, int64_t T, int window, float scal
 cudaError_t launch_sm100_pool(int B, int h, int dh, int S, int64_t T, float scale,
                               const void* seeds, const void* k, const void* v, void* o,
                               float* lse, WsHeader* ws, const Tile* tiles, cudaStream_t st);
+cudaError_t launch_sm100_window_bwd(int B, int h, int dh, int64_t T, int max_n, int window,
+                                    float scale, const int32_t* offsets, const void* q,
+                                    const void* k, const void* v, const void* o,
+                                    const float* lse, const void* dout, void* dq, void* dk,
+                                    void* dv, float* dq_acc, float* dsum, WsHeader* ws,
+                                    Tile* tiles, int64_t cap, cudaStream_t st);
+cudaError_t launch_sm100_pool_bwd(int B, int h, int dh, int S, int64_t T, int max_n, float scale,
+                                  const int32_t* offsets, const void* seeds, const void* k,
+                                  const void* v, const void* o, const float* lse,
+                                  const void* dout, float* dseeds, void* dk, void* dv,
+                                  float* dsum, WsHeader* ws, Tile* tiles, int64_t cap,
+                                  cudaStream_t st);
 
 namespace {
 
@@ -361,6 +373,99 @@ gdpa_status_t gdpa_window_fwd(int32_t B, int32_t h, int32_t dh, int64_t total_to
     e = launch_sm100_window(h, dh, total_tokens, window, scale, offsets, q, k, v, o, lse, ws,
                             tiles, st);
   return cuda_status(e);
+}
+
+namespace {
+// backward work list of the jagged-key variants: h x (T / 128 + B) items at most
+int64_t jkv_capacity(int32_t B, int32_t h, int64_t T) { return (int64_t)h * (T / 128 + B); }
+size_t jkv_list_bytes(int32_t B, int32_t h, int64_t T) {
+  return align_up(sizeof(WsHeader) + sizeof(Tile) * (size_t)jkv_capacity(B, h, T), 256);
+}
+// [list][dQ accumulator T x h x dh fp32][D h x T fp32]
+size_t window_bwd_ws_bytes(int32_t B, int32_t h, int32_t dh, int64_t T) {
+  return jkv_list_bytes(B, h, T) + align_up((size_t)T * h * dh * 4, 256) +
+         align_up((size_t)T * h * 4, 256);
+}
+// [list][D B x h x S fp32]
+size_t pool_bwd_ws_bytes(int32_t B, int32_t h, int32_t S, int64_t T) {
+  return jkv_list_bytes(B, h, T) + align_up((size_t)B * h * S * 4, 256);
+}
+}  // namespace
+
+gdpa_status_t gdpa_window_bwd_workspace_size(int32_t B, int32_t h, int32_t dh,
+                                             int64_t total_tokens, size_t* bytes) {
+  const int32_t max_n = total_tokens >= 0 && total_tokens < 0x7fffffff ? (int32_t)total_tokens : 0;
+  gdpa_status_t s = check_window(B, h, dh, total_tokens, max_n, 1, 1.f);
+  if (s != GDPA_OK) return s;
+  if (B > 4096) return GDPA_ERR_UNSUPPORTED;
+  if (!bytes) return GDPA_ERR_INVALID_ARG;
+  *bytes = window_bwd_ws_bytes(B, h, dh, total_tokens);
+  return GDPA_OK;
+}
+
+gdpa_status_t gdpa_window_bwd(int32_t B, int32_t h, int32_t dh, int64_t total_tokens,
+                              int32_t max_n, int32_t window, float scale, const void* q,
+                              const int32_t* offsets, const void* k, const void* v,
+                              const void* o, const float* lse, const void* dout, void* dq,
+                              void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  g_launches = 0;
+  gdpa_status_t s = check_window(B, h, dh, total_tokens, max_n, window, scale);
+  if (s != GDPA_OK) return s;
+  if (B > 4096) return GDPA_ERR_UNSUPPORTED;
+  const bool empty = total_tokens == 0;
+  if (!offsets || (!empty && (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv)))
+    return GDPA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || ((uintptr_t)offsets & 3u) ||
+      ((uintptr_t)lse & 3u))
+    return GDPA_ERR_INVALID_ARG;
+  s = check_ws(workspace, workspace_bytes, window_bwd_ws_bytes(B, h, dh, total_tokens));
+  if (s != GDPA_OK) return s;
+  char* base = (char*)workspace;
+  WsHeader* ws = (WsHeader*)base;
+  Tile* tiles = (Tile*)(base + sizeof(WsHeader));
+  float* dq_acc = (float*)(base + jkv_list_bytes(B, h, total_tokens));
+  float* dsum = (float*)((char*)dq_acc + align_up((size_t)total_tokens * h * dh * 4, 256));
+  return cuda_status(launch_sm100_window_bwd(
+      B, h, dh, total_tokens, max_n, window, scale, offsets, q, k, v, o, lse, dout, dq, dk, dv,
+      dq_acc, dsum, ws, tiles, jkv_capacity(B, h, total_tokens), (cudaStream_t)stream));
+}
+
+gdpa_status_t gdpa_pool_bwd_workspace_size(int32_t B, int32_t h, int32_t dh, int32_t S,
+                                           int64_t total_tokens, size_t* bytes) {
+  const gdpa_status_t s = check_pool(B, h, dh, S, 0, 0, 1.f);
+  if (s != GDPA_OK) return s;
+  if (!bytes || total_tokens < 0) return GDPA_ERR_INVALID_ARG;
+  *bytes = pool_bwd_ws_bytes(B, h, S, total_tokens);
+  return GDPA_OK;
+}
+
+gdpa_status_t gdpa_pool_bwd(int32_t B, int32_t h, int32_t dh, int32_t S, int64_t total_tokens,
+                            int32_t max_n, float scale, const void* seeds,
+                            const int32_t* offsets, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dout, float* dseeds, void* dk,
+                            void* dv, void* workspace, size_t workspace_bytes, void* stream) {
+  g_launches = 0;
+  gdpa_status_t s = check_pool(B, h, dh, S, total_tokens, max_n, scale);
+  if (s != GDPA_OK) return s;
+  const bool empty = total_tokens == 0;
+  if (!offsets || !seeds || !o || !lse || !dout || !dseeds || (!empty && (!k || !v || !dk || !dv)))
+    return GDPA_ERR_INVALID_ARG;
+  if (!aligned16(seeds) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dseeds) || !aligned16(dk) || !aligned16(dv) || ((uintptr_t)offsets & 3u) ||
+      ((uintptr_t)lse & 3u))
+    return GDPA_ERR_INVALID_ARG;
+  s = check_ws(workspace, workspace_bytes, pool_bwd_ws_bytes(B, h, S, total_tokens));
+  if (s != GDPA_OK) return s;
+  char* base = (char*)workspace;
+  WsHeader* ws = (WsHeader*)base;
+  Tile* tiles = (Tile*)(base + sizeof(WsHeader));
+  float* dsum = (float*)(base + jkv_list_bytes(B, h, total_tokens));
+  return cuda_status(launch_sm100_pool_bwd(B, h, dh, S, total_tokens, max_n, scale, offsets,
+                                           seeds, k, v, o, lse, dout, dseeds, dk, dv, dsum, ws,
+                                           tiles, jkv_capacity(B, h, total_tokens),
+                                           (cudaStream_t)stream));
 }
 
 gdpa_status_t gdpa_workspace_status(const void* workspace, void* stream, int32_t* status) {

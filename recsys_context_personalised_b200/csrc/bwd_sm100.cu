@@ -48,13 +48,15 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // ---------------------------------------------------------------- prep / convert
 
-// Zeroes the fp32 dQ workspace and, for softmax, writes D[head, t] =
-// sum_d dO[t, head, d] * O[t, head, d] (one warp per (t, head) row).
+// Zeroes the fp32 dQ workspace (n4 float4s) and, for softmax, writes the row
+// sums D = sum_d dO[row, d] * O[row, d] of the `rows` rows of DH elements:
+// at D[head, t] for token rows (t, head), or at D[row] when `flat` (the
+// pooled outputs [B, h, S, DH]).
 template <int DH>
 __global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ g,
                                 float* __restrict__ dsum, float4* __restrict__ dq_acc,
-                                int64_t rows, int h, int64_t T, int softmax) {
-  const int64_t n4 = rows * DH / 4;
+                                int64_t n4, int64_t rows, int h, int64_t T, int softmax,
+                                int flat) {
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t nth = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = tid; i < n4; i += nth) dq_acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -90,9 +92,15 @@ __global__ void bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __rest
 #pragma unroll
       for (int off = CPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
       const int64_t row = r0 + u * RPW + sub;
-      if (piece == 0 && row < rows) dsum[(int64_t)(row % h) * T + row / h] = acc;
+      if (piece == 0 && row < rows) dsum[flat ? row : (int64_t)(row % h) * T + row / h] = acc;
     }
   }
+}
+
+// x *= s over n floats (the pooled seeds' gradient, accumulated unscaled).
+__global__ void scale_f32_kernel(float* __restrict__ x, int64_t n, float scale) {
+  const int64_t nth = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += nth) x[i] *= scale;
 }
 
 // dQ = bf16(s * dq_acc), 8 elements per thread and iteration.
@@ -121,6 +129,8 @@ struct BwdArgs {
   float* db1;            // [B, h, m] its gradient, zeroed beforehand (may be NULL)
   int64_t T;
   int h, m;
+  int S;                 // seed pooling: seeds per head (query rows of every item)
+  int window;            // sliding window: keys t - window < t' <= t
   float scale, scale_log2;
 };
 
@@ -711,7 +721,14 @@ __device__ __forceinline__ uint32_t stage_chunk(uint32_t box, int r, int j) {
   return box + (uint32_t)(r * 2 * DH) + ((uint32_t)(j ^ sw) << 4);
 }
 
-template <int DH, int PHI, bool BIAS>
+// Modes of the half kernel: GDPA (keys and values per sample [B, h, m, dh]),
+// seed-query pooling (the seeds [h, S, dh] are the one query tile of every
+// item; keys and values are the jagged tokens) and the causal sliding window
+// (queries, keys and values are the jagged tokens; an item visits only the
+// query tiles whose window reaches its key block).
+constexpr int kModeGdpa = 0, kModePool = 1, kModeWindow = 2;
+
+template <int DH, int PHI, bool BIAS, int MODE>
 __global__ void __launch_bounds__(kHalfThreads, 1)
 gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmG,
@@ -722,6 +739,8 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmDK, const BwdArgs a) {
   using C = BwdHalfCfg<DH>;
   constexpr bool SOFTMAX = PHI == GDPA_PHI_SOFTMAX;
+  constexpr bool POOL = MODE == kModePool, WIN = MODE == kModeWindow, JAG = MODE != kModeGdpa;
+  static_assert(!JAG || (SOFTMAX && !BIAS), "pooling and the window are softmax attention");
   constexpr uint32_t IDESC_T = idesc_bf16(128, 64, 0, 0);    // S^T, dP^T of a half: N = 64 rows
   constexpr uint32_t IDESC_KV = idesc_bf16(128, DH, 0, 1);   // dV, dK (B MN-major)
   constexpr uint32_t IDESC_Q = idesc_bf16(128, DH, 1, 1);    // dQ (A and B MN-major)
@@ -785,6 +804,22 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
     while (t < count && a.tiles[t].rows == 0) t += gridDim.x;
     return t;
   };
+  // query tiles of an item: the first (fi, in 128-row tiles of the sample)
+  // and the count.  GDPA: all of the sample's tiles; pooling: the seed tile;
+  // window: the tiles whose rows t satisfy row0 <= t < row0 + 128 + window - 1.
+  auto tiles_of = [&](const Tile& it, int& fi) -> int {
+    if constexpr (POOL) {
+      fi = 0;
+      return 1;
+    } else if constexpr (WIN) {
+      fi = it.row0 >> 7;
+      const int last = min(it.rows - 1, it.row0 + 127 + a.window - 1);
+      return (last >> 7) - fi + 1;
+    } else {
+      fi = 0;
+      return (it.rows + 127) >> 7;
+    }
+  };
 
   if (wg == 0) {
     setmaxnreg_dec<72>();
@@ -796,15 +831,21 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
       for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
         const Tile it = a.tiles[t];
         if (it.rows == 0) continue;
-        const int nq = (it.rows + 127) >> 7;
+        int fi;
+        const int nq = tiles_of(it, fi);
         const int t0 = a.offsets[it.b];
         const uint32_t slot = kvi & 1u;
         if (!mbar_wait(bar(C::B_KVEMPTY + slot), ((kvi >> 1) & 1u) ^ 1u, abort_flag, kTimeoutNs))
           break;
         const uint32_t sK = sKV + slot * 2 * C::TILEB;
         mbar_expect_tx(bar(C::B_KVFULL + slot), 2 * C::TILEB);
-        tma_load_4d(sK, &tmK, bar(C::B_KVFULL + slot), 0, it.row0, it.head, it.b);
-        tma_load_4d(sK + C::TILEB, &tmV, bar(C::B_KVFULL + slot), 0, it.row0, it.head, it.b);
+        if constexpr (JAG) {          // tokens [T, h, DH]: rows past the sample are masked later
+          tma_load_3d(sK, &tmK, bar(C::B_KVFULL + slot), 0, it.head, t0 + it.row0);
+          tma_load_3d(sK + C::TILEB, &tmV, bar(C::B_KVFULL + slot), 0, it.head, t0 + it.row0);
+        } else {
+          tma_load_4d(sK, &tmK, bar(C::B_KVFULL + slot), 0, it.row0, it.head, it.b);
+          tma_load_4d(sK + C::TILEB, &tmV, bar(C::B_KVFULL + slot), 0, it.row0, it.head, it.b);
+        }
         for (int i = 0; i < nq; ++i) {
           if (!mbar_wait(bar(C::B_STEMPTY + stage), sphase ^ 1u, abort_flag, kTimeoutNs)) {
             ok = false;
@@ -812,8 +853,15 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
           }
           const uint32_t dst = sStg + stage * 2 * C::TILEB;
           mbar_expect_tx(bar(C::B_STFULL + stage), 2 * C::TILEB);
-          tma_load_3d(dst, &tmQ, bar(C::B_STFULL + stage), 0, it.head, t0 + 128 * i);
-          tma_load_3d(dst + C::TILEB, &tmG, bar(C::B_STFULL + stage), 0, it.head, t0 + 128 * i);
+          if constexpr (POOL) {       // seeds [h, S, DH], dO [B*h, S, DH]; rows >= S read as zero
+            tma_load_3d(dst, &tmQ, bar(C::B_STFULL + stage), 0, 0, it.head);
+            tma_load_3d(dst + C::TILEB, &tmG, bar(C::B_STFULL + stage), 0, 0,
+                        it.b * a.h + it.head);
+          } else {
+            tma_load_3d(dst, &tmQ, bar(C::B_STFULL + stage), 0, it.head, t0 + 128 * (fi + i));
+            tma_load_3d(dst + C::TILEB, &tmG, bar(C::B_STFULL + stage), 0, it.head,
+                        t0 + 128 * (fi + i));
+          }
           if (++stage == (uint32_t)C::NSTG) {
             stage = 0;
             sphase ^= 1u;
@@ -872,8 +920,9 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
       };
       // One pass over every (item, query tile) of this CTA.
       int t = next_item(blockIdx.x);
+      int fi_unused;
       if (t < count) {
-        int nq = (a.tiles[t].rows + 127) >> 7;
+        int nq = tiles_of(a.tiles[t], fi_unused);
         uint32_t slot = 0;
         ok = wait_bar(C::B_KVFULL + 0, 0) && wait_bar(C::B_STFULL + stage, sphase) &&
              issue_st(0, stage, 0, slot) && issue_st(0, stage, 1, slot);
@@ -943,7 +992,7 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
           if (!has_next) break;
           if (last) {
             t = tn;
-            nq = (a.tiles[t].rows + 127) >> 7;
+            nq = tiles_of(a.tiles[t], fi_unused);
             slot = nslot;
             kvi = nkvi;
             i = 0;
@@ -961,7 +1010,8 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
       for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
         const Tile it = a.tiles[t];
         if (it.rows == 0) continue;
-        const int nq = (it.rows + 127) >> 7;
+        int fi;
+        const int nq = tiles_of(it, fi);
         const int t0 = a.offsets[it.b];
         for (int i = 0; i < nq; ++i, ++q) {
           const uint32_t slot = q & 1u;
@@ -974,10 +1024,11 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
           float* ring = stats + slot * 256;
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int r = 32 * u + lane, rg = 128 * i + r;
+            const int r = 32 * u + lane, rg = 128 * (fi + i) + r;
             float l = 0.f, d = 0.f;
-            if (rg < it.rows) {
-              const int64_t at = (int64_t)it.head * a.T + t0 + rg;
+            if (POOL ? r < a.S : rg < it.rows) {
+              const int64_t at = POOL ? ((int64_t)it.b * a.h + it.head) * a.S + r
+                                      : (int64_t)it.head * a.T + t0 + rg;
               l = __ldg(a.lse + at) * 1.4426950408889634f;
               d = __ldg(a.dsum + at);
             }
@@ -1003,15 +1054,17 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
       const Tile it = a.tiles[t];
       const int n = it.rows;
       if (n == 0) continue;
-      const int nq = (n + 127) >> 7;
+      int fi;
+      const int nq = tiles_of(it, fi);
       // biased variant: this key's bias (log2 units for softmax, halved for
       // SiLU) and this thread's sum of dS over its half of the tokens (for db1)
       const int key = it.row0 + lrow;
+      const bool key_ok = !JAG || key < n;              // jagged keys: rows past the sample
       const float b1k = BIAS ? key_bias(a, it, key) : 0.f;
       const float b1l = b1k * 1.4426950408889634f, hb = 0.5f * b1k;
       float db1_acc = 0.f;
       for (int i = 0; i < nq; ++i, ++qs) {
-        const int rbase = 128 * i + 64 * grp;          // first sample row of this group's half
+        const int rbase = 128 * (fi + i) + 64 * grp;   // first sample row (seed) of this half
         const uint32_t dsb = sDS + (qs & 1u) * C::DSB + grp * 16384;
         const float* st_l = stats + (qs & 1u) * 256 + 64 * grp;
         const float* st_d = st_l + 128;
@@ -1062,7 +1115,14 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                 p = fmaf(x, sc, b1k);
                 ds = g;
               }
-              const bool valid = rbase + r < n;
+              const int qr = rbase + r;                   // query row (pooling: seed)
+              bool valid;
+              if constexpr (POOL)
+                valid = key_ok && qr < a.S;
+              else if constexpr (WIN)
+                valid = key_ok && qr < n && key <= qr && key > qr - a.window;
+              else
+                valid = qr < n;
               pv[e] = valid ? p : 0.f;
               dv2[e] = valid ? ds : 0.f;
               if constexpr (BIAS) db1_acc += dv2[e];
@@ -1146,6 +1206,25 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
       }
     };
+    // one key row of DH columns from TMEM, times `mul`, as bf16 straight to
+    // global memory at dst (NULL: read only; every lane takes part in the loads)
+    auto store_row = [&](uint32_t src, __nv_bfloat16* dst, float mul) {
+#pragma unroll
+      for (int c = 0; c < DH; c += 16) {
+        uint32_t v[16];
+        tmem_ld_x16(src + c, v);
+        tmem_wait_ld();
+        uint32_t pk[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          pk[u] = pack_bf16x2(__uint_as_float(v[2 * u]) * mul, __uint_as_float(v[2 * u + 1]) * mul);
+        if (dst) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+          d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+      }
+    };
     for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
       const Tile it = a.tiles[t];
       const int n = it.rows;
@@ -1163,7 +1242,8 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         continue;
       }
-      const int nq = (n + 127) >> 7;
+      int fi;
+      const int nq = tiles_of(it, fi);
       const int t0 = a.offsets[it.b];
       for (int i = 0; i < nq; ++i, ++qs) {
         const uint32_t b = qs & 1u;
@@ -1190,8 +1270,13 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
         if (lrow == 0) {
           // rows past the sample are exact zeros (their dS entries are zero);
           // rows past T are clipped by the map
-          tma_reduce_add_3d(&tmDQ, stg, 0, it.head, t0 + 128 * i);
-          tma_reduce_add_3d(&tmDQ, stg + 16384, DH / 2, it.head, t0 + 128 * i);
+          if constexpr (POOL) {       // dseeds [h, S, DH]: rows >= S are clipped by the map
+            tma_reduce_add_3d(&tmDQ, stg, 0, 0, it.head);
+            tma_reduce_add_3d(&tmDQ, stg + 16384, DH / 2, 0, it.head);
+          } else {
+            tma_reduce_add_3d(&tmDQ, stg, 0, it.head, t0 + 128 * (fi + i));
+            tma_reduce_add_3d(&tmDQ, stg + 16384, DH / 2, it.head, t0 + 128 * (fi + i));
+          }
           bulk_commit_group();
         }
         if (i + 1 == nq) {
@@ -1203,6 +1288,17 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
             break;
           }
           tc_fence_after();
+          if (JAG && it.row0 + 128 > n) {
+            // the key block ends inside the next sample's tokens: each thread
+            // writes its own key row when it belongs to this sample
+            const int64_t row = ((int64_t)(t0 + it.row0 + lrow) * a.h + it.head) * DH;
+            const bool mine = it.row0 + lrow < n;
+            store_row(tmem + lane_off + C::COL_DV, mine ? a.dv + row : nullptr, 1.f);
+            store_row(tmem + lane_off + C::COL_DK, mine ? a.dk + row : nullptr, sc);
+            tc_fence_before();
+            mbar_arrive(bar(C::B_ACCEMPTY));
+            ++ic;
+          } else {
           if (lrow == 0) bulk_wait_group_read0();
           if (!group_sync()) {
             ok = false;
@@ -1218,11 +1314,17 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
             break;
           }
           if (lrow == 0) {
-            tma_store_4d(&tmDV, stg, 0, it.row0, it.head, it.b);
-            tma_store_4d(&tmDK, stg + 16384, 0, it.row0, it.head, it.b);
+            if constexpr (JAG) {      // dV, dK [T, h, DH]: the whole block is this sample's
+              tma_store_3d(&tmDV, stg, 0, it.head, t0 + it.row0);
+              tma_store_3d(&tmDK, stg + 16384, 0, it.head, t0 + it.row0);
+            } else {
+              tma_store_4d(&tmDV, stg, 0, it.row0, it.head, it.b);
+              tma_store_4d(&tmDK, stg + 16384, 0, it.row0, it.head, it.b);
+            }
             bulk_commit_group();
           }
           ++ic;
+          }
         }
         if (lrow == 0) {                               // the staging area may be rewritten
           bulk_wait_group_read0();
@@ -1331,7 +1433,7 @@ cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* 
   args.scale_log2 = p.scale * 1.4426950408889634f;
   if constexpr (DH <= 64) {
     using H = BwdHalfCfg<DH>;
-    auto hk = gdpa_bwd_half_kernel<DH, PHI, BIAS>;
+    auto hk = gdpa_bwd_half_kernel<DH, PHI, BIAS, kModeGdpa>;
     CUtensorMap mdq, mdv, mdk, unused_q, unused_g;
     if (!make_dq_map<DH>(p, dq_acc, &mdq)) return cudaErrorInvalidValue;
     // the outputs dV, dK have the layout (and so the maps) of the inputs K, V
@@ -1382,7 +1484,151 @@ cudaError_t launch_bwd_bias(const gdpa_problem_t& p, const void* q, const int32_
                                   tiles, st);
 }
 
+// Backward of seed pooling (POOL) or of the sliding window on the half
+// kernel.  Maps: K, V, dK, dV are the jagged tokens [T, h, DH]; Q and dO are
+// the tokens too (window) or the seeds [h, S, DH] and the pooled dO
+// [B, h, S, DH] (pooling); the fp32 target of the dQ reduces is the token
+// accumulator [T, h, DH] (window) or the seeds' gradient [h, S, DH] (pooling).
+template <int DH, int MODE>
+cudaError_t launch_jag_bwd_t(int B, int h, int S, int64_t T, int window, float scale,
+                             const int32_t* offsets, const void* q, const void* g,
+                             const void* k, const void* v, const float* lse, const float* dsum,
+                             float* acc, void* dk, void* dv, WsHeader* ws, const Tile* tiles,
+                             cudaStream_t st) {
+  constexpr bool POOL = MODE == kModePool;
+  constexpr int CH = DH < 64 ? DH : 64;
+  using H = BwdHalfCfg<DH>;
+  auto enc = tensor_map_encoder();
+  if (!enc) return cudaErrorInvalidValue;
+  const CUtensorMapSwizzle sw = DH < 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  auto map3 = [&](CUtensorMap* m, CUtensorMapDataType ty, int esz, const void* ptr,
+                  cuuint64_t d1, cuuint64_t d2, cuuint32_t bx, cuuint32_t b1, cuuint32_t b2,
+                  CUtensorMapSwizzle swz) -> bool {
+    const cuuint64_t dims[3] = {(cuuint64_t)DH, d1, d2};
+    const cuuint64_t str[2] = {(cuuint64_t)DH * esz, d1 * DH * esz};
+    const cuuint32_t box[3] = {bx, b1, b2};
+    return enc(m, ty, 3, const_cast<void*>(ptr), dims, str, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const cuuint64_t Tm = T > 0 ? (cuuint64_t)T : 1;
+  const CUtensorMapSwizzle swq = DH / 2 * 4 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                                   : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUtensorMap mq, mg, mk, mv, mdq, mdv, mdk;
+  bool okm = map3(&mk, BF, 2, k, h, Tm, CH, 1, 128, sw) && map3(&mv, BF, 2, v, h, Tm, CH, 1, 128, sw) &&
+             map3(&mdk, BF, 2, dk, h, Tm, CH, 1, 128, sw) &&
+             map3(&mdv, BF, 2, dv, h, Tm, CH, 1, 128, sw);
+  if (POOL)
+    okm = okm && map3(&mq, BF, 2, q, S, h, CH, 128, 1, sw) &&
+          map3(&mg, BF, 2, g, S, (cuuint64_t)B * h, CH, 128, 1, sw) &&
+          map3(&mdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, acc, S, h, DH / 2, 128, 1, swq);
+  else
+    okm = okm && map3(&mq, BF, 2, q, h, Tm, CH, 1, 128, sw) &&
+          map3(&mg, BF, 2, g, h, Tm, CH, 1, 128, sw) &&
+          map3(&mdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, acc, h, Tm, DH / 2, 1, 128, swq);
+  if (!okm) return cudaErrorInvalidValue;
+  BwdArgs args = {};
+  args.tiles = tiles;
+  args.ws = ws;
+  args.offsets = offsets;
+  args.lse = lse;
+  args.dsum = dsum;
+  args.dq_acc = acc;
+  args.dk = reinterpret_cast<__nv_bfloat16*>(dk);
+  args.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+  args.T = T;
+  args.h = h;
+  args.m = 0;
+  args.S = S;
+  args.window = window;
+  args.scale = scale;
+  args.scale_log2 = scale * 1.4426950408889634f;
+  auto hk = gdpa_bwd_half_kernel<DH, GDPA_PHI_SOFTMAX, false, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(hk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H::SMEM);
+  if (e != cudaSuccess) return e;
+  KernelScope ks_(POOL ? "gdpa_pool_bwd_sm100" : "gdpa_window_bwd_sm100", st);
+  hk<<<device_sm_count(), kHalfThreads, H::SMEM, st>>>(mq, mg, mk, mv, mdq, mdv, mdk, args);
+  return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t launch_jag_bwd(int dh, int B, int h, int S, int64_t T, int window, float scale,
+                           const int32_t* offsets, const void* q, const void* g, const void* k,
+                           const void* v, const float* lse, const float* dsum, float* acc,
+                           void* dk, void* dv, WsHeader* ws, const Tile* tiles, cudaStream_t st) {
+  if (dh == 32)
+    return launch_jag_bwd_t<32, MODE>(B, h, S, T, window, scale, offsets, q, g, k, v, lse, dsum,
+                                      acc, dk, dv, ws, tiles, st);
+  if (dh == 64)
+    return launch_jag_bwd_t<64, MODE>(B, h, S, T, window, scale, offsets, q, g, k, v, lse, dsum,
+                                      acc, dk, dv, ws, tiles, st);
+  return cudaErrorInvalidValue;
+}
+
+template <int DH>
+cudaError_t launch_prep(const void* o, const void* g, float* dsum, float* acc, int64_t acc_elems,
+                        int64_t rows, int h, int64_t T, int flat, cudaStream_t st) {
+  const int sms = device_sm_count();
+  KernelScope ks_("gdpa_bwd_prep", st);
+  bwd_prep_kernel<DH><<<sms * 8, 256, 0, st>>>(reinterpret_cast<const uint4*>(o),
+                                               reinterpret_cast<const uint4*>(g), dsum,
+                                               reinterpret_cast<float4*>(acc), acc_elems / 4,
+                                               rows, h, T, 1, flat);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+// schedule (jagged key blocks) -> prep (zero the token dQ accumulator, D) ->
+// half kernel in window mode -> dQ conversion.
+cudaError_t launch_sm100_window_bwd(int B, int h, int dh, int64_t T, int max_n, int window,
+                                    float scale, const int32_t* offsets, const void* q,
+                                    const void* k, const void* v, const void* o,
+                                    const float* lse, const void* dout, void* dq, void* dk,
+                                    void* dv, float* dq_acc, float* dsum, WsHeader* ws,
+                                    Tile* tiles, int64_t cap, cudaStream_t st) {
+  cudaError_t e = launch_schedule_jkv(offsets, B, h, T, max_n, ws, tiles, cap, st);
+  if (e != cudaSuccess || T == 0) return e;
+  const int64_t rows = T * h;
+  e = dh == 32 ? launch_prep<32>(o, dout, dsum, dq_acc, rows * dh, rows, h, T, 0, st)
+               : launch_prep<64>(o, dout, dsum, dq_acc, rows * dh, rows, h, T, 0, st);
+  if (e != cudaSuccess) return e;
+  e = launch_jag_bwd<kModeWindow>(dh, B, h, 0, T, window, scale, offsets, q, dout, k, v, lse,
+                                  dsum, dq_acc, dk, dv, ws, tiles, st);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+  KernelScope ks_("gdpa_dq_convert", st);
+  dq_convert_kernel<<<sms * 8, 256, 0, st>>>(reinterpret_cast<const float4*>(dq_acc),
+                                              reinterpret_cast<uint4*>(dq), rows * dh / 8, scale);
+  return cudaGetLastError();
+}
+
+// schedule (jagged key blocks) -> prep (zero dseeds, D of the pooled rows) ->
+// half kernel in pooling mode (dseeds accumulates over every sample) -> scale.
+cudaError_t launch_sm100_pool_bwd(int B, int h, int dh, int S, int64_t T, int max_n, float scale,
+                                  const int32_t* offsets, const void* seeds, const void* k,
+                                  const void* v, const void* o, const float* lse,
+                                  const void* dout, float* dseeds, void* dk, void* dv,
+                                  float* dsum, WsHeader* ws, Tile* tiles, int64_t cap,
+                                  cudaStream_t st) {
+  cudaError_t e = launch_schedule_jkv(offsets, B, h, T, max_n, ws, tiles, cap, st);
+  if (e != cudaSuccess) return e;
+  const int64_t rows = (int64_t)B * h * S, nseed = (int64_t)h * S * dh;
+  e = dh == 32 ? launch_prep<32>(o, dout, dsum, dseeds, nseed, rows, h, T, 1, st)
+               : launch_prep<64>(o, dout, dsum, dseeds, nseed, rows, h, T, 1, st);
+  if (e != cudaSuccess) return e;
+  if (T > 0) {
+    e = launch_jag_bwd<kModePool>(dh, B, h, S, T, 0, scale, offsets, seeds, dout, k, v, lse, dsum,
+                                  dseeds, dk, dv, ws, tiles, st);
+    if (e != cudaSuccess) return e;
+  }
+  const int sms = device_sm_count();
+  KernelScope ks_("gdpa_seed_scale", st);
+  scale_f32_kernel<<<sms * 4, 256, 0, st>>>(dseeds, nseed, scale);
+  return cudaGetLastError();
+}
 
 int64_t sm100_bwd_items(const gdpa_problem_t& p) {
   return (int64_t)p.B * p.h * ((p.m + 127) / 128);
@@ -1407,8 +1653,8 @@ cudaError_t launch_sm100_bwd(const gdpa_problem_t& p, const void* q, const int32
     // with an output bias the softmax row sums come from the bias kernel (O - b2)
     prep<<<sms * 8, 256, 0, st>>>(reinterpret_cast<const uint4*>(o),
                                   reinterpret_cast<const uint4*>(dout), dsum,
-                                  reinterpret_cast<float4*>(dq_acc), rows, p.h, p.total_tokens,
-                                  softmax && !bs.b2 ? 1 : 0);
+                                  reinterpret_cast<float4*>(dq_acc), rows * p.dh / 4, rows, p.h,
+                                  p.total_tokens, softmax && !bs.b2 ? 1 : 0, 0);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -73,6 +73,10 @@ cudaError_t launch_schedule_kv(const gdpa_problem_t& p, const int32_t* offsets, 
 
 // Seed-pooling work list (one item per (sample with tokens, pair of heads),
 // longest first; B <= 4096) and the outputs of samples without tokens.
+// Backward list of the jagged-key variants: (sample, head, 128-token key block)
+// items of the samples with tokens, longest samples first (B <= 4096).
+cudaError_t launch_schedule_jkv(const int32_t* offsets, int B, int h, int64_t T, int max_n,
+                                WsHeader* ws, Tile* tiles, int64_t cap, cudaStream_t st);
 cudaError_t launch_schedule_pool(const int32_t* offsets, int B, int h, int64_t T, int max_n,
                                  WsHeader* ws, Tile* tiles, cudaStream_t st);
 cudaError_t launch_pool_empty(const int32_t* offsets, int B, int h, int S, int dh, void* o,

@@ -218,6 +218,100 @@ schedule_pool_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t 
   if (tid == 0) ws->tile_count = (int)items;
 }
 
+// Backward work list of the variants whose keys are the jagged tokens (seed
+// pooling, the sliding window): one item per (sample, head, 128-token key
+// block) of the samples that have tokens, samples in decreasing length order
+// (B <= 4096), head-major within a sample.  Item fields: b, head, row0 = first
+// key of the block (sample-local), rows = n_b.
+__global__ void __launch_bounds__(kSchedThreads)
+schedule_jkv_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T, int max_n,
+                    WsHeader* ws, Tile* __restrict__ tiles, int64_t cap) {
+  __shared__ int s_bad;
+  __shared__ long long s_carry;
+  __shared__ int s_scan[kSchedThreads];
+  __shared__ int2 s_key[kSortMax];   // (n_b, b)
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    s_bad = 0;
+    s_carry = 0;
+    ws->status = GDPA_OK;
+    if (offsets[0] != 0 || (int64_t)offsets[B] != T) s_bad = 1;
+  }
+  __syncthreads();
+  for (int b = tid; b < B; b += kSchedThreads) {
+    const int n = offsets[b + 1] - offsets[b];
+    if (n < 0 || n > max_n) s_bad = 1;
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (tid == 0) {
+      ws->status = GDPA_ERR_INVALID_ARG;
+      ws->tile_count = 0;
+    }
+    return;
+  }
+  int P2 = 1;
+  while (P2 < B) P2 <<= 1;
+  for (int i = tid; i < P2; i += kSchedThreads)
+    s_key[i] = i < B ? make_int2(offsets[i + 1] - offsets[i], i) : make_int2(-1, 0x7fffffff);
+  __syncthreads();
+  // bitonic sort: descending n, ascending b
+  for (int k = 2; k <= P2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < P2; i += kSchedThreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const int2 x = s_key[i], y = s_key[ixj];
+          const bool x_first = x.x > y.x || (x.x == y.x && x.y < y.y);
+          const bool up = (i & k) == 0;
+          if (up ? !x_first : x_first) {
+            s_key[i] = y;
+            s_key[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // exclusive scan of the key-block counts in sorted order, then the items
+  for (int base = 0; base < B; base += kSchedThreads) {
+    const int r = base + tid;
+    const int n = r < B ? max(s_key[r].x, 0) : 0;
+    const int nb = (n + 127) >> 7;
+    s_scan[tid] = nb;
+    __syncthreads();
+    for (int d = 1; d < kSchedThreads; d <<= 1) {
+      const int add = tid >= d ? s_scan[tid - d] : 0;
+      __syncthreads();
+      s_scan[tid] += add;
+      __syncthreads();
+    }
+    const long long excl = s_carry + s_scan[tid] - nb;
+    if (nb > 0) {
+      const int b = s_key[r].y;
+      for (int j = 0; j < h; ++j)
+        for (int kb = 0; kb < nb; ++kb) {
+          const long long idx = (long long)h * excl + (long long)j * nb + kb;
+          if (idx < cap) {
+            Tile w;
+            w.b = b;
+            w.head = j;
+            w.row0 = 128 * kb;
+            w.rows = n;
+            tiles[idx] = w;
+          }
+        }
+    }
+    __syncthreads();
+    if (tid == kSchedThreads - 1) s_carry += s_scan[kSchedThreads - 1];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    const long long total = (long long)h * s_carry;
+    ws->tile_count = (int)(total < cap ? total : cap);
+  }
+}
+
 // Outputs of the samples without tokens: O = 0 and LSE = -inf (every seed
 // pools over an empty set).  One thread per 8 columns of an output row.
 __global__ void pool_empty_kernel(const int32_t* __restrict__ offsets, int B, int h, int S,
@@ -261,6 +355,13 @@ cudaError_t launch_schedule_pool(const int32_t* offsets, int B, int h, int64_t T
                                  WsHeader* ws, Tile* tiles, cudaStream_t st) {
   KernelScope ks_("gdpa_schedule_pool", st);
   schedule_pool_kernel<<<1, kSchedThreads, 0, st>>>(offsets, B, h, T, max_n, ws, tiles);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_schedule_jkv(const int32_t* offsets, int B, int h, int64_t T, int max_n,
+                                WsHeader* ws, Tile* tiles, int64_t cap, cudaStream_t st) {
+  KernelScope ks_("gdpa_schedule_jkv", st);
+  schedule_jkv_kernel<<<1, kSchedThreads, 0, st>>>(offsets, B, h, T, max_n, ws, tiles, cap);
   return cudaGetLastError();
 }
 

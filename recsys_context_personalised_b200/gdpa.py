@@ -95,6 +95,15 @@ def load(path: str = LIB_PATH):
     lib.gdpa_window_fwd.argtypes = [i32, i32, i32, ctypes.c_int64, i32, i32, ctypes.c_float, vp,
                                     vp, vp, vp, vp, vp, vp, sz, vp]
     lib.gdpa_window_fwd.restype = ctypes.c_int
+    i64, f32 = ctypes.c_int64, ctypes.c_float
+    lib.gdpa_pool_bwd_workspace_size.argtypes = [i32, i32, i32, i32, i64, ctypes.POINTER(sz)]
+    lib.gdpa_pool_bwd_workspace_size.restype = ctypes.c_int
+    lib.gdpa_pool_bwd.argtypes = [i32, i32, i32, i32, i64, i32, f32] + [vp] * 10 + [sz, vp]
+    lib.gdpa_pool_bwd.restype = ctypes.c_int
+    lib.gdpa_window_bwd_workspace_size.argtypes = [i32, i32, i32, i64, ctypes.POINTER(sz)]
+    lib.gdpa_window_bwd_workspace_size.restype = ctypes.c_int
+    lib.gdpa_window_bwd.argtypes = [i32, i32, i32, i64, i32, i32, f32] + [vp] * 11 + [sz, vp]
+    lib.gdpa_window_bwd.restype = ctypes.c_int
     for name in EXPORTED[:8]:
         getattr(lib, name).restype = ctypes.c_int
     if path == LIB_PATH:
@@ -319,6 +328,57 @@ def window_fwd(q: torch.Tensor, offsets, k: torch.Tensor, v: torch.Tensor, windo
     if rc:
         raise GdpaError(rc, "gdpa_window_fwd")
     return o, lse
+
+
+def pool_bwd(seeds: torch.Tensor, offsets, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+             lse: torch.Tensor, dout: torch.Tensor, scale: float, offsets_host, dk=None, dv=None,
+             dseeds=None, ws=None, stream=None, shape=None):
+    """Run gdpa_pool_bwd: gradients of gdpa_pool_fwd for dout [B, h, S, dh];
+    returns (dseeds fp32 [h, S, dh], dk, dv bf16 [T, h, dh])."""
+    lib = load()
+    h, S, dh = seeds.shape
+    B, T, max_n = _batch_shape(offsets_host, shape)
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if dseeds is None:
+        dseeds = torch.empty((h, S, dh), dtype=torch.float32, device=seeds.device)
+    if ws is None:
+        n = ctypes.c_size_t()
+        rc = lib.gdpa_pool_bwd_workspace_size(B, h, dh, S, T, ctypes.byref(n))
+        if rc:
+            raise GdpaError(rc, "gdpa_pool_bwd_workspace_size")
+        ws = workspace(n.value, seeds.device)
+    rc = lib.gdpa_pool_bwd(B, h, dh, S, T, max_n, scale, _ptr(seeds), _ptr(offsets), _ptr(k),
+                           _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dseeds), _ptr(dk),
+                           _ptr(dv), _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise GdpaError(rc, "gdpa_pool_bwd")
+    return dseeds, dk, dv
+
+
+def window_bwd(q: torch.Tensor, offsets, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+               lse: torch.Tensor, dout: torch.Tensor, window: int, scale: float, offsets_host,
+               dq=None, dk=None, dv=None, ws=None, stream=None, shape=None):
+    """Run gdpa_window_bwd: gradients of gdpa_window_fwd for dout [T, h, dh];
+    returns (dq, dk, dv) bf16 [T, h, dh]."""
+    lib = load()
+    T, h, dh = q.shape
+    B, _, max_n = _batch_shape(offsets_host, shape)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if ws is None:
+        n = ctypes.c_size_t()
+        rc = lib.gdpa_window_bwd_workspace_size(B, h, dh, T, ctypes.byref(n))
+        if rc:
+            raise GdpaError(rc, "gdpa_window_bwd_workspace_size")
+        ws = workspace(n.value, q.device)
+    rc = lib.gdpa_window_bwd(B, h, dh, T, max_n, window, scale, _ptr(q), _ptr(offsets), _ptr(k),
+                             _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                             _ptr(dv), _ptr(ws), ws.numel(), _stream(stream))
+    if rc:
+        raise GdpaError(rc, "gdpa_window_bwd")
+    return dq, dk, dv
 
 
 def workspace_status(ws: torch.Tensor, stream=None) -> int:

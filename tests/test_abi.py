@@ -125,3 +125,28 @@ def test_pool_rejects_unsupported_shapes_on_host():
     assert lib.gdpa_pool_workspace_size(0, 2, 64, 16, ctypes.byref(n)) == 1
     assert lib.gdpa_pool_workspace_size(4, 3, 64, 16, ctypes.byref(n)) == 0
     assert n.value >= 256 + 16 * 4 * 2
+
+
+def test_pool_and_window_backward_check_arguments_on_host():
+    """Shape limits and workspace sizes of the two backward calls (no launch)."""
+    lib = pkg.load()
+    G.load()
+    n = ctypes.c_size_t()
+    assert lib.gdpa_pool_bwd_workspace_size(4, 2, 128, 16, 100, ctypes.byref(n)) == 2
+    assert lib.gdpa_pool_bwd_workspace_size(4, 2, 64, 129, 100, ctypes.byref(n)) == 2
+    assert lib.gdpa_pool_bwd_workspace_size(4, 2, 64, 16, -1, ctypes.byref(n)) == 1
+    assert lib.gdpa_pool_bwd_workspace_size(4, 3, 64, 16, 1000, ctypes.byref(n)) == 0
+    # list of h * (T / 128 + B) items and the row sums D [B, h, S]
+    assert n.value >= 16 * 3 * (1000 // 128 + 4) + 4 * 4 * 3 * 16
+    assert lib.gdpa_window_bwd_workspace_size(4097, 2, 64, 100, ctypes.byref(n)) == 2
+    assert lib.gdpa_window_bwd_workspace_size(4, 2, 128, 100, ctypes.byref(n)) == 2
+    assert lib.gdpa_window_bwd_workspace_size(4, 2, 64, 1000, ctypes.byref(n)) == 0
+    # the list, the fp32 dQ accumulator [T, h, dh] and D [h, T]
+    assert n.value >= 1000 * 2 * 64 * 4 + 2 * 1000 * 4
+    # argument checks come before any CUDA call: window 0, null offsets
+    assert lib.gdpa_window_bwd(4, 2, 64, 100, 50, 0, 1.0, *([4096] * 11), 1 << 20, None) == 1
+    assert lib.gdpa_window_bwd(4, 2, 64, 100, 50, 8, 1.0, 4096, None, *([4096] * 9), 1 << 20,
+                               None) == 1
+    assert lib.gdpa_pool_bwd(4, 2, 64, 129, 100, 50, 1.0, *([4096] * 10), 1 << 20, None) == 2
+    assert lib.gdpa_pool_bwd(4, 2, 64, 16, 100, 50, 1.0, 4096, None, *([4096] * 8), 1 << 20,
+                             None) == 1

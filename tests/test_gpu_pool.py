@@ -79,3 +79,59 @@ def test_pool_bad_offsets_reported():
     ws = pkg.workspace(4096, DEV)
     pkg.gdpa.pool_fwd(seeds.to(DEV), bad, k.to(DEV), v.to(DEV), 0.125, off, ws=ws)
     assert pkg.workspace_status(ws) == 1
+
+
+def _rel(x, r, scale_ref):
+    """max|x - r| over the larger of max|r| and max|scale_ref|: a sample with
+    one token pools it with weight 1, so its dS, dK and seed gradient are
+    exactly zero and are judged against the magnitude of dV."""
+    den = max(np.abs(r).max(), np.abs(scale_ref).max(), 1e-30)
+    return float(np.abs(x.float().cpu().numpy() - r).max() / den)
+
+
+@pytest.mark.parametrize("dh", [32, 64])
+@pytest.mark.parametrize("S", [1, 16, 64, 128])
+@pytest.mark.parametrize("n,h", [([130, 0, 17, 256, 1], 2), ([300, 5, 128], 3), ([1], 1),
+                                 ([0, 0, 40], 4)])
+def test_pool_backward_matches_oracle(n, h, S, dh):
+    """gdpa_pool_bwd (dseeds summed over the samples, dK and dV per token) on
+    the GPU forward's O and LSE, against the oracle's gradients."""
+    seeds, k, v, off = _case(len(n) * 17 + S + dh + h, n, h, S, dh)
+    g = torch.randn(len(n), h, S, dh, generator=torch.Generator().manual_seed(S + dh)).bfloat16()
+    scale = 1.0 / dh ** 0.5
+    offd = torch.tensor(off, dtype=torch.int32, device=DEV)
+    sd, kd, vd = seeds.to(DEV), k.to(DEV), v.to(DEV)
+    o, lse = pkg.gdpa.pool_fwd(sd, offd, kd, vd, scale, off)
+    dseeds, dk, dv = pkg.gdpa.pool_bwd(sd, offd, kd, vd, o, lse, g.to(DEV), scale, off)
+    torch.cuda.synchronize()
+    rs, rk, rv = oracle.pool_bwd(seeds, k, v, g, off, scale)
+    assert dseeds.dtype == torch.float32 and dseeds.shape == (h, S, dh)
+    if int(off[-1]) > 0:
+        assert _rel(dseeds, rs, rv) <= TOL
+        assert _rel(dk, rk, rv) <= TOL and _rel(dv, rv, rv) <= TOL
+    else:
+        assert float(dseeds.abs().max()) == 0.0
+
+
+def test_pool_backward_power_law_batch_and_guard():
+    """The power-law batch (256 samples of lengths 32..4096, h = 16, S = 64,
+    dh = 64); dK and dV sit inside sentinel-filled buffers that must stay
+    untouched, including after key blocks that end inside the next sample."""
+    import synthetic as syn
+    n = syn.lengths(syn.WORKLOADS[5])[:256]
+    h, S, dh = 16, 64, 64
+    seeds, k, v, off = _case(7, n, h, S, dh)
+    T = int(off[-1])
+    g = torch.randn(len(n), h, S, dh, generator=torch.Generator().manual_seed(5)).bfloat16()
+    offd = torch.tensor(off, dtype=torch.int32, device=DEV)
+    sd, kd, vd = seeds.to(DEV), k.to(DEV), v.to(DEV)
+    o, lse = pkg.gdpa.pool_fwd(sd, offd, kd, vd, 0.125, off)
+    guard = [torch.full((T + 256, h, dh), 3.0, dtype=torch.bfloat16, device=DEV) for _ in range(2)]
+    dseeds, dk, dv = pkg.gdpa.pool_bwd(sd, offd, kd, vd, o, lse, g.to(DEV), 0.125, off,
+                                       dk=guard[0][128:128 + T], dv=guard[1][128:128 + T])
+    torch.cuda.synchronize()
+    for b in guard:
+        assert (b[:128] == 3.0).all() and (b[128 + T:] == 3.0).all()
+    rs, rk, rv = oracle.pool_bwd(seeds, k, v, g, off, 0.125)
+    assert _rel(dseeds, rs, rv) <= TOL
+    assert _rel(dk, rk, rv) <= TOL and _rel(dv, rv, rv) <= TOL

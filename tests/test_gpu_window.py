@@ -47,3 +47,52 @@ def test_window_output_guard():
     pkg.gdpa.window_fwd(q.to(DEV), offd, k.to(DEV), v.to(DEV), 100, 0.125, off, o=o)
     torch.cuda.synchronize()
     assert (big[:64] == 7.0).all() and (big[64 + T:] == 7.0).all()
+
+
+def _rel(x, r, scale_ref):
+    """max|x - r| over the larger of max|r| and max|scale_ref|: with w = 1
+    each token attends to itself alone, so dQ and dK are exactly zero and are
+    judged against the magnitude of dV, the gradient of the same dO."""
+    den = max(np.abs(r).max(), np.abs(scale_ref).max(), 1e-30)
+    return float(np.abs(x.float().cpu().numpy() - r).max() / den)
+
+
+@pytest.mark.parametrize("dh", [32, 64])
+@pytest.mark.parametrize("w", [1, 37, 128, 200, 5000])
+@pytest.mark.parametrize("n,h", [([130, 0, 17, 300, 1], 2), ([513, 64], 3), ([256], 1)])
+def test_window_backward_matches_oracle(n, h, w, dh):
+    """gdpa_window_bwd on the GPU forward's O and LSE against the oracle's
+    dQ, dK, dV (key blocks whose window reaches several query tiles, blocks
+    that end inside the next sample, empty samples)."""
+    q, k, v, off = _case(len(n) * 3 + w + dh + h, n, h, dh)
+    T = int(off[-1])
+    g = torch.randn(T, h, dh, generator=torch.Generator().manual_seed(w + dh)).bfloat16()
+    scale = 1.0 / dh ** 0.5
+    offd = torch.tensor(off, dtype=torch.int32, device=DEV)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    o, lse = pkg.gdpa.window_fwd(qd, offd, kd, vd, w, scale, off)
+    dq, dk, dv = pkg.gdpa.window_bwd(qd, offd, kd, vd, o, lse, g.to(DEV), w, scale, off)
+    torch.cuda.synchronize()
+    rq, rk, rv = oracle.win_bwd(q, k, v, g, off, w, scale)
+    assert _rel(dq, rq, rv) <= TOL and _rel(dk, rk, rv) <= TOL and _rel(dv, rv, rv) <= TOL
+
+
+def test_window_backward_guard():
+    """dQ, dK, dV inside sentinel-filled buffers: nothing outside the T rows
+    is written."""
+    q, k, v, off = _case(11, [200, 50, 300], 2, 64)
+    T = int(off[-1])
+    g = torch.randn(T, 2, 64, generator=torch.Generator().manual_seed(2)).bfloat16()
+    offd = torch.tensor(off, dtype=torch.int32, device=DEV)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    o, lse = pkg.gdpa.window_fwd(qd, offd, kd, vd, 100, 0.125, off)
+    bufs = [torch.full((T + 256, 2, 64), 5.0, dtype=torch.bfloat16, device=DEV) for _ in range(3)]
+    pkg.gdpa.window_bwd(qd, offd, kd, vd, o, lse, g.to(DEV), 100, 0.125, off,
+                        dq=bufs[0][128:128 + T], dk=bufs[1][128:128 + T], dv=bufs[2][128:128 + T])
+    torch.cuda.synchronize()
+    for b in bufs:
+        assert (b[:128] == 5.0).all() and (b[128 + T:] == 5.0).all()
+    rq, rk, rv = oracle.win_bwd(q, k, v, g, off, 100, 0.125)
+    T_ = slice(128, 128 + T)
+    assert _rel(bufs[0][T_], rq, rv) <= TOL and _rel(bufs[1][T_], rk, rv) <= TOL
+    assert _rel(bufs[2][T_], rv, rv) <= TOL
