@@ -98,7 +98,7 @@ def load(path: str = LIB_PATH):
     i64, f32 = ctypes.c_int64, ctypes.c_float
     lib.gdpa_pool_bwd_workspace_size.argtypes = [i32, i32, i32, i32, i64, ctypes.POINTER(sz)]
     lib.gdpa_pool_bwd_workspace_size.restype = ctypes.c_int
-    lib.gdpa_pool_bwd.argtypes = [i32, i32, i32, i32, i64, i32, f32] + [vp] * 10 + [sz, vp]
+    lib.gdpa_pool_bwd.argtypes = [i32, i32, i32, i32, i64, i32, f32] + [vp] * 11 + [sz, vp]
     lib.gdpa_pool_bwd.restype = ctypes.c_int
     lib.gdpa_window_bwd_workspace_size.argtypes = [i32, i32, i32, i64, ctypes.POINTER(sz)]
     lib.gdpa_window_bwd_workspace_size.restype = ctypes.c_int

@@ -147,6 +147,31 @@ def test_pool_and_window_backward_check_arguments_on_host():
     assert lib.gdpa_window_bwd(4, 2, 64, 100, 50, 0, 1.0, *([4096] * 11), 1 << 20, None) == 1
     assert lib.gdpa_window_bwd(4, 2, 64, 100, 50, 8, 1.0, 4096, None, *([4096] * 9), 1 << 20,
                                None) == 1
-    assert lib.gdpa_pool_bwd(4, 2, 64, 129, 100, 50, 1.0, *([4096] * 10), 1 << 20, None) == 2
-    assert lib.gdpa_pool_bwd(4, 2, 64, 16, 100, 50, 1.0, 4096, None, *([4096] * 8), 1 << 20,
+    assert lib.gdpa_pool_bwd(4, 2, 64, 129, 100, 50, 1.0, *([4096] * 11), 1 << 20, None) == 2
+    assert lib.gdpa_pool_bwd(4, 2, 64, 16, 100, 50, 1.0, 4096, None, *([4096] * 9), 1 << 20,
                              None) == 1
+
+
+def _declared_arity():
+    """Parameter count of every GDPA_API function in include/gdpa.h."""
+    src = open(os.path.join(ROOT, "include", "gdpa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"GDPA_API\s+[\w\s\*]+?\b(gdpa_\w+)\s*\(([^)]*)\)", src):
+        args = m.group(2).strip()
+        out[m.group(1)] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_argtypes_match_the_header():
+    """Every entry point the binding types has exactly the header's number of
+    parameters (a missing one would hand the stream to an untyped argument)."""
+    lib = G.load()
+    arity = _declared_arity()
+    typed = 0
+    for name, n in arity.items():
+        fn = getattr(lib, name)
+        if fn.argtypes is not None:
+            assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+            typed += 1
+    assert typed >= 20
