@@ -748,7 +748,7 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(C::B_QFULL + i), 1);
-      mbar_init(bar(C::B_QEMPTY + i), 1);
+      mbar_init(bar(C::B_QEMPTY + i), 2);      // both issuers' last S of an item
       mbar_init(bar(C::B_SFULL + i), 1);
       mbar_init(bar(C::B_PFULL + i), 128);
       mbar_init(bar(C::B_OFULL + i), 1);
@@ -756,10 +756,10 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
       mbar_init(bar(C::B_SFREE + i), 128);
       mbar_init(bar(C::B_PFREE + i), 1);
     }
-    mbar_init(bar(C::B_DRAIN), 1);
+    mbar_init(bar(C::B_DRAIN), 2);
     for (int i = 0; i < C::NS; ++i) {
       mbar_init(bar(C::B_KVFULL + i), 1);
-      mbar_init(bar(C::B_KVEMPTY + i), 1);
+      mbar_init(bar(C::B_KVEMPTY + i), 2);     // two releases per load (see the issuers)
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -886,32 +886,45 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
           if (ok) ok = load_both(&tmV, pr, j);
         }
       }
-    } else if (warp == 1 && lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
-      uint32_t slot = 0, sphase = 0;
-      uint32_t s_cnt[2] = {0u, 0u};    // S products issued per tile slot
-      uint32_t pv_cnt[2] = {0u, 0u};   // PV groups issued per tile slot
-      uint32_t o_cnt[2] = {0u, 0u};    // items finished per tile slot
+    } else if ((warp == 1 || warp == 3) && lane == 0) {
+      // ---------------------------------------------------------- MMA issuers
+      // One issuer per tile slot x (warp 1: A, warp 3: B), so that neither
+      // tile's products wait behind the other's in one in-order stream.  Both
+      // replay the producer's load order to find the ring slot of each of
+      // their K/V blocks.  Every load is released twice on KVEMPTY: once by
+      // each issuer when A and B share it, else twice by its one reader.  The
+      // Q stage of an item is released twice on QEMPTY the same way.
+      const int x = warp == 1 ? 0 : 1;
+      uint32_t seq = 0;                 // ring loads replayed so far
+      uint32_t s_cnt = 0, pv_cnt = 0, o_cnt = 0;
       bool ok = true;
-      auto take = [&]() -> int {
-        if (!mbar_wait(bar(C::B_KVFULL + slot), sphase, abort_flag, kTimeoutNs)) return -1;
-        tc_fence_after();
-        const int s = (int)slot;
-        if (++slot == (uint32_t)C::NS) {
-          slot = 0;
-          sphase ^= 1u;
-        }
-        return s;
+      auto replay = [&](const Pair& pr) -> uint32_t {   // load_both: this tile's load index
+        const uint32_t ia = seq++;
+        const uint32_t ib = pr.share ? ia : seq++;
+        return x == 0 ? ia : ib;
       };
-      auto release = [&](int s) { mma_commit(bar(C::B_KVEMPTY + s)); };
-      // S_x = Q_x K^T once the group has read the previous S_x out of TMEM;
-      // the last S of an item frees its Q stage.
-      auto issue_s = [&](int x, uint32_t qs, int ks, bool frees_q) -> bool {
-        if (s_cnt[x] > 0 &&
-            !mbar_wait(bar(C::B_SFREE + x), (s_cnt[x] - 1) & 1u, abort_flag, kTimeoutNs))
+      auto mine = [&](const Pair& pr) { return x == 0 || pr.has_b; };
+      auto releases = [&](const Pair& pr) -> int { return pr.has_b && pr.share ? 1 : 2; };
+      auto wait_load = [&](uint32_t idx) -> bool {
+        if (!mbar_wait(bar(C::B_KVFULL + (int)(idx % C::NS)), (idx / C::NS) & 1u, abort_flag,
+                       kTimeoutNs))
           return false;
-        ++s_cnt[x];
         tc_fence_after();
+        return true;
+      };
+      auto release = [&](uint32_t idx, int n) {
+        for (int r = 0; r < n; ++r) mma_commit(bar(C::B_KVEMPTY + (int)(idx % C::NS)));
+      };
+      // S_x = Q_x K^T once the group has read the previous S_x out of TMEM;
+      // the last S of an item releases its Q stage.
+      auto issue_s = [&](const Pair& pr, uint32_t qs, uint32_t kidx, bool last) -> bool {
+        if (!wait_load(kidx)) return false;
+        if (s_cnt > 0 &&
+            !mbar_wait(bar(C::B_SFREE + x), (s_cnt - 1) & 1u, abort_flag, kTimeoutNs))
+          return false;
+        ++s_cnt;
+        tc_fence_after();
+        const int ks = (int)(kidx % C::NS);
         const uint64_t a0 = smem_desc(sQ + qs * 2 * C::TILEB + x * C::TILEB, 16, C::ATOM, C::SW);
         const uint64_t b0 = smem_desc(sKV + ks * C::TILEB, 16, C::ATOM, C::SW);
         const uint32_t dcol = tmem + C::COL_S + 128 * x;
@@ -921,31 +934,24 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
           mma_ss(dcol, desc_advance(a0, off), desc_advance(b0, off), IDESC_S, k > 0 ? 1u : 0u);
         }
         mma_commit(bar(C::B_SFULL + x));
-        if (frees_q) mma_commit(bar(C::B_QEMPTY + qs));
-        return true;
-      };
-      auto issue_s_pair = [&](const Pair& pr, uint32_t qs, int j) -> bool {
-        const bool sep = !pr.share;
-        const bool last = j == pair_nkv(pr) - 1;
-        const int ka = take();
-        if (ka < 0 || !issue_s(0, qs, ka, last && !pr.has_b)) return false;
-        if (!pr.has_b || sep) release(ka);
-        if (pr.has_b) {
-          const int kb = sep ? take() : ka;
-          if (kb < 0 || !issue_s(1, qs, kb, last)) return false;
-          release(kb);
+        if (last) {
+          mma_commit(bar(C::B_QEMPTY + qs));
+          if (!pr.has_b) mma_commit(bar(C::B_QEMPTY + qs));
         }
+        release(kidx, releases(pr));
         return true;
       };
       // O_x += P_x V once the group has written P_x; PFREE_x reports that P_x
       // has been read, OFULL_x (last key block) that O_x is complete.
-      auto issue_pv = [&](int x, int vs, int j, int nkv) -> bool {
-        if (!mbar_wait(bar(C::B_PFULL + x), pv_cnt[x] & 1u, abort_flag, kTimeoutNs)) return false;
-        ++pv_cnt[x];
+      auto issue_pv = [&](const Pair& pr, uint32_t vidx, int j, int nkv) -> bool {
+        if (!wait_load(vidx)) return false;
+        if (!mbar_wait(bar(C::B_PFULL + x), pv_cnt & 1u, abort_flag, kTimeoutNs)) return false;
+        ++pv_cnt;
         if (j == 0 &&
-            !mbar_wait(bar(C::B_OEMPTY + x), (o_cnt[x] & 1u) ^ 1u, abort_flag, kTimeoutNs))
+            !mbar_wait(bar(C::B_OEMPTY + x), (o_cnt & 1u) ^ 1u, abort_flag, kTimeoutNs))
           return false;
         tc_fence_after();
+        const int vs = (int)(vidx % C::NS);
         const uint64_t v0 = smem_desc(sKV + vs * C::TILEB, C::CHUNKB, C::ATOM, C::SW);
         const uint32_t ocol = tmem + C::COL_O + DH * x;
         const uint32_t pcol = tmem + C::COL_P + 64 * x;
@@ -956,43 +962,42 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
         mma_commit(bar(C::B_PFREE + x));
         if (j == nkv - 1) {
           mma_commit(bar(C::B_OFULL + x));
-          ++o_cnt[x];
+          ++o_cnt;
         }
-        return true;
-      };
-      auto issue_pv_pair = [&](const Pair& pr, int j) -> bool {
-        const bool sep = !pr.share;
-        const int nkv = pair_nkv(pr);
-        const int va = take();
-        if (va < 0 || !issue_pv(0, va, j, nkv)) return false;
-        if (!pr.has_b || sep) release(va);
-        if (pr.has_b) {
-          const int vb = sep ? take() : va;
-          if (vb < 0 || !issue_pv(1, vb, j, nkv)) return false;
-          release(vb);
-        }
+        release(vidx, releases(pr));
         return true;
       };
       int p = blockIdx.x;
-      if (p < npairs) {
-        const Pair pr = get_pair(p);
-        ok = mbar_wait(bar(C::B_QFULL + 0), 0u, abort_flag, kTimeoutNs) && issue_s_pair(pr, 0, 0);
-      }
+      uint32_t k0 = 0;                   // this tile's K(0) load of item p
+      bool s0_done = false;              // S_x(0) of item p already issued
+      if (p < npairs) k0 = replay(get_pair(p));
       for (uint32_t ic = 0; ok && p < npairs; p += stride, ++ic) {
         const Pair pr = get_pair(p);
         const int nkv = pair_nkv(pr);
-        const uint32_t qs = ic % C::QST;
+        const uint32_t qs = ic % C::QST, qph = (ic / C::QST) & 1u;
         const bool has_next = p + stride < npairs;
+        const bool me = mine(pr);
+        if (me && !s0_done)
+          ok = mbar_wait(bar(C::B_QFULL + qs), qph, abort_flag, kTimeoutNs) &&
+               issue_s(pr, qs, k0, nkv == 1);
+        s0_done = false;
         for (int j = 0; ok && j < nkv; ++j) {
           if (j + 1 < nkv) {
-            ok = issue_s_pair(pr, qs, j + 1);
+            const uint32_t kn = replay(pr);
+            if (me) ok = issue_s(pr, qs, kn, j + 2 == nkv);
           } else if (has_next) {
+            // the next item's first S, ahead of this item's last PV
             const Pair pn = get_pair(p + stride);
-            const uint32_t qn = (ic + 1) % C::QST, qph = ((ic + 1) / C::QST) & 1u;
-            ok = mbar_wait(bar(C::B_QFULL + qn), qph, abort_flag, kTimeoutNs) &&
-                 issue_s_pair(pn, qn, 0);
+            k0 = replay(pn);
+            if (mine(pn)) {
+              const uint32_t qn = (ic + 1) % C::QST, qnph = ((ic + 1) / C::QST) & 1u;
+              ok = mbar_wait(bar(C::B_QFULL + qn), qnph, abort_flag, kTimeoutNs) &&
+                   issue_s(pn, qn, k0, pair_nkv(pn) == 1);
+              s0_done = true;
+            }
           }
-          if (ok) ok = issue_pv_pair(pr, j);
+          const uint32_t vi = replay(pr);
+          if (ok && me) ok = issue_pv(pr, vi, j, nkv);
         }
       }
     }
@@ -1251,8 +1256,8 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
   if (*abort_flag) {
     report(a.ws, GDPA_ERR_TIMEOUT);
     volatile int never = 0;
-    if (warp == 1 && lane == 0) {
-      mma_commit(bar(C::B_DRAIN));                       // all MMAs issued so far
+    if ((warp == 1 || warp == 3) && lane == 0) {         // both issuers' MMAs
+      mma_commit(bar(C::B_DRAIN));
       mbar_wait(bar(C::B_DRAIN), 0, &never, kTimeoutNs);
     }
     if (warp == 0 && lane == 0) {                         // let in-flight TMA loads land
