@@ -449,8 +449,10 @@ def run_variant(args, rank, world, local_rank):
 
     wl = syn.WORKLOADS[args.workload]
     lens = syn.lengths(wl, seed=rank)
+    if 0 < args.samples < len(lens):
+        lens = lens[:args.samples]          # the small profiling case
     offs = syn.offsets_from_lengths(lens)
-    B, T, h, dh = wl.B, int(offs[-1]), wl.h, wl.dh
+    B, T, h, dh = len(lens), int(offs[-1]), wl.h, wl.dh
     S, W = int(args.pool), int(args.window)
     scale = 1.0 / dh ** 0.5
     gen = torch.Generator(device=dev)
@@ -630,7 +632,9 @@ def run_variant(args, rank, world, local_rank):
               "warmup": args.warmup, "ms_per_step": agg["ms_max"] / args.steps,
               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
               "data": "synthetic",
-              "config": {"workload": f"{what}_tokens_of_{wl.name}", "B": B, "h": h, "dh": dh,
+              "config": {"workload": f"{what}_tokens_of_{wl.name}" +
+                                     (f" (first {B} samples only: profiling case)"
+                                      if B < wl.B else ""), "B": B, "h": h, "dh": dh,
                          "seeds": S or None, "window": W or None, "lengths": wl.lengths,
                          "tokens_per_rank": T, "scale": scale,
                          "inputs": "N(0,1) bf16 from a seeded torch generator per tensor",

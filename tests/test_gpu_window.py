@@ -96,3 +96,24 @@ def test_window_backward_guard():
     T_ = slice(128, 128 + T)
     assert _rel(bufs[0][T_], rq, rv) <= TOL and _rel(bufs[1][T_], rk, rv) <= TOL
     assert _rel(bufs[2][T_], rv, rv) <= TOL
+
+
+def test_window_power_law_batch():
+    """The first 128 samples of the power-law workload's lengths (32..4096),
+    h = 16, dh = 64, w = 256: forward and backward against the oracle."""
+    import synthetic as syn
+    n = syn.lengths(syn.WORKLOADS[5])[:128]
+    h, dh, w = 16, 64, 256
+    q, k, v, off = _case(21, n, h, dh)
+    T = int(off[-1])
+    g = torch.randn(T, h, dh, generator=torch.Generator().manual_seed(4)).bfloat16()
+    offd = torch.tensor(off, dtype=torch.int32, device=DEV)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    o, lse = pkg.gdpa.window_fwd(qd, offd, kd, vd, w, 0.125, off)
+    dq, dk, dv = pkg.gdpa.window_bwd(qd, offd, kd, vd, o, lse, g.to(DEV), w, 0.125, off)
+    torch.cuda.synchronize()
+    ro, rl = oracle.win_fwd(q, k, v, off, w, 0.125)
+    assert _rel(o, ro, ro) <= TOL
+    assert np.abs(lse.cpu().numpy() - rl).max() <= 1e-2
+    rq, rk, rv = oracle.win_bwd(q, k, v, g, off, w, 0.125)
+    assert _rel(dq, rq, rv) <= TOL and _rel(dk, rk, rv) <= TOL and _rel(dv, rv, rv) <= TOL
