@@ -501,6 +501,7 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             float pv[2], dv2[2];
+            float2 gp, gd;                                // GELU: phi and phi' of the pair
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int r = 32 * ch + c + e;
@@ -522,9 +523,12 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 p = relu_f(u);
                 ds = g * relu_grad(u);
               } else if constexpr (PHI == GDPA_PHI_GELU) {
-                const float u = fmaf(x, sc, b1k);
-                p = gelu_f(u);
-                ds = g * gelu_grad(u);
+                if (e == 0)           // both columns of the pair, in packed arithmetic
+                  gelu_fg2(__ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                      make_float2(sc, sc), make_float2(b1k, b1k)),
+                           gp, gd);
+                p = e ? gp.y : gp.x;
+                ds = g * (e ? gd.y : gd.x);
               } else {
                 p = fmaf(x, sc, b1k);
                 ds = g;
@@ -1087,6 +1091,7 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             float pv[2], dv2[2];
+            float2 gp, gd;                                // GELU: phi and phi' of the pair
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int r = 32 * ch + c + e;
@@ -1108,9 +1113,12 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                 p = relu_f(u);
                 ds = g * relu_grad(u);
               } else if constexpr (PHI == GDPA_PHI_GELU) {
-                const float u = fmaf(x, sc, b1k);
-                p = gelu_f(u);
-                ds = g * gelu_grad(u);
+                if (e == 0)           // both columns of the pair, in packed arithmetic
+                  gelu_fg2(__ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                      make_float2(sc, sc), make_float2(b1k, b1k)),
+                           gp, gd);
+                p = e ? gp.y : gp.x;
+                ds = g * (e ? gd.y : gd.x);
               } else {
                 p = fmaf(x, sc, b1k);
                 ds = g;

@@ -1186,8 +1186,9 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
                 p0 = relu_f(x.x * sm);
                 p1 = relu_f(x.y * sm);
               } else if constexpr (PHI == GDPA_PHI_GELU) {
-                p0 = gelu_f(x.x * sm);
-                p1 = gelu_f(x.y * sm);
+                const float2 y = gelu_f2(BIAS ? x : __fmul2_rn(x, make_float2(sm, sm)));
+                p0 = y.x;
+                p1 = y.y;
               } else {
                 const float2 y = __fmul2_rn(x, make_float2(sm, sm));
                 p0 = y.x;
