@@ -80,6 +80,9 @@ def parse(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-chunks", type=int, default=E2E_CHUNKS,
+                    help="sample groups of the end-to-end step (copy-in, compute and copy-out "
+                         "of successive groups overlap)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-passes", type=int, default=3,
@@ -853,7 +856,7 @@ def main(argv=None):
         token_major_out = [True, True, False, False]
         offs = [int(x) for x in d["offsets"]]
         chunks = []
-        for (b0, b1), (t0_, t1_) in e2e_chunks(offs, E2E_CHUNKS):
+        for (b0, b1), (t0_, t1_) in e2e_chunks(offs, max(1, args.e2e_chunks)):
             coff = [x - t0_ for x in offs[b0:b1 + 1]]
             cp_ = pkg.problem_for(q[t0_:t1_], k[b0:b1], coff, wl.phi_name, wl.scale,
                                   max_n=max(coff[i + 1] - coff[i] for i in range(b1 - b0)))

@@ -1141,7 +1141,11 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
               m_run = m_blk;
               resc = true;
             }
-            const float2 negm = make_float2(-m_run, -m_run);
+            // masked logits hold -inf (+inf for a negative scale), so their exp2 is
+            // exactly 0; a row with no visible key yet keeps m_run = -inf and takes
+            // offset 0 (its exponents are all -inf as well)
+            const float mo = m_run == -INFINITY ? 0.f : -m_run;
+            const float2 negm = make_float2(mo, mo);
             float2 acc[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) acc[u] = make_float2(0.f, 0.f);
@@ -1156,10 +1160,6 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
               } else {
                 e.x = ex2_approx(x.x);
                 e.y = ex2_approx(x.y);
-              }
-              if (partial) {
-                e.x = 2 * i >= clo && 2 * i <= chi ? e.x : 0.f;
-                e.y = 2 * i + 1 >= clo && 2 * i + 1 <= chi ? e.y : 0.f;
               }
               acc[i & 3] = __fadd2_rn(acc[i & 3], e);
               pk[i] = pack_bf16x2(e.x, e.y);

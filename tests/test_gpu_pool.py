@@ -135,3 +135,19 @@ def test_pool_backward_power_law_batch_and_guard():
     rs, rk, rv = oracle.pool_bwd(seeds, k, v, g, off, 0.125)
     assert _rel(dseeds, rs, rv) <= TOL
     assert _rel(dk, rk, rv) <= TOL and _rel(dv, rv, rv) <= TOL
+
+
+def test_pool_backward_of_an_empty_batch():
+    """No tokens at all: every seed pools nothing, dseeds is zero and no
+    kernel touches dK/dV."""
+    h, S, dh = 2, 16, 64
+    seeds = torch.randn(h, S, dh).bfloat16().to(DEV)
+    off = np.zeros(4, dtype=np.int64)
+    offd = torch.tensor(off, dtype=torch.int32, device=DEV)
+    k = torch.empty(0, h, dh, dtype=torch.bfloat16, device=DEV)
+    o, lse = pkg.gdpa.pool_fwd(seeds, offd, k, k, 0.125, off)
+    g = torch.randn(3, h, S, dh).bfloat16().to(DEV)
+    dseeds, dk, dv = pkg.gdpa.pool_bwd(seeds, offd, k, k, o, lse, g, 0.125, off)
+    torch.cuda.synchronize()
+    assert float(o.float().abs().max()) == 0.0 and bool(torch.isneginf(lse).all())
+    assert float(dseeds.abs().max()) == 0.0 and dk.numel() == 0

@@ -117,3 +117,13 @@ def test_window_power_law_batch():
     assert np.abs(lse.cpu().numpy() - rl).max() <= 1e-2
     rq, rk, rv = oracle.win_bwd(q, k, v, g, off, w, 0.125)
     assert _rel(dq, rq, rv) <= TOL and _rel(dk, rk, rv) <= TOL and _rel(dv, rv, rv) <= TOL
+
+
+def test_window_backward_of_an_empty_batch():
+    off = np.zeros(3, dtype=np.int64)
+    offd = torch.tensor(off, dtype=torch.int32, device=DEV)
+    z = torch.empty(0, 2, 64, dtype=torch.bfloat16, device=DEV)
+    o, lse = pkg.gdpa.window_fwd(z, offd, z, z, 8, 0.125, off)
+    dq, dk, dv = pkg.gdpa.window_bwd(z, offd, z, z, o, lse, z, 8, 0.125, off)
+    torch.cuda.synchronize()
+    assert dq.numel() == dk.numel() == dv.numel() == 0
