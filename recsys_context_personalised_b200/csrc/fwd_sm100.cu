@@ -718,7 +718,9 @@ __device__ __forceinline__ float row_extreme(const uint32_t (&s)[128]) {
   return NEG ? fmin3(fminf(e[0], e[1]), e[2], e[3]) : fmax3(fmaxf(e[0], e[1]), e[2], e[3]);
 }
 
-template <int DH, int PHI, bool BIAS, int MODE>
+// KEYMASK = false: every key block is full (GDPA with m a multiple of 128),
+// so the softmax needs no key mask and the kernel carries none.
+template <int DH, int PHI, bool BIAS, int MODE, bool KEYMASK = true>
 __global__ void __launch_bounds__(kThreads, 1)
 gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
@@ -1125,8 +1127,9 @@ gdpa_fwd_early_kernel(const __grid_constant__ CUtensorMap tmQ,
               clo = max(0, qpos - a.window + 1 - kb0);
               chi = min(C::BN - 1, qpos - kb0);
             }
-            const bool partial = WIN ? __any_sync(0xffffffffu, clo > 0 || chi < C::BN - 1)
-                                     : valid < C::BN;
+            const bool partial =
+                KEYMASK && (WIN ? __any_sync(0xffffffffu, clo > 0 || chi < C::BN - 1)
+                                : valid < C::BN);
             if (partial) {
               const uint32_t fill = __float_as_uint(neg ? INFINITY : -INFINITY);
 #pragma unroll
@@ -1306,10 +1309,10 @@ bool make_maps(const gdpa_problem_t& p, const void* q, const void* k, const void
 }
 
 // dh <= 64 (P in TMEM columns of its own): S released early; dh = 128: P aliases S.
-template <int DH, int PHI, bool BIAS>
+template <int DH, int PHI, bool BIAS, bool KEYMASK>
 constexpr auto fwd_kernel() {
   if constexpr (DH <= 64)
-    return gdpa_fwd_early_kernel<DH, PHI, BIAS, kModeGdpa>;
+    return gdpa_fwd_early_kernel<DH, PHI, BIAS, kModeGdpa, KEYMASK>;
   else
     return gdpa_fwd_sm100_kernel<DH, PHI, BIAS>;
 }
@@ -1321,7 +1324,10 @@ cudaError_t launch_fwd_t(const gdpa_problem_t& p, const void* q, const void* k, 
   using C = FwdCfg<DH>;
   CUtensorMap mq, mk, mv;
   if (!make_maps<DH>(p, q, k, v, &mq, &mk, &mv)) return cudaErrorInvalidValue;
-  auto kern = fwd_kernel<DH, PHI, BIAS>();
+  // softmax over a last key block with fewer than 128 keys needs the key mask
+  // (the other activations give 0 on the zero-filled keys past m)
+  auto kern = PHI == GDPA_PHI_SOFTMAX && p.m % 128 != 0 ? fwd_kernel<DH, PHI, BIAS, true>()
+                                                         : fwd_kernel<DH, PHI, BIAS, false>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
   FwdArgs args = {};
