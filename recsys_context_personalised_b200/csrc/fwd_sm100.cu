@@ -677,14 +677,16 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 // (three-input max), keeps the running offset while the block maximum stays
 // within 2^8 of it and otherwise moves it and rescales O (rare).  A fixed
 // share of the exp2 evaluations (kPolyPairs of every 8 pairs of columns) runs
-// on the FMA pipe (exp2_fma2) instead of the MUFU unit, which alone would cap
-// the dh = 64 forward: one transcendental per logit against 4 * dh = 256
-// tensor FLOPs per logit.
+// on the FMA pipe (exp2_fma2) instead of the MUFU unit, which the exp2 and the
+// bf16 packs keep the busiest pipe of the dh = 64 forward: one transcendental
+// per logit against 4 * dh = 256 tensor FLOPs per logit.  Two of eight
+// measured 2.5% faster than none on the power-law softmax forward; three of
+// eight slower (the FMA and ALU work of the polynomial).
 //
 // Registers: the launch gives 168 per thread (384 x 168 = 64,512); warps 0-3
 // drop to 80 and the two activation warpgroups rise to 208 (a thread holds a
 // whole 128-column S row): 128 x 80 + 256 x 208 = 63,488 <= 64,512.
-constexpr int kPolyPairs = 0;
+constexpr int kPolyPairs = 2;
 
 // Modes of the dh <= 64 forward kernel: the GDPA operator, seed-query pooling
 // (first level of HSP) and sliding-window self-attention on the jagged tokens.
