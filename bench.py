@@ -59,10 +59,10 @@ KERNEL_SOURCES = {"gdpa_fwd_sm100": ("fwd_sm100.cu", "sm100.cuh", "gdpa_internal
 # sha16 of the kernel's sources at capture time)}}.  An entry whose hash no
 # longer matches the sources is not used (the traffic is then reported null).
 TRAFFIC_PER_UNIT = {
-    # 64-sample case of workload 5: 582.3 MB read + 35.9 MB written in one launch
-    "gdpa_fwd_sm100": {5: (0.0141410, "2363958718f94a13")},
-    # same case: 743.4 MB read + 588.6 MB written in one launch
-    "gdpa_bwd_sm100": {5: (0.0304685, "a56564a9f4c5f1a4")},
+    # 64-sample case of workload 5: 582.5 MB read + 36.9 MB written in one launch
+    "gdpa_fwd_sm100": {5: (0.0141676, "0ca16e7cbae83405")},
+    # same case: 741.4 MB read + 588.3 MB written in one launch
+    "gdpa_bwd_sm100": {5: (0.0304155, "7212f118d73e1f69")},
 }
 # fp32 FFMA peak for the SIMT kernels: 148 SMs * 128 FMA/clk * 2 flop * 1.965 GHz
 SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
