@@ -202,7 +202,9 @@ __device__ __forceinline__ void store_o_rows(uint32_t my_o, uint32_t ostg, float
   }
 }
 
-template <int DH, int PHI, bool BIAS>
+// KEYMASK = false: every key block is full (m a multiple of 128), so the
+// softmax carries no key mask.
+template <int DH, int PHI, bool BIAS, bool KEYMASK = true>
 __global__ void __launch_bounds__(kThreads, 1)
 gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
@@ -510,7 +512,7 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
               for (int i = 0; i < 64; ++i) {
                 const float x = __uint_as_float(sh[i]);
-                if (valid == C::BN || 64 * hf + i < valid)
+                if (!KEYMASK || valid == C::BN || 64 * hf + i < valid)
                   m8[i & 7] = c2e >= 0.f ? fmaxf(m8[i & 7], x) : fminf(m8[i & 7], x);
               }
             }
@@ -534,7 +536,7 @@ gdpa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 const int col = 64 * hf + 2 * i;
                 float p0 = ex2_approx(fmaf(__uint_as_float(sh[2 * i]), c2e, neg_m));
                 float p1 = ex2_approx(fmaf(__uint_as_float(sh[2 * i + 1]), c2e, neg_m));
-                if (valid < C::BN) {
+                if (KEYMASK && valid < C::BN) {
                   p0 = col < valid ? p0 : 0.f;
                   p1 = col + 1 < valid ? p1 : 0.f;
                 }
@@ -1316,7 +1318,7 @@ constexpr auto fwd_kernel() {
   if constexpr (DH <= 64)
     return gdpa_fwd_early_kernel<DH, PHI, BIAS, kModeGdpa, KEYMASK>;
   else
-    return gdpa_fwd_sm100_kernel<DH, PHI, BIAS>;
+    return gdpa_fwd_sm100_kernel<DH, PHI, BIAS, KEYMASK>;
 }
 
 template <int DH, int PHI, bool BIAS>
