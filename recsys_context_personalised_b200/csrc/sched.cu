@@ -78,11 +78,42 @@ schedule_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T, in
   }
 }
 
+constexpr int kSortMax = 4096;   // 32 KB of static shared memory
+
+// Sorts the samples by length, longest first (ties: lower index first), into
+// s_key[0, B) as (n_b, b); entries [B, P2) pad with (-1, INT_MAX).  B <= kSortMax.
+// A bitonic sorting network over the next power of two P2, all threads taking
+// part (Batcher, "Sorting networks and their applications", AFIPS 1968).
+__device__ void sort_by_length(const int32_t* __restrict__ offsets, int B, int2* s_key) {
+  const int tid = threadIdx.x;
+  int P2 = 1;
+  while (P2 < B) P2 <<= 1;
+  for (int i = tid; i < P2; i += kSchedThreads)
+    s_key[i] = i < B ? make_int2(offsets[i + 1] - offsets[i], i) : make_int2(-1, 0x7fffffff);
+  __syncthreads();
+  for (int k = 2; k <= P2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < P2; i += kSchedThreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const int2 x = s_key[i], y = s_key[ixj];
+          const bool x_first = x.x > y.x || (x.x == y.x && x.y < y.y);
+          const bool up = (i & k) == 0;
+          if (up ? !x_first : x_first) {
+            s_key[i] = y;
+            s_key[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
 // Backward work list: one item per (sample, head, 128-key block), samples in
 // decreasing length order (longest-processing-time first), so that a static
 // round-robin over CTAs gives every SM about the same number of query tiles.
 // Item fields: b, head, row0 = first key of the block, rows = n_b.
-constexpr int kSortMax = 4096;   // 32 KB of static shared memory
 
 __global__ void __launch_bounds__(kSchedThreads)
 schedule_kv_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T, int max_n,
@@ -109,31 +140,7 @@ schedule_kv_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T,
     return;
   }
   const bool sorted = B <= kSortMax;
-  int P2 = 1;
-  while (P2 < B) P2 <<= 1;
-  if (sorted) {
-    for (int i = tid; i < P2; i += kSchedThreads)
-      s_key[i] = i < B ? make_int2(offsets[i + 1] - offsets[i], i) : make_int2(-1, 0x7fffffff);
-    __syncthreads();
-    // bitonic sort: descending n, ascending b
-    for (int k = 2; k <= P2; k <<= 1) {
-      for (int j = k >> 1; j > 0; j >>= 1) {
-        for (int i = tid; i < P2; i += kSchedThreads) {
-          const int ixj = i ^ j;
-          if (ixj > i) {
-            const int2 x = s_key[i], y = s_key[ixj];
-            const bool x_first = x.x > y.x || (x.x == y.x && x.y < y.y);
-            const bool up = (i & k) == 0;
-            if (up ? !x_first : x_first) {
-              s_key[i] = y;
-              s_key[ixj] = x;
-            }
-          }
-        }
-        __syncthreads();
-      }
-    }
-  }
+  if (sorted) sort_by_length(offsets, B, s_key);
   const long long per_sample = (long long)h * nkv;
   for (long long idx = tid; idx < (long long)B * per_sample; idx += kSchedThreads) {
     const int r = (int)(idx / per_sample);
@@ -181,29 +188,7 @@ schedule_pool_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t 
     }
     return;
   }
-  int P2 = 1;
-  while (P2 < B) P2 <<= 1;
-  for (int i = tid; i < P2; i += kSchedThreads)
-    s_key[i] = i < B ? make_int2(offsets[i + 1] - offsets[i], i) : make_int2(-1, 0x7fffffff);
-  __syncthreads();
-  // bitonic sort: descending n, ascending b (samples without tokens sort last)
-  for (int k = 2; k <= P2; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < P2; i += kSchedThreads) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const int2 x = s_key[i], y = s_key[ixj];
-          const bool x_first = x.x > y.x || (x.x == y.x && x.y < y.y);
-          const bool up = (i & k) == 0;
-          if (up ? !x_first : x_first) {
-            s_key[i] = y;
-            s_key[ixj] = x;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
+  sort_by_length(offsets, B, s_key);         // samples without tokens sort last
   const int hp = (h + 1) / 2;
   const long long items = (long long)s_nz * hp;
   for (long long idx = tid; idx < items; idx += kSchedThreads) {
@@ -250,29 +235,7 @@ schedule_jkv_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T
     }
     return;
   }
-  int P2 = 1;
-  while (P2 < B) P2 <<= 1;
-  for (int i = tid; i < P2; i += kSchedThreads)
-    s_key[i] = i < B ? make_int2(offsets[i + 1] - offsets[i], i) : make_int2(-1, 0x7fffffff);
-  __syncthreads();
-  // bitonic sort: descending n, ascending b
-  for (int k = 2; k <= P2; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < P2; i += kSchedThreads) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const int2 x = s_key[i], y = s_key[ixj];
-          const bool x_first = x.x > y.x || (x.x == y.x && x.y < y.y);
-          const bool up = (i & k) == 0;
-          if (up ? !x_first : x_first) {
-            s_key[i] = y;
-            s_key[ixj] = x;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
+  sort_by_length(offsets, B, s_key);
   // exclusive scan of the key-block counts in sorted order, then the items
   for (int base = 0; base < B; base += kSchedThreads) {
     const int r = base + tid;
