@@ -912,14 +912,16 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
         const uint32_t qaddr = sStg + st * 2 * C::TILEB + 64 * h * C::ROWB;
         const uint64_t gmn = smem_desc(qaddr + C::TILEB, C::TILEB, C::ATOM, C::SW);   // dO, MN-major
         const uint64_t qmn = smem_desc(qaddr, C::TILEB, C::ATOM, C::SW);              // Q, MN-major
-        const uint64_t dsk = smem_desc(sDS + c * C::DSB + h * 16384, 16, 1024, kSw128);  // dS^T, K-major
+        // both A operands from TMEM (P^T_h over S^T_h's first columns, dS^T_h over
+        // dP^T_h's): only the 2 KB B tiles come from shared memory, whose
+        // bandwidth N = 64 products are short of
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           mma_ts(tmem + C::COL_DV, tmem + 128 * h + 8 * k, desc_advance(gmn, k * 2 * C::ATOM),
                  IDESC_KV, (first && k == 0) ? 0u : 1u);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          mma_ss(tmem + C::COL_DK, desc_advance(dsk, k * 32), desc_advance(qmn, k * 2 * C::ATOM),
+          mma_ts(tmem + C::COL_DK, tmem + 128 * h + 64 + 8 * k, desc_advance(qmn, k * 2 * C::ATOM),
                  IDESC_KV, (first && k == 0) ? 0u : 1u);
       };
       // One pass over every (item, query tile) of this CTA.
@@ -1139,6 +1141,8 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
             dd[c / 2] = pack_bf16x2(dv2[0], dv2[1]);
           }
           tmem_st_x16(tmem + lane_off + 128 * grp + 16 * ch, pp);
+          // dS^T_h as bf16 over dP^T_h's first 32 columns (read above) for the dK product
+          tmem_st_x16(tmem + lane_off + 128 * grp + 64 + 16 * ch, dd);
           // dS^T line `lrow` of this half's chunk, 16-byte pieces 4ch..4ch+3, 128B swizzle
           const uint32_t line = dsb + lrow * 128;
 #pragma unroll
