@@ -676,11 +676,14 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 //     (bulk reduce-add) and dV/dK (bulk store), and warp 2 loads the softmax
 //     row statistics one tile ahead, so the two activation groups only form
 //     P^T and dS^T.
-// The drain group stages each tile's dQ, and an item's dV/dK, in the tile's
-// own dS^T buffer: its readers are all in the completed products.  Before the
-// MMA thread issues the S^T products of the tile that will overwrite a buffer
-// (two tiles later), it waits on STGFREE of that buffer, which the drain group
-// arrives on once its bulk copies have read the staging area.
+// Each drain warp reduces the dQ of its own 32 rows through a 4 KB staging box
+// of its own, one column half at a time, and skips rows that all lie past the
+// sample.  An item's dV/dK are staged in its last tile's dS^T buffer (whose
+// readers are all in the completed products).  Before the MMA thread issues
+// the S^T products of the tile that will overwrite a dS^T buffer (two tiles
+// later), it waits on STGFREE of that buffer: the drain group arrives on it as
+// soon as the tile's dQ products complete, or, at an item's last tile, once
+// the dV/dK stores have read the buffer.
 // Registers (512 threads at 128 each): warps 0-3 drop to 72, the drain group
 // to 104, the activation groups rise to 168 (4 x 128 x (72+104+168+168) = 65536).
 constexpr int kHalfThreads = 512;
@@ -695,7 +698,7 @@ struct BwdHalfCfg {
   static constexpr int NSTG = 2, NKV = 2;
   static constexpr uint32_t DSB = 2 * 128 * 128;           // one dS^T buffer, two 16 KB halves
   static constexpr uint32_t COL_DV = 256, COL_DK = 256 + DH, COL_DQ = 256 + 2 * DH;
-  // staging rows: DH/2 fp32 (dQ box) or DH bf16 (dV/dK box), both 2*DH bytes
+  // dV/dK staging rows: DH bf16
   static constexpr uint32_t SROWB = 2 * DH;
   static constexpr int B_KVFULL = 0, B_KVEMPTY = 2, B_SFULL = 4, B_PFULL = 6, B_DQFULL = 8,
                        B_DQEMPTY = 10, B_ACCFULL = 12, B_ACCEMPTY = 13, B_DRAIN = 14,
@@ -708,12 +711,16 @@ struct BwdHalfCfg {
   static constexpr uint32_t OFF_CTL = OFF_DS + 2 * DSB;
   // + a two-slot ring of row statistics: [slot][log2-scaled LSE, D][128 rows] fp32
   static constexpr uint32_t CTL_BYTES = 1024 + 2 * 2 * 128 * 4;
-  static constexpr uint32_t SMEM_USED = 1024 + OFF_CTL + CTL_BYTES;
+  // + one dQ staging box per drain warp: its 32 rows x DH/2 fp32 (a column half)
+  static constexpr uint32_t DQSB = 32 * 2 * DH;
+  static constexpr uint32_t OFF_DQS = (OFF_CTL + CTL_BYTES + 1023u) & ~1023u;
+  static constexpr uint32_t SMEM_USED = 1024 + OFF_DQS + 4 * DQSB;
   static constexpr uint32_t SMEM = SMEM_USED > 120u * 1024u ? SMEM_USED : 120u * 1024u;
   static_assert(SMEM <= 232448u, "exceeds the 227 KB of shared memory a CTA can have");
   static_assert(COL_DQ + 2 * DH <= 512, "TMEM columns");
   static_assert(128 * SROWB <= DSB / 2, "a staging box fits in a dS^T half");
-  static_assert(OFF_STG % 1024 == 0 && OFF_DS % 1024 == 0, "swizzle atoms need 1024-B alignment");
+  static_assert(OFF_STG % 1024 == 0 && OFF_DS % 1024 == 0 && OFF_DQS % 1024 == 0 &&
+                DQSB % 1024 == 0, "swizzle atoms need 1024-B alignment");
   static_assert(8 * NBAR + 8 <= 1024, "barriers, TMEM slot and abort flag share the first 1 KB");
 };
 
@@ -754,6 +761,7 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t sKV = base + C::OFF_KV, sStg = base + C::OFF_STG, sDS = base + C::OFF_DS;
+  const uint32_t sDQS = base + C::OFF_DQS;
   uint8_t* ctl = gbase + C::OFF_CTL;
   const uint32_t bar0 = smem_u32(ctl);
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
@@ -1182,22 +1190,8 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
       sync_phase ^= 1u;
       return __all_sync(0xffffffffu, w);
     };
-    // one row of 2*DH bytes from 16-column TMEM loads, packed as fp32 (dQ) or
-    // as bf16 times `mul` (dV, dK), into 16-byte chunks of a staging box
-    auto stage_f32 = [&](uint32_t src, uint32_t box) {
-#pragma unroll
-      for (int c = 0; c < DH / 2; c += 16) {
-        uint32_t v[16];
-        tmem_ld_x16(src + c, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                       ::"r"(stage_chunk<DH>(box, lrow, c / 4 + j)), "r"(v[4 * j]),
-                       "r"(v[4 * j + 1]), "r"(v[4 * j + 2]), "r"(v[4 * j + 3])
-                       : "memory");
-      }
-    };
+    // one key row of DH columns from 16-column TMEM loads, as bf16 times `mul`
+    // (dV, dK), into 16-byte chunks of a staging box
     auto stage_bf16 = [&](uint32_t src, uint32_t box, float mul) {
 #pragma unroll
       for (int c = 0; c < DH; c += 16) {
@@ -1259,9 +1253,7 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
       const int t0 = a.offsets[it.b];
       for (int i = 0; i < nq; ++i, ++qs) {
         const uint32_t b = qs & 1u;
-        // dQ of tile qs.  Its dS^T buffer b is free: the tile's products are
-        // complete, and the bulk copies that last read it (tile qs-2) finished
-        // before STGFREE let the MMA thread start this tile.
+        // dQ of tile qs: the tile's products are complete
         bool w = mbar_wait(bar(C::B_DQFULL + (int)b), (qs >> 1) & 1u, abort_flag, kTimeoutNs);
         if (!__all_sync(0xffffffffu, w)) {
           ok = false;
@@ -1269,31 +1261,54 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         tc_fence_after();
         const uint32_t stg = sDS + b * C::DSB;
-        const uint32_t src = tmem + lane_off + C::COL_DQ + b * DH;
-        stage_f32(src, stg);                           // columns [0, DH/2)
-        stage_f32(src + DH / 2, stg + 16384);          // columns [DH/2, DH)
-        tc_fence_before();
-        mbar_arrive(bar(C::B_DQEMPTY + (int)b));
-        fence_proxy_async_smem();
-        if (!group_sync()) {
-          ok = false;
-          break;
-        }
-        if (lrow == 0) {
-          // rows past the sample are exact zeros (their dS entries are zero);
-          // rows past T are clipped by the map
-          if constexpr (POOL) {       // dseeds [h, S, DH]: rows >= S are clipped by the map
-            tma_reduce_add_3d(&tmDQ, stg, 0, 0, it.head);
-            tma_reduce_add_3d(&tmDQ, stg + 16384, DH / 2, 0, it.head);
-          } else {
-            tma_reduce_add_3d(&tmDQ, stg, 0, it.head, t0 + 128 * (fi + i));
-            tma_reduce_add_3d(&tmDQ, stg + 16384, DH / 2, it.head, t0 + 128 * (fi + i));
+        // within an item the tile's dS^T buffer has no readers left
+        if (i + 1 < nq && lrow == 0) mbar_arrive(bar(C::B_STGFREE + (int)b));
+        {
+          // Each warp reduces its own 32 rows into the fp32 accumulator, one
+          // column half at a time through its staging box.  Rows past the
+          // sample (pooling: past the seeds) are exact zeros, since their dS
+          // entries are zero: a warp whose rows all lie there adds nothing, and
+          // rows past T are clipped by the map.
+          const int rows_here = POOL ? a.S : n - 128 * (fi + i);
+          const bool adds = quad * 32 < rows_here;
+          const uint32_t box = sDQS + quad * C::DQSB;
+          const uint32_t src = tmem + lane_off + C::COL_DQ + b * DH;
+#pragma unroll
+          for (int hc = 0; hc < 2; ++hc) {
+            uint32_t v[DH / 2];
+#pragma unroll
+            for (int c = 0; c < DH / 2; c += 16)
+              tmem_ld_x16(src + hc * (DH / 2) + c, *reinterpret_cast<uint32_t(*)[16]>(&v[c]));
+            tmem_wait_ld();
+            if (hc == 1) {
+              tc_fence_before();
+              mbar_arrive(bar(C::B_DQEMPTY + (int)b));
+            }
+            if (adds) {
+              if (lane == 0) bulk_wait_group_read0();   // the box's previous reduce has read it
+              __syncwarp();
+#pragma unroll
+              for (int j = 0; j < DH / 8; ++j)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                             ::"r"(stage_chunk<DH>(box, lane, j)), "r"(v[4 * j]),
+                             "r"(v[4 * j + 1]), "r"(v[4 * j + 2]), "r"(v[4 * j + 3])
+                             : "memory");
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                if constexpr (POOL)   // dseeds [h, S, DH]
+                  tma_reduce_add_3d(&tmDQ, box, hc * (DH / 2), 32 * quad, it.head);
+                else
+                  tma_reduce_add_3d(&tmDQ, box, hc * (DH / 2), it.head,
+                                    t0 + 128 * (fi + i) + 32 * quad);
+                bulk_commit_group();
+              }
+            }
           }
-          bulk_commit_group();
         }
         if (i + 1 == nq) {
-          // dV and s*dK of this key block, through the same buffer once the
-          // reduces have read it
+          // dV and s*dK of this key block, staged in the tile's dS^T buffer
+          // (all of its readers are in the completed products)
           w = mbar_wait(bar(C::B_ACCFULL), ic & 1u, abort_flag, kTimeoutNs);
           if (!__all_sync(0xffffffffu, w)) {
             ok = false;
@@ -1338,13 +1353,13 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
           ++ic;
           }
         }
-        if (lrow == 0) {                               // the staging area may be rewritten
+        if (i + 1 == nq && lrow == 0) {                // the staging area may be rewritten
           bulk_wait_group_read0();
           mbar_arrive(bar(C::B_STGFREE + (int)b));
         }
       }
     }
-    if (lrow == 0) bulk_wait_group0();                // copies done before the CTA exits
+    if (lane == 0) bulk_wait_group0();                // copies done before the CTA exits
   }
 
   // ------------------------------------------------------------ teardown
@@ -1402,7 +1417,7 @@ bool make_bwd_maps(const gdpa_problem_t& p, const void* q, const void* g, const 
 }
 
 // The fp32 dQ accumulator [T, h, DH] as the target of the half kernel's bulk
-// reduces: boxes of DH/2 columns x 128 rows of one head.
+// reduces: boxes of DH/2 columns x 32 rows (one drain warp's rows) of one head.
 template <int DH>
 bool make_dq_map(const gdpa_problem_t& p, float* dq_acc, CUtensorMap* m) {
   auto enc = tensor_map_encoder();
@@ -1412,7 +1427,7 @@ bool make_dq_map(const gdpa_problem_t& p, float* dq_acc, CUtensorMap* m) {
   const cuuint64_t d[3] = {(cuuint64_t)DH, (cuuint64_t)p.h,
                            (cuuint64_t)(p.total_tokens > 0 ? p.total_tokens : 1)};
   const cuuint64_t str[2] = {(cuuint64_t)DH * 4, (cuuint64_t)p.h * DH * 4};
-  const cuuint32_t box[3] = {(cuuint32_t)(DH / 2), 1, 128};
+  const cuuint32_t box[3] = {(cuuint32_t)(DH / 2), 1, 32};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dq_acc, d, str, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -1535,11 +1550,11 @@ cudaError_t launch_jag_bwd_t(int B, int h, int S, int64_t T, int window, float s
   if (POOL)
     okm = okm && map3(&mq, BF, 2, q, S, h, CH, 128, 1, sw) &&
           map3(&mg, BF, 2, g, S, (cuuint64_t)B * h, CH, 128, 1, sw) &&
-          map3(&mdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, acc, S, h, DH / 2, 128, 1, swq);
+          map3(&mdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, acc, S, h, DH / 2, 32, 1, swq);
   else
     okm = okm && map3(&mq, BF, 2, q, h, Tm, CH, 1, 128, sw) &&
           map3(&mg, BF, 2, g, h, Tm, CH, 1, 128, sw) &&
-          map3(&mdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, acc, h, Tm, DH / 2, 1, 128, swq);
+          map3(&mdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, acc, h, Tm, DH / 2, 1, 32, swq);
   if (!okm) return cudaErrorInvalidValue;
   BwdArgs args = {};
   args.tiles = tiles;
