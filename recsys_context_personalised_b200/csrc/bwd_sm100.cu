@@ -1091,6 +1091,19 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
           break;
         }
         tc_fence_after();
+        // every query row (seed) of this half lies past the sample: its P^T and
+        // dS^T columns are zero, and the dQ rows it would feed are never added
+        const bool empty_half = rbase >= (POOL ? a.S : n);
+        if (empty_half) {
+          uint32_t z[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) z[u] = 0u;
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            tmem_st_x16(tmem + lane_off + 128 * grp + 16 * ch, z);
+            tmem_st_x16(tmem + lane_off + 128 * grp + 64 + 16 * ch, z);
+          }
+        } else {
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           uint32_t s[32], dp[32];
@@ -1161,6 +1174,7 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                          "r"(dd[4 * jj + 1]), "r"(dd[4 * jj + 2]), "r"(dd[4 * jj + 3])
                          : "memory");
           }
+        }
         }
         tmem_wait_st();
         fence_proxy_async_smem();
