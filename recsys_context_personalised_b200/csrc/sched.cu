@@ -10,36 +10,124 @@
 #include "gdpa_internal.cuh"
 
 namespace gdpa {
+
+int device_sm_count();
+
 namespace {
 
 constexpr int kSchedThreads = 1024;
+constexpr int kSortMax = 4096;   // samples whose per-sample data a CTA keeps in shared memory
+
+// Checks the offsets (offsets[0] = 0, offsets[B] = T, 0 <= n_b <= max_n) in
+// every CTA; CTA 0 records the outcome in the workspace header.  Returns
+// whether they are valid (the same answer in every thread of the grid).
+__device__ bool offsets_valid(const int32_t* __restrict__ offsets, int B, int64_t T, int max_n,
+                              WsHeader* ws, int* s_bad) {
+  const int tid = threadIdx.x;
+  if (tid == 0) *s_bad = (offsets[0] != 0 || (int64_t)offsets[B] != T) ? 1 : 0;
+  __syncthreads();
+  for (int b = tid; b < B; b += blockDim.x) {
+    const int n = offsets[b + 1] - offsets[b];
+    if (n < 0 || n > max_n) *s_bad = 1;
+  }
+  __syncthreads();
+  const bool ok = *s_bad == 0;
+  if (blockIdx.x == 0 && tid == 0) {
+    ws->status = ok ? GDPA_OK : GDPA_ERR_INVALID_ARG;
+    if (!ok) ws->tile_count = 0;
+  }
+  return ok;
+}
+
+// Exclusive prefix sums of cnt(i), i in [0, N), handed to put(i, sum);
+// returns the total.  All threads of the block take part; thread i reads
+// cnt(i) before any put of its chunk.
+template <typename F, typename G>
+__device__ long long block_prefix(int N, F cnt, G put, int* s_warp, long long* s_carry) {
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
+  if (tid == 0) *s_carry = 0;
+  __syncthreads();
+  for (int base = 0; base < N; base += blockDim.x) {
+    const int i = base + tid;
+    const int v = i < N ? cnt(i) : 0;
+    int x = v;                                      // inclusive scan within the warp
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, d);
+      if (lane >= d) x += y;
+    }
+    if (lane == 31) s_warp[wid] = x;
+    __syncthreads();
+    if (wid == 0) {                                 // scan of the warp totals
+      int w = lane < nw ? s_warp[lane] : 0;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, d);
+        if (lane >= d) w += y;
+      }
+      if (lane < nw) s_warp[lane] = w;             // inclusive
+    }
+    __syncthreads();
+    const long long before = *s_carry + (wid > 0 ? s_warp[wid - 1] : 0);
+    if (i < N) put(i, (int)(before + x - v));
+    __syncthreads();
+    if (tid == 0) *s_carry += s_warp[nw - 1];
+    __syncthreads();
+  }
+  return *s_carry;
+}
+
+// The largest i in [0, N) with h * pre(i) <= idx (pre non-decreasing, pre(0) = 0).
+template <typename F>
+__device__ __forceinline__ int find_owner(F pre, int N, int h, long long idx) {
+  int lo = 0, hi = N - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((long long)h * pre(mid) <= idx) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
 
 __global__ void __launch_bounds__(kSchedThreads)
 schedule_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T, int max_n,
                 int bm, WsHeader* ws, Tile* __restrict__ tiles, int64_t cap) {
   __shared__ int s_bad;
-  __shared__ int s_scan[kSchedThreads];
+  __shared__ int s_pre[kSortMax];
+  __shared__ int s_warp[32];
   __shared__ long long s_carry;
+  if (!offsets_valid(offsets, B, T, max_n, ws, &s_bad)) return;
   const int tid = threadIdx.x;
-  if (tid == 0) {
-    s_bad = 0;
-    s_carry = 0;
-    ws->status = GDPA_OK;
-    if (offsets[0] != 0 || (int64_t)offsets[B] != T) s_bad = 1;
-  }
-  __syncthreads();
-  for (int b = tid; b < B; b += kSchedThreads) {
-    const int n = offsets[b + 1] - offsets[b];
-    if (n < 0 || n > max_n) s_bad = 1;
-  }
-  __syncthreads();
-  if (s_bad) {
-    if (tid == 0) {
-      ws->status = GDPA_ERR_INVALID_ARG;
-      ws->tile_count = 0;
+  if (B <= kSortMax) {
+    // every CTA forms the prefix of the tile counts, then the grid writes the
+    // items, each thread finding its item's sample by binary search
+    auto ntiles = [&](int b) { return (offsets[b + 1] - offsets[b] + bm - 1) / bm; };
+    auto put = [&](int b, int v) { s_pre[b] = v; };
+    auto pre = [&](int b) { return s_pre[b]; };
+    const long long total = block_prefix(B, ntiles, put, s_warp, &s_carry);
+    const long long items = (long long)h * total < cap ? (long long)h * total : cap;
+    for (long long idx = (long long)blockIdx.x * blockDim.x + tid; idx < items;
+         idx += (long long)gridDim.x * blockDim.x) {
+      const int b = find_owner(pre, B, h, idx);
+      const int n = offsets[b + 1] - offsets[b];
+      const int nt = (n + bm - 1) / bm;
+      const int rem = (int)(idx - (long long)h * s_pre[b]);
+      const int t = rem % nt;
+      Tile w;
+      w.b = b;
+      w.head = rem / nt;
+      w.row0 = offsets[b] + t * bm;
+      w.rows = min(bm, n - t * bm);
+      tiles[idx] = w;
     }
+    if (blockIdx.x == 0 && tid == 0) ws->tile_count = (int)items;
     return;
   }
+  // more samples than a CTA keeps: CTA 0 alone, one thread per sample
+  if (blockIdx.x != 0) return;
+  int* s_scan = s_pre;
+  if (tid == 0) s_carry = 0;
+  __syncthreads();
   for (int base = 0; base < B; base += kSchedThreads) {
     const int b = base + tid;
     const int n = b < B ? offsets[b + 1] - offsets[b] : 0;
@@ -77,8 +165,6 @@ schedule_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T, in
     ws->tile_count = (int)(total < cap ? total : cap);
   }
 }
-
-constexpr int kSortMax = 4096;   // 32 KB of static shared memory
 
 // Sorts the samples by length, longest first (ties: lower index first), into
 // s_key[0, B) as (n_b, b); entries [B, P2) pad with (-1, INT_MAX).  B <= kSortMax.
@@ -120,29 +206,13 @@ schedule_kv_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T,
                    int nkv, WsHeader* ws, Tile* __restrict__ tiles) {
   __shared__ int s_bad;
   __shared__ int2 s_key[kSortMax];   // (n_b, b)
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-    s_bad = 0;
-    ws->status = GDPA_OK;
-    if (offsets[0] != 0 || (int64_t)offsets[B] != T) s_bad = 1;
-  }
-  __syncthreads();
-  for (int b = tid; b < B; b += kSchedThreads) {
-    const int n = offsets[b + 1] - offsets[b];
-    if (n < 0 || n > max_n) s_bad = 1;
-  }
-  __syncthreads();
-  if (s_bad) {
-    if (tid == 0) {
-      ws->status = GDPA_ERR_INVALID_ARG;
-      ws->tile_count = 0;
-    }
-    return;
-  }
+  if (!offsets_valid(offsets, B, T, max_n, ws, &s_bad)) return;
+  // every CTA sorts; the grid writes the items
   const bool sorted = B <= kSortMax;
   if (sorted) sort_by_length(offsets, B, s_key);
   const long long per_sample = (long long)h * nkv;
-  for (long long idx = tid; idx < (long long)B * per_sample; idx += kSchedThreads) {
+  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+       idx < (long long)B * per_sample; idx += (long long)gridDim.x * blockDim.x) {
     const int r = (int)(idx / per_sample);
     const int rem = (int)(idx % per_sample);
     const int b = sorted ? s_key[r].y : r;
@@ -153,9 +223,8 @@ schedule_kv_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T,
     w.rows = offsets[b + 1] - offsets[b];
     tiles[idx] = w;
   }
-  if (tid == 0) ws->tile_count = (int)((long long)B * per_sample);
+  if (blockIdx.x == 0 && threadIdx.x == 0) ws->tile_count = (int)((long long)B * per_sample);
 }
-
 
 // Seed-pooling work list: one item per (sample, pair of heads 2k, 2k+1) of the
 // samples that have tokens, longest samples first (B <= 4096): item fields
@@ -212,67 +281,33 @@ __global__ void __launch_bounds__(kSchedThreads)
 schedule_jkv_kernel(const int32_t* __restrict__ offsets, int B, int h, int64_t T, int max_n,
                     WsHeader* ws, Tile* __restrict__ tiles, int64_t cap) {
   __shared__ int s_bad;
+  __shared__ int s_warp[32];
   __shared__ long long s_carry;
-  __shared__ int s_scan[kSchedThreads];
-  __shared__ int2 s_key[kSortMax];   // (n_b, b)
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-    s_bad = 0;
-    s_carry = 0;
-    ws->status = GDPA_OK;
-    if (offsets[0] != 0 || (int64_t)offsets[B] != T) s_bad = 1;
-  }
-  __syncthreads();
-  for (int b = tid; b < B; b += kSchedThreads) {
-    const int n = offsets[b + 1] - offsets[b];
-    if (n < 0 || n > max_n) s_bad = 1;
-  }
-  __syncthreads();
-  if (s_bad) {
-    if (tid == 0) {
-      ws->status = GDPA_ERR_INVALID_ARG;
-      ws->tile_count = 0;
-    }
-    return;
-  }
+  __shared__ int2 s_key[kSortMax];   // (n_b, b), then (prefix of the key-block counts, b)
+  if (!offsets_valid(offsets, B, T, max_n, ws, &s_bad)) return;
+  // every CTA sorts and forms the prefix of the key-block counts in sorted
+  // order (samples without tokens sort last); the grid writes the items
   sort_by_length(offsets, B, s_key);
-  // exclusive scan of the key-block counts in sorted order, then the items
-  for (int base = 0; base < B; base += kSchedThreads) {
-    const int r = base + tid;
-    const int n = r < B ? max(s_key[r].x, 0) : 0;
+  auto nblocks = [&](int r) { return (max(s_key[r].x, 0) + 127) >> 7; };
+  auto put = [&](int r, int v) { s_key[r].x = v; };
+  auto pre = [&](int r) { return s_key[r].x; };
+  const long long total = block_prefix(B, nblocks, put, s_warp, &s_carry);
+  const long long items = (long long)h * total < cap ? (long long)h * total : cap;
+  for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < items;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int r = find_owner(pre, B, h, idx);
+    const int b = s_key[r].y;
+    const int n = offsets[b + 1] - offsets[b];
     const int nb = (n + 127) >> 7;
-    s_scan[tid] = nb;
-    __syncthreads();
-    for (int d = 1; d < kSchedThreads; d <<= 1) {
-      const int add = tid >= d ? s_scan[tid - d] : 0;
-      __syncthreads();
-      s_scan[tid] += add;
-      __syncthreads();
-    }
-    const long long excl = s_carry + s_scan[tid] - nb;
-    if (nb > 0) {
-      const int b = s_key[r].y;
-      for (int j = 0; j < h; ++j)
-        for (int kb = 0; kb < nb; ++kb) {
-          const long long idx = (long long)h * excl + (long long)j * nb + kb;
-          if (idx < cap) {
-            Tile w;
-            w.b = b;
-            w.head = j;
-            w.row0 = 128 * kb;
-            w.rows = n;
-            tiles[idx] = w;
-          }
-        }
-    }
-    __syncthreads();
-    if (tid == kSchedThreads - 1) s_carry += s_scan[kSchedThreads - 1];
-    __syncthreads();
+    const int rem = (int)(idx - (long long)h * s_key[r].x);
+    Tile w;
+    w.b = b;
+    w.head = rem / nb;
+    w.row0 = 128 * (rem % nb);
+    w.rows = n;
+    tiles[idx] = w;
   }
-  if (tid == 0) {
-    const long long total = (long long)h * s_carry;
-    ws->tile_count = (int)(total < cap ? total : cap);
-  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) ws->tile_count = (int)items;
 }
 
 // Outputs of the samples without tokens: O = 0 and LSE = -inf (every seed
@@ -297,7 +332,7 @@ __global__ void pool_empty_kernel(const int32_t* __restrict__ offsets, int B, in
 cudaError_t launch_schedule_kv(const gdpa_problem_t& p, const int32_t* offsets, WsHeader* ws,
                                Tile* tiles, cudaStream_t st) {
   KernelScope ks_("gdpa_schedule_kv", st);
-  schedule_kv_kernel<<<1, kSchedThreads, 0, st>>>(offsets, p.B, p.h, p.total_tokens, p.max_n,
+  schedule_kv_kernel<<<device_sm_count(), kSchedThreads, 0, st>>>(offsets, p.B, p.h, p.total_tokens, p.max_n,
                                                    (p.m + 127) / 128, ws, tiles);
   return cudaGetLastError();
 }
@@ -305,7 +340,7 @@ cudaError_t launch_schedule_kv(const gdpa_problem_t& p, const int32_t* offsets, 
 cudaError_t launch_schedule(const gdpa_problem_t& p, const int32_t* offsets, int bm,
                             WsHeader* ws, Tile* tiles, cudaStream_t st) {
   KernelScope ks_("gdpa_schedule", st);
-  schedule_kernel<<<1, kSchedThreads, 0, st>>>(offsets, p.B, p.h, p.total_tokens, p.max_n,
+  schedule_kernel<<<device_sm_count(), kSchedThreads, 0, st>>>(offsets, p.B, p.h, p.total_tokens, p.max_n,
                                                 bm, ws, tiles, tile_capacity(p, bm));
   return cudaGetLastError();
 }
@@ -324,7 +359,7 @@ cudaError_t launch_schedule_pool(const int32_t* offsets, int B, int h, int64_t T
 cudaError_t launch_schedule_jkv(const int32_t* offsets, int B, int h, int64_t T, int max_n,
                                 WsHeader* ws, Tile* tiles, int64_t cap, cudaStream_t st) {
   KernelScope ks_("gdpa_schedule_jkv", st);
-  schedule_jkv_kernel<<<1, kSchedThreads, 0, st>>>(offsets, B, h, T, max_n, ws, tiles, cap);
+  schedule_jkv_kernel<<<device_sm_count(), kSchedThreads, 0, st>>>(offsets, B, h, T, max_n, ws, tiles, cap);
   return cudaGetLastError();
 }
 
