@@ -185,7 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmG,
                       const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, const BwdArgs a) {
+                      const __grid_constant__ CUtensorMap tmV,
+                      const __grid_constant__ CUtensorMap tmDQ, const BwdArgs a) {
   static_assert(DH == 128, "dh <= 64 runs gdpa_bwd_half_kernel");
   using C = BwdCfg<DH>;
   constexpr bool SOFTMAX = PHI == GDPA_PHI_SOFTMAX;
@@ -415,14 +416,17 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         if (!__all_sync(0xffffffffu, w)) return false;
         tc_fence_after();
         // Lane = query row.  This group's DH/2 columns go through the warp's
-        // shared-memory area, 32 fp32 columns (128 B of a row) at a time, so
-        // that each vector reduction instruction covers 4 whole row pieces.
+        // shared-memory area, 32 fp32 columns (128 B of a row) at a time, as a
+        // swizzled [32 x 32] box that one lane adds into the fp32 accumulator
+        // with a bulk tensor reduce-add.  Rows past the sample are exact zeros
+        // (their dS is zero): a warp whose rows all lie there adds nothing, and
+        // rows past T are clipped by the map.
         const uint32_t kstg = base + C::OFF_KSTG + (uint32_t)(warp - 4) * C::KSTG_WARP;
-        const int rl = lane >> 3, jl = lane & 7;
-        float* rows = a.dq_acc + ((int64_t)(t0 + 128 * ii + quad * 32) * a.h + it.head) * DH +
-                      grp * (DH / 2);
+        const bool adds = 128 * ii + quad * 32 < n;
 #pragma unroll
         for (int c0 = 0; c0 < DH / 2; c0 += 32) {
+          if (lane == 0) bulk_wait_group_read0();      // the area's last bulk copy has read it
+          __syncwarp();
 #pragma unroll
           for (int c = 0; c < 32; c += 16) {
             uint32_t v[16];
@@ -441,18 +445,12 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                            : "memory");
             }
           }
+          fence_proxy_async_smem();
           __syncwarp();
-#pragma unroll
-          for (int it4 = 0; it4 < 8; ++it4) {
-            const int r = it4 * 4 + rl;                  // row within this warp's 32
-            float4 val;
-            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                         : "=f"(val.x), "=f"(val.y), "=f"(val.z), "=f"(val.w)
-                         : "r"(kstg + r * 128 + (((uint32_t)jl ^ (uint32_t)(r & 7)) << 4)));
-            if (128 * ii + quad * 32 + r < n)
-              red_add_v4(rows + (int64_t)r * a.h * DH + c0 + jl * 4, val.x, val.y, val.z, val.w);
+          if (adds && lane == 0) {
+            tma_reduce_add_3d(&tmDQ, kstg, grp * (DH / 2) + c0, it.head, t0 + 128 * ii + quad * 32);
+            bulk_commit_group();
           }
-          __syncwarp();
         }
         return true;
       };
@@ -590,6 +588,8 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         const int rl = lane >> 3, jl = lane & 7;         // read-back: row in group of 4, chunk
 #pragma unroll
         for (int c0 = 0; c0 < DH; c0 += 64) {
+          if (lane == 0) bulk_wait_group_read0();      // a dQ reduce may still read the area
+          __syncwarp();
 #pragma unroll
           for (int c = 0; c < 64; c += 16) {
             uint32_t v[16];
@@ -629,6 +629,7 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
       ++ic;
     }
+    if (lane == 0) bulk_wait_group0();                // reduces done before the CTA exits
   }
 
   // ------------------------------------------------------------ teardown
@@ -1430,18 +1431,20 @@ bool make_bwd_maps(const gdpa_problem_t& p, const void* q, const void* g, const 
   return true;
 }
 
-// The fp32 dQ accumulator [T, h, DH] as the target of the half kernel's bulk
-// reduces: boxes of DH/2 columns x 32 rows (one drain warp's rows) of one head.
+// The fp32 dQ accumulator [T, h, DH] as the target of the bulk reduces: boxes
+// of 32 rows (one warp's rows) of one head, DH/2 columns (dh <= 64) or 32
+// (dh = 128: at most 128 B of a row under the swizzle).
 template <int DH>
 bool make_dq_map(const gdpa_problem_t& p, float* dq_acc, CUtensorMap* m) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
-  const CUtensorMapSwizzle sw = DH / 2 * 4 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  constexpr int BX = DH / 2 > 32 ? 32 : DH / 2;
+  const CUtensorMapSwizzle sw = BX * 4 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   const cuuint32_t estr[3] = {1, 1, 1};
   const cuuint64_t d[3] = {(cuuint64_t)DH, (cuuint64_t)p.h,
                            (cuuint64_t)(p.total_tokens > 0 ? p.total_tokens : 1)};
   const cuuint64_t str[2] = {(cuuint64_t)DH * 4, (cuuint64_t)p.h * DH * 4};
-  const cuuint32_t box[3] = {(cuuint32_t)(DH / 2), 1, 32};
+  const cuuint32_t box[3] = {(cuuint32_t)BX, 1, 32};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dq_acc, d, str, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -1488,10 +1491,12 @@ cudaError_t launch_bwd_t(const gdpa_problem_t& p, const void* q, const int32_t* 
   } else {
     using C = BwdCfg<DH>;
     auto kern = gdpa_bwd_sm100_kernel<DH, PHI, BIAS>;     // dh = 128 only
+    CUtensorMap mdq;
+    if (!make_dq_map<DH>(p, dq_acc, &mdq)) return cudaErrorInvalidValue;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     if (e != cudaSuccess) return e;
     KernelScope ks_("gdpa_bwd_sm100", st);
-    kern<<<device_sm_count(), kThreads, C::SMEM, st>>>(mq, mg, mk, mv, args);
+    kern<<<device_sm_count(), kThreads, C::SMEM, st>>>(mq, mg, mk, mv, mdq, args);
     return cudaGetLastError();
   }
 }
