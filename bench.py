@@ -59,11 +59,11 @@ KERNEL_SOURCES = {"gdpa_fwd_sm100": ("fwd_sm100.cu", "sm100.cuh", "gdpa_internal
 # sha16 of the kernel's sources at capture time)}}.  An entry whose hash no
 # longer matches the sources is not used (the traffic is then reported null).
 TRAFFIC_PER_UNIT = {
-    # 64-sample cases: workload 5, 583.1 MB read + 36.0 MB written in one launch;
-    # workload 4, 347.2 MB + 60.6 MB
-    "gdpa_fwd_sm100": {5: (0.0141601, "209e3f60a671ea6a"), 4: (0.0101353, "209e3f60a671ea6a")},
-    # workload 5: 748.9 MB read + 592.6 MB written; workload 4: 597.1 MB + 376.4 MB
-    "gdpa_bwd_sm100": {5: (0.0306869, "2b7bb8db654a3d62"), 4: (0.0241974, "7212f118d73e1f69")},
+    # 64-sample cases: workload 5, 582.3 MB read + 36.1 MB written in one launch;
+    # workload 4, 347.1 MB + 60.0 MB
+    "gdpa_fwd_sm100": {5: (0.0141458, "209e3f60a671ea6a"), 4: (0.0101203, "209e3f60a671ea6a")},
+    # workload 5: 733.3 MB read + 580.2 MB written; workload 4: 599.3 MB + 377.8 MB
+    "gdpa_bwd_sm100": {5: (0.0300473, "70ea3c79d420f1b8"), 4: (0.0242885, "70ea3c79d420f1b8")},
 }
 # fp32 FFMA peak for the SIMT kernels: 148 SMs * 128 FMA/clk * 2 flop * 1.965 GHz
 SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
