@@ -768,7 +768,7 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctl + 8 * C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctl + 8 * C::NBAR + 4);
-  float* stats = reinterpret_cast<float*>(ctl + 1024);   // [2 slots][LSE, D][128]
+  float* stats = reinterpret_cast<float*>(ctl + 1024);   // [2 slots][-LSE, -D][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -1019,7 +1019,7 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
     }
     else if (warp == 2 && SOFTMAX) {
       // -------------------------------------------------------- row statistics
-      // log2-scaled LSE and D of each query tile into the ring, one tile ahead
+      // -LSE (log2-scaled) and -D of each query tile into the ring, one tile ahead
       uint32_t q = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < count; t += gridDim.x) {
@@ -1036,7 +1036,7 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
             ok = false;
             break;
           }
-          float* ring = stats + slot * 256;
+          float* ring = stats + slot * 256;      // negated, as the activation adds them
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int r = 32 * u + lane, rg = 128 * (fi + i) + r;
@@ -1047,8 +1047,8 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
               l = __ldg(a.lse + at) * 1.4426950408889634f;
               d = __ldg(a.dsum + at);
             }
-            ring[r] = l;
-            ring[128 + r] = d;
+            ring[r] = -l;
+            ring[128 + r] = -d;
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(C::B_STATFULL + (int)slot));
@@ -1115,7 +1115,7 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             float pv[2], dv2[2];
-            float2 gp, gd;                                // GELU: phi and phi' of the pair
+            float2 gp, gd;              // softmax: P and dS, GELU: phi and phi' of the pair
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int r = 32 * ch + c + e;
@@ -1124,8 +1124,19 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
               float p, ds;
               // u = s x + b1 (the biased logit; b1k = 0 without a key bias)
               if constexpr (SOFTMAX) {
-                p = ex2_approx(fmaf(x, c2, BIAS ? b1l - st_l[r] : -st_l[r]));
-                ds = p * (g - st_d[r]);
+                if (e == 0) {         // both columns of the pair, in packed arithmetic
+                  const float2 nl = *reinterpret_cast<const float2*>(st_l + r);   // -LSE
+                  const float2 nd = *reinterpret_cast<const float2*>(st_d + r);   // -D
+                  const float2 u = __ffma2_rn(
+                      make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                      make_float2(c2, c2), BIAS ? __fadd2_rn(nl, make_float2(b1l, b1l)) : nl);
+                  gp = make_float2(ex2_approx(u.x), ex2_approx(u.y));
+                  gd = __fmul2_rn(gp, __fadd2_rn(make_float2(__uint_as_float(dp[c]),
+                                                             __uint_as_float(dp[c + 1])),
+                                                 nd));
+                }
+                p = e ? gp.y : gp.x;
+                ds = e ? gd.y : gd.x;
               } else if constexpr (PHI == GDPA_PHI_SILU) {
                 const float hx = fmaf(x, half_sc, hb);
                 const float th = tanh_approx(hx);
