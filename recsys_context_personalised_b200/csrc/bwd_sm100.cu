@@ -1040,7 +1040,9 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int r = 32 * u + lane, rg = 128 * (fi + i) + r;
-            float l = 0.f, d = 0.f;
+            // rows past the sample (pooling: seeds >= S) take -LSE = -inf, so
+            // that their P and dS come out exactly 0
+            float l = INFINITY, d = 0.f;
             if (POOL ? r < a.S : rg < it.rows) {
               const int64_t at = POOL ? ((int64_t)it.b * a.h + it.head) * a.S + r
                                       : (int64_t)it.head * a.T + t0 + rg;
@@ -1164,6 +1166,8 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                 valid = key_ok && qr < a.S;
               else if constexpr (WIN)
                 valid = key_ok && qr < n && key <= qr && key > qr - a.window;
+              else if constexpr (SOFTMAX)
+                valid = true;         // rows past the sample: P = exp2(-inf) = 0, dS = 0
               else
                 valid = qr < n;
               pv[e] = valid ? p : 0.f;
