@@ -46,6 +46,19 @@ using namespace sm100;
 constexpr int kThreads = 384;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
+// SiLU and its gradient on a pair of columns, in packed arithmetic: with
+// hx = u/2, phi(u) = hx (1 + tanh hx) and dS = dP * sg * (1 + u (1 - sg)),
+// sg = logistic(u) = (1 + tanh hx) / 2.
+__device__ __forceinline__ void silu_fg2(float2 hx, float2 g, float2& p, float2& ds) {
+  const float2 th = make_float2(tanh_approx(hx.x), tanh_approx(hx.y));
+  const float2 sg = __ffma2_rn(make_float2(0.5f, 0.5f), th, make_float2(0.5f, 0.5f));
+  p = __ffma2_rn(hx, th, hx);
+  const float2 t = __ffma2_rn(__fadd2_rn(hx, hx), __fadd2_rn(make_float2(1.f, 1.f),
+                                                             make_float2(-sg.x, -sg.y)),
+                              make_float2(1.f, 1.f));
+  ds = __fmul2_rn(__fmul2_rn(g, sg), t);
+}
+
 // ---------------------------------------------------------------- prep / convert
 
 // Zeroes the fp32 dQ workspace (n4 float4s) and, for softmax, writes the row
@@ -460,7 +473,7 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int rg = 128 * ii + 64 * grp + 32 * u + lane;
-          nl[u] = 0.f;
+          nl[u] = INFINITY;                            // rows past the sample: P = 0
           nd[u] = 0.f;
           if (rg < n) {
             const int64_t at = (int64_t)it.head * a.T + t0 + rg;
@@ -475,10 +488,9 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         if constexpr (SOFTMAX) {
           __syncwarp();
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            wst[32 * u + lane] = nl[u] * 1.4426950408889634f;   // log2 units
-            wst[64 + 32 * u + lane] = nd[u];
-          }
+          for (int u = 0; u < 2; ++u)        // (-LSE in log2 units, -D) per row
+            *reinterpret_cast<float2*>(wst + 2 * (32 * u + lane)) =
+                make_float2(-nl[u] * 1.4426950408889634f, -nd[u]);
           __syncwarp();
           if (i + 1 < nq) load_stats(i + 1);
         }
@@ -499,7 +511,7 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             float pv[2], dv2[2];
-            float2 gp, gd;                                // GELU: phi and phi' of the pair
+            float2 gp, gd;              // phi and dS (GELU: phi') of the pair
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int r = 32 * ch + c + e;
@@ -508,14 +520,26 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
               float p, ds;
               // u = s x + b1 (the biased logit; b1k = 0 without a key bias)
               if constexpr (SOFTMAX) {
-                p = ex2_approx(fmaf(x, c2, BIAS ? b1l - wst[r] : -wst[r]));
-                ds = p * (g - wst[64 + r]);
+                if (e == 0) {         // both columns of the pair, in packed arithmetic
+                  const float4 q4 = *reinterpret_cast<const float4*>(wst + 2 * r);  // rows r, r+1
+                  const float2 nlv = make_float2(q4.x, q4.z), ndv = make_float2(q4.y, q4.w);
+                  const float2 u = __ffma2_rn(
+                      make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                      make_float2(c2, c2), BIAS ? __fadd2_rn(nlv, make_float2(b1l, b1l)) : nlv);
+                  gp = make_float2(ex2_approx(u.x), ex2_approx(u.y));
+                  gd = __fmul2_rn(gp, __fadd2_rn(make_float2(__uint_as_float(dp[c]),
+                                                             __uint_as_float(dp[c + 1])),
+                                                 ndv));
+                }
+                p = e ? gp.y : gp.x;
+                ds = e ? gd.y : gd.x;
               } else if constexpr (PHI == GDPA_PHI_SILU) {
-                const float hx = fmaf(x, half_sc, hb);
-                const float th = tanh_approx(hx);
-                const float sg = fmaf(0.5f, th, 0.5f);          // logistic(u)
-                p = fmaf(hx, th, hx);                             // u * logistic(u)
-                ds = g * sg * fmaf(hx + hx, 1.f - sg, 1.f);
+                if (e == 0)           // both columns of the pair, in packed arithmetic
+                  silu_fg2(__ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                      make_float2(half_sc, half_sc), make_float2(hb, hb)),
+                           make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), gp, gd);
+                p = e ? gp.y : gp.x;
+                ds = e ? gd.y : gd.x;
               } else if constexpr (PHI == GDPA_PHI_RELU) {
                 const float u = fmaf(x, sc, b1k);
                 p = relu_f(u);
@@ -531,7 +555,8 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                 p = fmaf(x, sc, b1k);
                 ds = g;
               }
-              const bool valid = rbase + r < n;
+              // softmax rows past the sample already give P = dS = 0 (-LSE = -inf)
+              const bool valid = SOFTMAX || rbase + r < n;
               pv[e] = valid ? p : 0.f;
               dv2[e] = valid ? ds : 0.f;
               if constexpr (BIAS) db1_acc += dv2[e];
@@ -1140,11 +1165,12 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                 p = e ? gp.y : gp.x;
                 ds = e ? gd.y : gd.x;
               } else if constexpr (PHI == GDPA_PHI_SILU) {
-                const float hx = fmaf(x, half_sc, hb);
-                const float th = tanh_approx(hx);
-                const float sg = fmaf(0.5f, th, 0.5f);          // logistic(u)
-                p = fmaf(hx, th, hx);                             // u * logistic(u)
-                ds = g * sg * fmaf(hx + hx, 1.f - sg, 1.f);
+                if (e == 0)           // both columns of the pair, in packed arithmetic
+                  silu_fg2(__ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                      make_float2(half_sc, half_sc), make_float2(hb, hb)),
+                           make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), gp, gd);
+                p = e ? gp.y : gp.x;
+                ds = e ? gd.y : gd.x;
               } else if constexpr (PHI == GDPA_PHI_RELU) {
                 const float u = fmaf(x, sc, b1k);
                 p = relu_f(u);
