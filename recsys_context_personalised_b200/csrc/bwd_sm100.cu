@@ -1104,9 +1104,13 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
       const bool key_ok = !JAG || key < n;              // jagged keys: rows past the sample
       const float b1k = BIAS ? key_bias(a, it, key) : 0.f;
       const float b1l = b1k * 1.4426950408889634f, hb = 0.5f * b1k;
+      // added to the softmax exponent of every pair of this key (log2 units)
+      const float kterm = BIAS ? b1l : (key_ok ? 0.f : -INFINITY);
       float db1_acc = 0.f;
       for (int i = 0; i < nq; ++i, ++qs) {
         const int rbase = 128 * (fi + i) + 64 * grp;   // first sample row (seed) of this half
+        const int band0 = rbase - key;                 // window: row rbase + r is in band iff
+                                                       // 0 <= band0 + r < window
         const uint32_t dsb = sDS + (qs & 1u) * C::DSB + grp * 16384;
         const float* st_l = stats + (qs & 1u) * 256 + 64 * grp;
         const float* st_d = st_l + 128;
@@ -1154,9 +1158,15 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (e == 0) {         // both columns of the pair, in packed arithmetic
                   const float2 nl = *reinterpret_cast<const float2*>(st_l + r);   // -LSE
                   const float2 nd = *reinterpret_cast<const float2*>(st_d + r);   // -D
-                  const float2 u = __ffma2_rn(
+                  // the key's term: its bias, or -inf for a jagged key past the sample
+                  float2 u = __ffma2_rn(
                       make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
-                      make_float2(c2, c2), BIAS ? __fadd2_rn(nl, make_float2(b1l, b1l)) : nl);
+                      make_float2(c2, c2),
+                      BIAS || JAG ? __fadd2_rn(nl, make_float2(kterm, kterm)) : nl);
+                  if constexpr (WIN) {    // the band key <= t < key + window
+                    u.x = (uint32_t)(band0 + r) < (uint32_t)a.window ? u.x : -INFINITY;
+                    u.y = (uint32_t)(band0 + r + 1) < (uint32_t)a.window ? u.y : -INFINITY;
+                  }
                   gp = make_float2(ex2_approx(u.x), ex2_approx(u.y));
                   gd = __fmul2_rn(gp, __fadd2_rn(make_float2(__uint_as_float(dp[c]),
                                                              __uint_as_float(dp[c + 1])),
@@ -1186,16 +1196,9 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                 p = fmaf(x, sc, b1k);
                 ds = g;
               }
-              const int qr = rbase + r;                   // query row (pooling: seed)
-              bool valid;
-              if constexpr (POOL)
-                valid = key_ok && qr < a.S;
-              else if constexpr (WIN)
-                valid = key_ok && qr < n && key <= qr && key > qr - a.window;
-              else if constexpr (SOFTMAX)
-                valid = true;         // rows past the sample: P = exp2(-inf) = 0, dS = 0
-              else
-                valid = qr < n;
+              // softmax: rows past the sample (-LSE = -inf), keys past it and
+              // pairs outside the window (exponent -inf) give P = dS = 0 exactly
+              const bool valid = SOFTMAX || rbase + r < n;
               pv[e] = valid ? p : 0.f;
               dv2[e] = valid ? ds : 0.f;
               if constexpr (BIAS) db1_acc += dv2[e];
