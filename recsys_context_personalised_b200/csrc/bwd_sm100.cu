@@ -488,9 +488,10 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         if constexpr (SOFTMAX) {
           __syncwarp();
 #pragma unroll
-          for (int u = 0; u < 2; ++u)        // (-LSE in log2 units, -D) per row
-            *reinterpret_cast<float2*>(wst + 2 * (32 * u + lane)) =
-                make_float2(-nl[u] * 1.4426950408889634f, -nd[u]);
+          for (int u = 0; u < 2; ++u) {      // -LSE (log2 units) and -D of the 64 rows
+            wst[32 * u + lane] = -nl[u] * 1.4426950408889634f;
+            wst[64 + 32 * u + lane] = -nd[u];
+          }
           __syncwarp();
           if (i + 1 < nq) load_stats(i + 1);
         }
@@ -508,6 +509,7 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           tmem_ld_x32(tmem + lane_off + C::COL_DP + col, dp);
           tmem_wait_ld();
           uint32_t pp[16], dd[16];
+          float4 nl4, nd4;            // softmax: -LSE and -D of rows c..c+3
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             float pv[2], dv2[2];
@@ -521,8 +523,12 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
               // u = s x + b1 (the biased logit; b1k = 0 without a key bias)
               if constexpr (SOFTMAX) {
                 if (e == 0) {         // both columns of the pair, in packed arithmetic
-                  const float4 q4 = *reinterpret_cast<const float4*>(wst + 2 * r);  // rows r, r+1
-                  const float2 nlv = make_float2(q4.x, q4.z), ndv = make_float2(q4.y, q4.w);
+                  if ((c & 2) == 0) {   // rows r..r+3 (16-byte aligned)
+                    nl4 = *reinterpret_cast<const float4*>(wst + r);
+                    nd4 = *reinterpret_cast<const float4*>(wst + 64 + r);
+                  }
+                  const float2 nlv = (c & 2) ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
+                  const float2 ndv = (c & 2) ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
                   const float2 u = __ffma2_rn(
                       make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
                       make_float2(c2, c2), BIAS ? __fadd2_rn(nlv, make_float2(b1l, b1l)) : nlv);
@@ -1143,6 +1149,7 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
           tmem_ld_x32(tmem + lane_off + 128 * grp + 64 + 32 * ch, dp);
           tmem_wait_ld();
           uint32_t pp[16], dd[16];
+          float4 nl4, nd4;            // softmax: -LSE and -D of rows c..c+3
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             float pv[2], dv2[2];
@@ -1156,8 +1163,12 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
               // u = s x + b1 (the biased logit; b1k = 0 without a key bias)
               if constexpr (SOFTMAX) {
                 if (e == 0) {         // both columns of the pair, in packed arithmetic
-                  const float2 nl = *reinterpret_cast<const float2*>(st_l + r);   // -LSE
-                  const float2 nd = *reinterpret_cast<const float2*>(st_d + r);   // -D
+                  if ((c & 2) == 0) {   // rows r..r+3 (16-byte aligned)
+                    nl4 = *reinterpret_cast<const float4*>(st_l + r);
+                    nd4 = *reinterpret_cast<const float4*>(st_d + r);
+                  }
+                  const float2 nl = (c & 2) ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
+                  const float2 nd = (c & 2) ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
                   // the key's term: its bias, or -inf for a jagged key past the sample
                   float2 u = __ffma2_rn(
                       make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
