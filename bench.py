@@ -59,11 +59,11 @@ KERNEL_SOURCES = {"gdpa_fwd_sm100": ("fwd_sm100.cu", "sm100.cuh", "gdpa_internal
 # sha16 of the kernel's sources at capture time)}}.  An entry whose hash no
 # longer matches the sources is not used (the traffic is then reported null).
 TRAFFIC_PER_UNIT = {
-    # 64-sample cases: workload 5, 582.2 MB read + 36.2 MB written in one launch;
-    # workload 4, 347.1 MB + 59.1 MB
-    "gdpa_fwd_sm100": {5: (0.0141466, "209e3f60a671ea6a"), 4: (0.0100976, "209e3f60a671ea6a")},
-    # workload 5: 732.4 MB read + 579.0 MB written; workload 4: 599.4 MB + 379.5 MB
-    "gdpa_bwd_sm100": {5: (0.0299975, "ad8d085c9f60628c"), 4: (0.0243329, "ad8d085c9f60628c")},
+    # 64-sample cases: workload 5, 582.4 MB read + 35.7 MB written in one launch;
+    # workload 4, 347.2 MB + 59.9 MB
+    "gdpa_fwd_sm100": {5: (0.0141401, "209e3f60a671ea6a"), 4: (0.0101205, "209e3f60a671ea6a")},
+    # workload 5: 734.0 MB read + 580.0 MB written; workload 4: 599.8 MB + 380.7 MB
+    "gdpa_bwd_sm100": {5: (0.0300559, "95bf26a9bb1d5d5c"), 4: (0.0243723, "95bf26a9bb1d5d5c")},
 }
 # fp32 FFMA peak for the SIMT kernels: 148 SMs * 128 FMA/clk * 2 flop * 1.965 GHz
 SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
