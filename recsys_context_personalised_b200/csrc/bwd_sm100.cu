@@ -503,87 +503,96 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           break;
         }
         tc_fence_after();
+        // FULL: every query row of the group's half lies in the sample, so the
+        // activations other than softmax need no row mask either
+        auto half_body = [&](auto full_tag) {
+          constexpr bool FULL = decltype(full_tag)::value;
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          const uint32_t col = 64 * grp + 32 * ch;
-          uint32_t s[32], dp[32];
-          tmem_ld_x32(tmem + lane_off + C::COL_S + col, s);
-          tmem_ld_x32(tmem + lane_off + C::COL_DP + col, dp);
-          tmem_wait_ld();
-          uint32_t pp[16], dd[16];
-          float4 nl4, nd4;            // softmax: -LSE and -D of rows c..c+3
+          for (int ch = 0; ch < 2; ++ch) {
+            const uint32_t col = 64 * grp + 32 * ch;
+            uint32_t s[32], dp[32];
+            tmem_ld_x32(tmem + lane_off + C::COL_S + col, s);
+            tmem_ld_x32(tmem + lane_off + C::COL_DP + col, dp);
+            tmem_wait_ld();
+            uint32_t pp[16], dd[16];
+            [[maybe_unused]] float4 nl4, nd4;   // softmax: -LSE and -D of rows c..c+3
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float pv[2], dv2[2];
-            float2 gp, gd;              // phi and dS (GELU: phi') of the pair
+            for (int c = 0; c < 32; c += 2) {
+              float pv[2], dv2[2];
+              [[maybe_unused]] float2 gp, gd;   // phi and dS (GELU: phi') of the pair
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int r = 32 * ch + c + e;
-              const float x = __uint_as_float(s[c + e]);
-              const float g = __uint_as_float(dp[c + e]);
-              float p, ds;
-              // u = s x + b1 (the biased logit; b1k = 0 without a key bias)
-              if constexpr (SOFTMAX) {
-                if (e == 0) {         // both columns of the pair, in packed arithmetic
-                  if ((c & 2) == 0) {   // rows r..r+3 (16-byte aligned)
-                    nl4 = *reinterpret_cast<const float4*>(wst + r);
-                    nd4 = *reinterpret_cast<const float4*>(wst + 64 + r);
+              for (int e = 0; e < 2; ++e) {
+                const int r = 32 * ch + c + e;
+                const float x = __uint_as_float(s[c + e]);
+                const float g = __uint_as_float(dp[c + e]);
+                float p, ds;
+                // u = s x + b1 (the biased logit; b1k = 0 without a key bias)
+                if constexpr (SOFTMAX) {
+                  if (e == 0) {         // both columns of the pair, in packed arithmetic
+                    if ((c & 2) == 0) {   // rows r..r+3 (16-byte aligned)
+                      nl4 = *reinterpret_cast<const float4*>(wst + r);
+                      nd4 = *reinterpret_cast<const float4*>(wst + 64 + r);
+                    }
+                    const float2 nlv = (c & 2) ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
+                    const float2 ndv = (c & 2) ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
+                    const float2 u = __ffma2_rn(
+                        make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                        make_float2(c2, c2), BIAS ? __fadd2_rn(nlv, make_float2(b1l, b1l)) : nlv);
+                    gp = make_float2(ex2_approx(u.x), ex2_approx(u.y));
+                    gd = __fmul2_rn(gp, __fadd2_rn(make_float2(__uint_as_float(dp[c]),
+                                                               __uint_as_float(dp[c + 1])),
+                                                   ndv));
                   }
-                  const float2 nlv = (c & 2) ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
-                  const float2 ndv = (c & 2) ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
-                  const float2 u = __ffma2_rn(
-                      make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
-                      make_float2(c2, c2), BIAS ? __fadd2_rn(nlv, make_float2(b1l, b1l)) : nlv);
-                  gp = make_float2(ex2_approx(u.x), ex2_approx(u.y));
-                  gd = __fmul2_rn(gp, __fadd2_rn(make_float2(__uint_as_float(dp[c]),
-                                                             __uint_as_float(dp[c + 1])),
-                                                 ndv));
+                  p = e ? gp.y : gp.x;
+                  ds = e ? gd.y : gd.x;
+                } else if constexpr (PHI == GDPA_PHI_SILU) {
+                  if (e == 0)           // both columns of the pair, in packed arithmetic
+                    silu_fg2(__ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                        make_float2(half_sc, half_sc), make_float2(hb, hb)),
+                             make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), gp, gd);
+                  p = e ? gp.y : gp.x;
+                  ds = e ? gd.y : gd.x;
+                } else if constexpr (PHI == GDPA_PHI_RELU) {
+                  const float u = fmaf(x, sc, b1k);
+                  p = relu_f(u);
+                  ds = g * relu_grad(u);
+                } else if constexpr (PHI == GDPA_PHI_GELU) {
+                  if (e == 0)           // both columns of the pair, in packed arithmetic
+                    gelu_fg2(__ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                        make_float2(sc, sc), make_float2(b1k, b1k)),
+                             gp, gd);
+                  p = e ? gp.y : gp.x;
+                  ds = g * (e ? gd.y : gd.x);
+                } else {
+                  p = fmaf(x, sc, b1k);
+                  ds = g;
                 }
-                p = e ? gp.y : gp.x;
-                ds = e ? gd.y : gd.x;
-              } else if constexpr (PHI == GDPA_PHI_SILU) {
-                if (e == 0)           // both columns of the pair, in packed arithmetic
-                  silu_fg2(__ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
-                                      make_float2(half_sc, half_sc), make_float2(hb, hb)),
-                           make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), gp, gd);
-                p = e ? gp.y : gp.x;
-                ds = e ? gd.y : gd.x;
-              } else if constexpr (PHI == GDPA_PHI_RELU) {
-                const float u = fmaf(x, sc, b1k);
-                p = relu_f(u);
-                ds = g * relu_grad(u);
-              } else if constexpr (PHI == GDPA_PHI_GELU) {
-                if (e == 0)           // both columns of the pair, in packed arithmetic
-                  gelu_fg2(__ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
-                                      make_float2(sc, sc), make_float2(b1k, b1k)),
-                           gp, gd);
-                p = e ? gp.y : gp.x;
-                ds = g * (e ? gd.y : gd.x);
-              } else {
-                p = fmaf(x, sc, b1k);
-                ds = g;
+                // softmax rows past the sample already give P = dS = 0 (-LSE = -inf)
+                const bool valid = SOFTMAX || FULL || rbase + r < n;
+                pv[e] = valid ? p : 0.f;
+                dv2[e] = valid ? ds : 0.f;
+                if constexpr (BIAS) db1_acc += dv2[e];
               }
-              // softmax rows past the sample already give P = dS = 0 (-LSE = -inf)
-              const bool valid = SOFTMAX || rbase + r < n;
-              pv[e] = valid ? p : 0.f;
-              dv2[e] = valid ? ds : 0.f;
-              if constexpr (BIAS) db1_acc += dv2[e];
+              pp[c / 2] = pack_bf16x2(pv[0], pv[1]);
+              dd[c / 2] = pack_bf16x2(dv2[0], dv2[1]);
             }
-            pp[c / 2] = pack_bf16x2(pv[0], pv[1]);
-            dd[c / 2] = pack_bf16x2(dv2[0], dv2[1]);
-          }
-          tmem_st_x16(tmem + lane_off + C::COL_S + 64 * grp + 16 * ch, pp);
-          // dS^T line `lrow` of chunk `grp`, 16-byte pieces 4ch..4ch+3, 128B swizzle
-          const uint32_t line = sDS + grp * 16384 + lrow * 128;
+            tmem_st_x16(tmem + lane_off + C::COL_S + 64 * grp + 16 * ch, pp);
+            // dS^T line `lrow` of chunk `grp`, 16-byte pieces 4ch..4ch+3, 128B swizzle
+            const uint32_t line = sDS + grp * 16384 + lrow * 128;
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            const uint32_t j = 4 * ch + jj;
-            const uint32_t addr = line + ((j ^ (uint32_t)(lrow & 7)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dd[4 * jj]),
-                         "r"(dd[4 * jj + 1]), "r"(dd[4 * jj + 2]), "r"(dd[4 * jj + 3])
-                         : "memory");
+            for (int jj = 0; jj < 4; ++jj) {
+              const uint32_t j = 4 * ch + jj;
+              const uint32_t addr = line + ((j ^ (uint32_t)(lrow & 7)) << 4);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dd[4 * jj]),
+                           "r"(dd[4 * jj + 1]), "r"(dd[4 * jj + 2]), "r"(dd[4 * jj + 3])
+                           : "memory");
+            }
           }
-        }
+        };
+        if (SOFTMAX || rbase + 64 <= n)
+          half_body(std::true_type{});
+        else
+          half_body(std::false_type{});
         tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
