@@ -59,11 +59,11 @@ KERNEL_SOURCES = {"gdpa_fwd_sm100": ("fwd_sm100.cu", "sm100.cuh", "gdpa_internal
 # sha16 of the kernel's sources at capture time)}}.  An entry whose hash no
 # longer matches the sources is not used (the traffic is then reported null).
 TRAFFIC_PER_UNIT = {
-    # 64-sample cases: workload 5, 582.3 MB read + 35.9 MB written in one launch;
-    # workload 4, 347.2 MB + 61.8 MB
-    "gdpa_fwd_sm100": {5: (0.0141402, "209e3f60a671ea6a"), 4: (0.0101671, "209e3f60a671ea6a")},
-    # workload 5: 732.7 MB read + 578.8 MB written; workload 4: 599.3 MB + 379.6 MB
-    "gdpa_bwd_sm100": {5: (0.0299974, "7603f7174c81c773"), 4: (0.0243348, "7603f7174c81c773")},
+    # 64-sample cases: workload 5, 582.2 MB read + 36.3 MB written in one launch;
+    # workload 4, 347.3 MB + 60.0 MB
+    "gdpa_fwd_sm100": {5: (0.0141478, "209e3f60a671ea6a"), 4: (0.0101234, "209e3f60a671ea6a")},
+    # workload 5: 734.8 MB read + 581.8 MB written; workload 4: 599.3 MB + 380.3 MB
+    "gdpa_bwd_sm100": {5: (0.0301167, "2fe31e59c24fa0ae"), 4: (0.0243502, "2fe31e59c24fa0ae")},
 }
 # fp32 FFMA peak for the SIMT kernels: 148 SMs * 128 FMA/clk * 2 flop * 1.965 GHz
 SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12

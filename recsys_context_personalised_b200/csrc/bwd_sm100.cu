@@ -553,9 +553,16 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                   p = e ? gp.y : gp.x;
                   ds = e ? gd.y : gd.x;
                 } else if constexpr (PHI == GDPA_PHI_RELU) {
-                  const float u = fmaf(x, sc, b1k);
-                  p = relu_f(u);
-                  ds = g * relu_grad(u);
+                  if (e == 0) {         // both columns of the pair, in packed arithmetic
+                    const float2 u = __ffma2_rn(
+                        make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                        make_float2(sc, sc), make_float2(b1k, b1k));
+                    gp = make_float2(relu_f(u.x), relu_f(u.y));
+                    gd = __fmul2_rn(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])),
+                                    make_float2(relu_grad(u.x), relu_grad(u.y)));
+                  }
+                  p = e ? gp.y : gp.x;
+                  ds = e ? gd.y : gd.x;
                 } else if constexpr (PHI == GDPA_PHI_GELU) {
                   if (e == 0)           // both columns of the pair, in packed arithmetic
                     gelu_fg2(__ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
@@ -564,7 +571,10 @@ gdpa_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                   p = e ? gp.y : gp.x;
                   ds = g * (e ? gd.y : gd.x);
                 } else {
-                  p = fmaf(x, sc, b1k);
+                  if (e == 0)           // both columns of the pair, in packed arithmetic
+                    gp = __ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                    make_float2(sc, sc), make_float2(b1k, b1k));
+                  p = e ? gp.y : gp.x;
                   ds = g;
                 }
                 // softmax rows past the sample already give P = dS = 0 (-LSE = -inf)
@@ -1208,9 +1218,16 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                     p = e ? gp.y : gp.x;
                     ds = e ? gd.y : gd.x;
                   } else if constexpr (PHI == GDPA_PHI_RELU) {
-                    const float u = fmaf(x, sc, b1k);
-                    p = relu_f(u);
-                    ds = g * relu_grad(u);
+                    if (e == 0) {         // both columns of the pair, in packed arithmetic
+                      const float2 u = __ffma2_rn(
+                          make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                          make_float2(sc, sc), make_float2(b1k, b1k));
+                      gp = make_float2(relu_f(u.x), relu_f(u.y));
+                      gd = __fmul2_rn(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])),
+                                      make_float2(relu_grad(u.x), relu_grad(u.y)));
+                    }
+                    p = e ? gp.y : gp.x;
+                    ds = e ? gd.y : gd.x;
                   } else if constexpr (PHI == GDPA_PHI_GELU) {
                     if (e == 0)           // both columns of the pair, in packed arithmetic
                       gelu_fg2(__ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
@@ -1219,7 +1236,10 @@ gdpa_bwd_half_kernel(const __grid_constant__ CUtensorMap tmQ,
                     p = e ? gp.y : gp.x;
                     ds = g * (e ? gd.y : gd.x);
                   } else {
-                    p = fmaf(x, sc, b1k);
+                    if (e == 0)           // both columns of the pair, in packed arithmetic
+                      gp = __ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                      make_float2(sc, sc), make_float2(b1k, b1k));
+                    p = e ? gp.y : gp.x;
                     ds = g;
                   }
                   // softmax: rows past the sample (-LSE = -inf), keys past it and
